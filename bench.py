@@ -1,0 +1,487 @@
+#!/usr/bin/env python
+"""Benchmark of the paged decode hot path on B200.
+
+One step = one decode step of one attention layer over a batch:
+  copy-on-write block copies (when the step has any) -> cache append of one
+  new token per sequence -> paged decode (or verify) attention over the
+  grown contexts (+ the split-context merge).
+Host bookkeeping (slot reservation) for every step is done before timing;
+the e2e figure repeats the steps through the public API with host buffers.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                       [--impl ours|reference]
+Multi-GPU (weak scaling, independent replicas, no data-path collective):
+  torchrun --nproc-per-node N bench.py --gpus N ...
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention KV GB/s and % of B200 HBM peak; tokens·heads/s"
+DEFAULT_WORKLOAD = "llama7b_mha"
+FALLBACK_HBM_GBS = 6650.0
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank runs its own replica of the workload (weak scaling)."""
+    return base_seed + 7919 * rank
+
+
+def algorithmic_bytes(lens, Hq, Hkv, D, bs, q_len):
+    """(K/V bytes read, all bytes) of one attention launch: K and V rows of
+    every visible token, q and out, the used table entries and the lengths."""
+    L = [int(x) for x in lens]
+    kv = sum(L) * Hkv * D * 2 * 2
+    qo = len(L) * q_len * Hq * D * 2 * 2
+    tab = sum(-(-x // bs) for x in L) * 4 + len(L) * 4
+    return kv, kv + qo + tab
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for name in ("paged_attention.cu", "kv_ptx.cuh"):
+        with open(os.path.join(ROOT, "paged_kv_cache_371_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload):
+    """DRAM bytes per launch of the attention kernel from a committed ncu
+    summary, if it was taken on the current kernel source (else None)."""
+    sha = kernel_source_sha()
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        kv = {}
+        with open(path, encoding="utf-8") as f:
+            for line in f:
+                if ":" in line and line.startswith("- "):
+                    k, v = line[2:].split(":", 1)
+                    kv[k.strip()] = v.strip().strip("`")
+        if (kv.get("workload") == workload and kv.get("kernel_source_sha256") == sha
+                and "traffic_bytes_per_launch" in kv):
+            try:
+                return int(float(kv["traffic_bytes_per_launch"]))
+            except ValueError:
+                return None
+    return None
+
+
+class ClockSampler:
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.gpu = gpu_index
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={CLOCK_QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+
+def adopt_workload(pkv, wl, extra_cap):
+    """Host block manager in the state the generator's placement describes:
+    the same ids, allocated in the same order (prefix blocks forked)."""
+    import numpy as np
+    bs = wl.spec.bs
+    B = wl.B
+    cap = wl.block_tables.shape[1] + extra_cap
+    pool = pkv.KVPool(wl.num_blocks, bs, num_kv_heads=wl.spec.Hkv, head_dim=wl.q.shape[-1],
+                      order=wl.order)
+    tables = np.full((B, cap), -1, np.int32)
+    nblk = np.zeros(B, np.int32)
+    P = wl.extra.get("prefix_blocks", 0)
+    prefix = pool.alloc(P) if P else []
+    for s in range(B):
+        need = int(-(-int(wl.lens[s]) // bs))
+        if P:
+            if s:
+                pool.fork(prefix)
+            tables[s, :P] = prefix
+        ids = pool.alloc(need - P)
+        tables[s, P:need] = ids
+        nblk[s] = need
+        assert tables[s, :need].tolist() == wl.block_tables[s, :need].tolist()
+    return pool, tables, nblk
+
+
+def build_steps(pkv, wl, n_steps, device, seed):
+    """Per-step inputs: slots / copy pairs from the host block manager, new
+    K/V, queries, tables and lengths after the append."""
+    import numpy as np
+    import torch
+    from workloads import normal_fp16
+    bs = wl.spec.bs
+    Hq, Hkv, D = wl.q.shape[-2], wl.spec.Hkv, wl.q.shape[-1]
+    q_len = wl.q.shape[1]
+    pool, tables, nblk = adopt_workload(pkv, wl, extra_cap=n_steps // bs + 2)
+    lens = wl.lens.astype(np.int32).copy()
+    steps = []
+    for i in range(n_steps):
+        slots, pairs = pool.reserve_slots(tables, nblk, lens)
+        lens = lens + 1
+        st = {
+            "q": normal_fp16((wl.B, q_len, Hq, D), seed * 100003 + 3 * i, device),
+            "k_new": normal_fp16((wl.B, Hkv, D), seed * 100003 + 3 * i + 1, device),
+            "v_new": normal_fp16((wl.B, Hkv, D), seed * 100003 + 3 * i + 2, device),
+            "slots": torch.as_tensor(slots, device=device),
+            "pairs": torch.as_tensor(pairs, device=device) if len(pairs) else None,
+            "tables": torch.as_tensor(tables.copy(), device=device),
+            "lens": torch.as_tensor(lens.copy(), device=device),
+            "lens_host": lens.copy(),
+        }
+        steps.append(st)
+    return steps
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_371_b200 as pkv
+    from workloads import make_workload
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+
+    from workloads.synth import CONFIGS
+    spec = CONFIGS[args.workload]
+    seed = rank_seed(spec.seed, rank)
+    wl = make_workload(args.workload, device, seed=seed)
+    q_len = spec.q_len
+    Hq, Hkv, D, bs = spec.Hq, spec.Hkv, spec.D, spec.bs
+    n_distinct = min(args.warmup + args.steps, 64)
+    steps = build_steps(pkv, wl, n_distinct, device, seed)
+    out = torch.empty((wl.B, q_len, Hq, D), dtype=torch.float16, device=device)
+    ws = torch.empty(pkv.workspace_size(Hq, Hkv, q_len, D), dtype=torch.uint8, device=device)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(i, ev=None):
+        st = steps[i % n_distinct]
+        if st["pairs"] is not None:
+            pkv.paged_kv_copy_blocks(wl.k_pool, wl.v_pool, st["pairs"])
+        pkv.paged_kv_append(st["k_new"], st["v_new"], st["slots"], wl.k_pool, wl.v_pool)
+        if ev is not None:
+            ev.record(stream)
+        if q_len == 1:
+            pkv.paged_decode_attention(st["q"], wl.k_pool, wl.v_pool, st["tables"], st["lens"],
+                                       wl.scale, out=out, workspace=ws)
+        else:
+            pkv.paged_verify_attention(st["q"], wl.k_pool, wl.v_pool, st["tables"], st["lens"],
+                                       wl.scale, q_len, out=out, workspace=ws)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert pkv.device_error() == 0, "device error during warm-up"
+
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    launches = 0
+    kv_bytes_total = 0
+    alg_attn = []
+    th_tokens = 0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    phys = vis.split(",")[local] if vis and len(vis.split(",")) > local else str(local)
+    with ClockSampler(phys) as clk:
+        for k in range(args.steps):
+            i = args.warmup + k
+            st = steps[i % n_distinct]
+            flush.zero_()
+            ev_s[k].record(stream)
+            step(i, ev_a[k])
+            ev_e[k].record(stream)
+            launches += 3 + (1 if st["pairs"] is not None else 0)
+            kvb, allb = algorithmic_bytes(st["lens_host"], Hq, Hkv, D, bs, q_len)
+            kv_bytes_total += kvb
+            alg_attn.append(allb)
+            th_tokens += int(st["lens_host"].sum()) * Hq * q_len
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = [ev_s[k].elapsed_time(ev_e[k]) for k in range(args.steps)]
+    attn_ms = [ev_a[k].elapsed_time(ev_e[k]) for k in range(args.steps)]
+    err = pkv.device_error()
+    assert err == 0, f"device error word {err}"
+    total_ms = sum(step_ms)
+
+    # whole-job aggregate: bytes of all ranks / slowest rank's time
+    tot = torch.tensor([kv_bytes_total, th_tokens], dtype=torch.float64, device=device)
+    tmax = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+    kv_all, th_all = tot.tolist()
+    t_all = tmax.item()
+    value = kv_all / (t_all * 1e-3) / 1e9
+
+    # e2e: same steps through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(pkv, wl, steps, n_distinct, args, out, ws, flush, stream, device, Hq, Hkv, D,
+                      bs, q_len, world)
+
+    peak, peak_kind = measured_hbm_peak()
+    attn_avg_ms = statistics.mean(attn_ms)
+    achieved = statistics.mean(alg_attn) / (attn_avg_ms * 1e-3) / 1e9
+    result = None
+    if rank == 0:
+        result = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(t_all / args.steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {
+                "workload": args.workload, "description": spec.description, "B": wl.B,
+                "Hq": Hq, "Hkv": Hkv, "head_dim": D, "block_size": bs, "q_len": q_len,
+                "mean_context": float(np.mean(wl.lens)),
+                "step": "copy-on-write copies + append 1 token/sequence + paged attention + merge",
+                "l2": "flushed before every timed step (memset of 2x L2)",
+                "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "hbm_frac": round(value / peak, 4),
+            "hbm_peak_gbs": peak, "hbm_peak_kind": peak_kind,
+            "tokens_heads_per_s": round(th_all / (t_all * 1e-3), 1),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": ncu_traffic(args.workload),
+                         "kernel": "paged_attention_kernel + lse_merge_kernel",
+                         "peak_kind": peak_kind},
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+        }
+        if e2e:
+            result["e2e"] = e2e
+        if world == 1:
+            result["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
+    if world > 1:
+        dist.destroy_process_group()
+    return result
+
+
+def run_e2e(pkv, wl, steps, n_distinct, args, out, ws, flush, stream, device, Hq, Hkv, D, bs, q_len,
+            world):
+    import torch
+    import torch.distributed as dist
+    host = []
+    for st in steps:
+        h = {k: st[k].cpu().pin_memory() for k in ("q", "k_new", "v_new", "slots", "tables", "lens")}
+        h["pairs"] = st["pairs"].cpu().pin_memory() if st["pairs"] is not None else None
+        host.append(h)
+    dev = {k: torch.empty_like(steps[0][k]) for k in ("q", "k_new", "v_new", "slots", "lens")}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = 0
+    d2h = out.numel() * out.element_size()
+    times = []
+    kvb_total = 0
+    tables = torch.empty(host[0]["tables"].shape, dtype=torch.int32, device=device)
+    for k in range(args.warmup + args.steps):
+        h = host[k % n_distinct]
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        nbytes = 0
+        for name in ("q", "k_new", "v_new", "slots", "lens"):
+            dev[name].copy_(h[name], non_blocking=True)
+            nbytes += h[name].numel() * h[name].element_size()
+        tables.copy_(h["tables"], non_blocking=True)
+        nbytes += h["tables"].numel() * 4
+        if h["pairs"] is not None:
+            pairs = h["pairs"].to(device, non_blocking=True)
+            nbytes += h["pairs"].numel() * 4
+            pkv.paged_kv_copy_blocks(wl.k_pool, wl.v_pool, pairs)
+        pkv.paged_kv_append(dev["k_new"], dev["v_new"], dev["slots"], wl.k_pool, wl.v_pool)
+        if q_len == 1:
+            pkv.paged_decode_attention(dev["q"], wl.k_pool, wl.v_pool, tables, dev["lens"],
+                                       wl.scale, out=out, workspace=ws)
+        else:
+            pkv.paged_verify_attention(dev["q"], wl.k_pool, wl.v_pool, tables, dev["lens"],
+                                       wl.scale, q_len, out=out, workspace=ws)
+        out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if k >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+            kvb_total += algorithmic_bytes(steps[k % n_distinct]["lens_host"], Hq, Hkv, D, bs,
+                                           q_len)[0]
+            h2d = nbytes
+    t = torch.tensor([sum(times)], dtype=torch.float64, device=device)
+    kv = torch.tensor([float(kvb_total)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(kv, op=dist.ReduceOp.SUM)
+    return {"value": round(kv.item() / (t.item() * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": round(t.item() / args.steps, 5)}
+
+
+# ---------------------------------------------------------------------------
+# oracle timing (CPU baseline and the reference arm)
+
+def oracle_sample(workload, target_s, seed_offset=0):
+    """A bounded sample of the workload (fewer sequences, same recipe) sized so
+    one oracle call takes about target_s seconds on this host."""
+    import oracle
+    from workloads import make_workload
+    from workloads.synth import CONFIGS
+    spec = CONFIGS[workload]
+    probe = make_workload(workload, "cpu", B=1, seed=spec.seed + seed_offset)
+    t0 = time.perf_counter()
+    oracle.paged_attention(probe.q.numpy(), probe.k_pool.numpy(), probe.v_pool.numpy(),
+                           probe.block_tables, probe.lens, scale=probe.scale, q_len=spec.q_len)
+    t1 = max(time.perf_counter() - t0, 1e-4)
+    n = int(max(1, min(max(1, spec.B // 4), round(target_s / t1))))
+    return make_workload(workload, "cpu", B=n, seed=spec.seed + seed_offset)
+
+
+def time_oracle(wl):
+    import oracle
+    q, k, v = wl.q.numpy(), wl.k_pool.numpy(), wl.v_pool.numpy()
+    t0 = time.perf_counter()
+    oracle.paged_attention(q, k, v, wl.block_tables, wl.lens, scale=wl.scale, q_len=wl.q.shape[1])
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(workload, target_s):
+    import oracle
+    wl = oracle_sample(workload, target_s)
+    dt = time_oracle(wl)
+    s = wl.spec
+    kvb = algorithmic_bytes(wl.lens, s.Hq, s.Hkv, s.D, s.bs, s.q_len)[0]
+    return {"value": round(kvb / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{wl.B} of {s.B} sequences of {workload} (same length recipe), "
+                      f"{int(wl.lens.sum())} tokens, fp64 C oracle, {dt:.2f} s"}
+
+
+def run_reference(args):
+    import oracle
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    from workloads.synth import CONFIGS
+    spec = CONFIGS[args.workload]
+    per_step = max(0.2, min(2.0, 120.0 / max(1, args.steps + args.warmup)))
+    wl = oracle_sample(args.workload, per_step)
+    for _ in range(args.warmup):
+        time_oracle(wl)
+    times = [time_oracle(wl) for _ in range(args.steps)]
+    kvb = algorithmic_bytes(wl.lens, spec.Hq, spec.Hkv, spec.D, spec.bs, spec.q_len)[0]
+    total = sum(times)
+    value = kvb * args.steps / total / 1e9
+    sample = (f"{wl.B} of {spec.B} sequences of {args.workload} per step (same length recipe), "
+              f"{int(wl.lens.sum())} tokens, fp64 C oracle")
+    return {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": args.workload, "description": spec.description},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "kind": "oracle",
+                             "cores": oracle.num_threads(), "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    res = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

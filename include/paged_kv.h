@@ -1,0 +1,221 @@
+/*
+ * paged_kv.h — C ABI of the B200 (sm_100a) paged KV-cache library.
+ *
+ * The operation follows four web pages on LLM inference (cited by title and
+ * section):
+ *   [T1] "LLM推理优化实战：从KV Cache到Speculative Decoding，把延迟打下来"
+ *   [T2] "大模型推理加速：从 KV Cache 到投机采样的工程实践"
+ *   [T3] "LLM 推理优化：KV Cache、PagedAttention 与量化"
+ *   [T4] "大模型推理加速与显存黑科技 (Inference Acceleration & KV Cache)"
+ *
+ * Data layout (the pages fix none; all device arrays are row-major, dense):
+ *   k_pool, v_pool  fp16 [num_blocks][Hkv][block_size][head_dim]
+ *                   (one (block, kv-head) tile is block_size*head_dim*2
+ *                   contiguous bytes; base 16-byte aligned, head_dim*2 a
+ *                   multiple of 16)
+ *   block_tables    int32 [B][max_blocks_per_seq]; entry b of row s is the
+ *                   physical block holding tokens [b*bs, b*bs+bs) of sequence s
+ *   context_lens    int32 [B]; tokens of sequence s already in the cache
+ *                   (including any token appended this step)
+ *   q, out          fp16 [B][q_len][Hq][head_dim]  (q_len = 1 for decode)
+ *   k_new, v_new    fp16 [T][Hkv][head_dim]
+ *   slot_mapping    int64 [T]; slot = physical_block*block_size + offset,
+ *                   negative = padding (skipped)
+ * Query head h reads KV head h / (Hq / Hkv) (contiguous GQA groups).
+ *
+ * Ownership: the caller allocates and owns every device buffer (pools, q,
+ * out, tables, lengths, workspace) and every host array it passes.  The
+ * library owns only the host bookkeeping behind an opaque kv_pool*.  Device
+ * calls are asynchronous on the caller's stream (a cudaStream_t passed as
+ * void*; NULL = legacy default stream); they never allocate device memory.
+ *
+ * Errors: every call returns a status.  On KV_ERR_INVALID nothing was
+ * launched or changed; KV_ERR_CUDA means a CUDA call failed (text in
+ * kv_last_error_string()).  Kernels never trap: an out-of-range block id or
+ * slot met on the device is skipped and recorded in a per-device error word
+ * read by kv_device_error().
+ */
+#ifndef PAGED_KV_H
+#define PAGED_KV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KV_OK 0
+#define KV_ERR_INVALID 1     /* bad argument, shape, id or state */
+#define KV_ERR_OOM 2         /* pool exhausted: the pages' preemption trigger */
+#define KV_ERR_DOUBLE_FREE 3 /* a free would take a refcount below zero */
+#define KV_ERR_CUDA 4        /* a CUDA runtime call failed */
+#define KV_ERR_TIMEOUT 5     /* unused by the host; device-word bit, see below */
+
+/* Bits of the device error word. */
+#define KV_DEV_BAD_BLOCK 1   /* a block-table entry outside [0, num_blocks) */
+#define KV_DEV_BAD_SLOT 2    /* an append slot beyond the pool */
+#define KV_DEV_TIMEOUT 4     /* a pipeline wait ran past its limit */
+
+/* Text of the last error raised on the calling thread ("" if none). */
+const char* kv_last_error_string(void);
+
+/* Library version, for the binding's load check. */
+int kv_version(void);
+
+/* ---------------------------------------------------------------------------
+ * Pool configuration and sizing.
+ * [T2] §"KV Cache的内存挑战" and [T4] §2.1: KV bytes =
+ * 2 x layers x heads x head_dim x seq_len x batch x dtype_size.  For a pool,
+ * seq_len x batch is its capacity num_blocks x block_size tokens and heads are
+ * the KV heads (under MQA/GQA only KV heads are cached, [T2] §"主流优化策略").
+ */
+typedef struct kv_pool_config {
+    int32_t num_blocks;   /* physical blocks in the pool, > 0 */
+    int32_t block_size;   /* tokens per block: 16 (default) or 8 ([T3] §2.2) */
+    int32_t num_kv_heads; /* Hkv */
+    int32_t head_dim;     /* D: 64 or 128 on the decode path */
+    int32_t num_layers;   /* layers sharing one block table (sizing only) */
+    int32_t dtype_bytes;  /* 2 (fp16) */
+} kv_pool_config;
+
+/* per_layer_bytes = K+V bytes of one layer's pools; total_bytes = per layer x
+ * num_layers.  Either output may be NULL. */
+int kv_pool_bytes(const kv_pool_config* cfg, uint64_t* per_layer_bytes, uint64_t* total_bytes);
+
+/* ---------------------------------------------------------------------------
+ * Host block manager ([T3] §2.3 (1)-(3)): fixed-capacity pool, on-demand
+ * allocation, immediate reuse of freed blocks, per-block reference counts,
+ * block-level copy-on-write, prefix sharing by pointing several tables at the
+ * same blocks.  Policy (fixed so results are bit-exact and testable):
+ *   - the free list is a LIFO stack; it first pops ids in ascending order, or
+ *     in the order of `order` (a permutation of 0..num_blocks-1) if given;
+ *     freed blocks are pushed on top and reused first;
+ *   - block_alloc is all-or-nothing (KV_ERR_OOM and no change on shortage);
+ *   - block_free drops one reference per listed id, pushing ids whose count
+ *     reaches zero in list order; KV_ERR_DOUBLE_FREE (no change) if any count
+ *     would go below zero;
+ *   - block_fork adds one reference per listed (live) id.
+ * A kv_pool is not thread-safe; use one per thread or lock around it.
+ */
+typedef struct kv_pool kv_pool;
+
+int kv_pool_create(const kv_pool_config* cfg, const int32_t* order /* nullable */,
+                   kv_pool** out);
+int kv_pool_destroy(kv_pool* pool);
+int kv_pool_num_free(const kv_pool* pool, int32_t* n_out);
+int block_alloc(kv_pool* pool, int32_t n, int32_t* ids_out /* [n] */);
+int block_free(kv_pool* pool, const int32_t* ids, int32_t n);
+int block_fork(kv_pool* pool, const int32_t* ids, int32_t n);
+int block_refcount(const kv_pool* pool, int32_t id, int32_t* rc_out);
+
+/* Reserve the cache slot of token number ctx_len (0-based) of one sequence
+ * whose table holds *n_blocks == ceil(ctx_len / block_size) entries
+ * ([T3] §2.3 (1) on-demand allocation, (2) copy-on-write):
+ *   - ctx_len % block_size == 0: a new block is allocated and appended;
+ *   - the last block is shared (refcount > 1): a new block replaces it in the
+ *     table, one reference to the old block is dropped and (*cow_src_out,
+ *     *cow_dst_out) = (old, new): the caller must copy that block on the
+ *     device (paged_kv_copy_blocks) before appending;
+ *   - otherwise the token goes into the last block.
+ * cow_* are -1 when no copy is needed.  table_capacity bounds the table. */
+int kv_seq_reserve_slot(kv_pool* pool, int32_t* table, int32_t table_capacity,
+                        int32_t* n_blocks, int32_t ctx_len, int64_t* slot_out,
+                        int32_t* cow_src_out, int32_t* cow_dst_out);
+
+/* The same for B sequences in order (table row s = tables + s*table_capacity).
+ * Copy pairs are written as (src, dst) into cow_pairs_out[2*k], [2*k+1] and
+ * counted in *n_cow_out.  On an error at sequence i the earlier sequences keep
+ * their reservations, *n_done_out = i and the error is returned. */
+int kv_batch_reserve_slots(kv_pool* pool, int32_t B, int32_t* tables, int32_t table_capacity,
+                           int32_t* n_blocks /* [B] */, const int32_t* ctx_lens /* [B] */,
+                           int64_t* slots_out /* [B] */, int32_t* cow_pairs_out /* [2B] */,
+                           int32_t* n_cow_out, int32_t* n_done_out);
+
+/* ---------------------------------------------------------------------------
+ * Device calls.
+ */
+
+/* Cache append: for each t with slot_mapping[t] >= 0,
+ *   k_pool[slot/bs][h][slot%bs][:] = k_new[t][h][:]  (and V), every h.
+ * Bit-exact copy.  Slots >= num_blocks*bs are skipped and flag
+ * KV_DEV_BAD_SLOT.  Distinct tokens must target distinct slots. */
+int paged_kv_append(const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                    void* k_pool, void* v_pool, int32_t T, int32_t Hkv, int32_t head_dim,
+                    int32_t block_size, int32_t num_blocks, void* stream);
+
+/* Copy-on-write block copy ([T3] §2.3 (2)): for each i, physical block
+ * pairs[2i+1] of both pools becomes a copy of block pairs[2i] (all heads and
+ * slots).  pairs is a DEVICE int32 array [n][2]; destinations must be
+ * distinct and no destination may also be a source.  Out-of-range ids are
+ * skipped and flag KV_DEV_BAD_BLOCK. */
+int paged_kv_copy_blocks(void* k_pool, void* v_pool, const int32_t* pairs, int32_t n,
+                         int32_t Hkv, int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                         void* stream);
+
+/* Bytes of device workspace paged_decode_attention / paged_verify_attention
+ * need for these head counts on the current device (partial results of
+ * context splits).  grid_ctas: 0 for the default launch, else the value given
+ * in paged_attention_opts.grid_ctas.  The workspace holds no state between
+ * calls and needs no initialisation. */
+int paged_attention_workspace_size(int32_t Hq, int32_t Hkv, int32_t q_len, int32_t head_dim,
+                                   int32_t grid_ctas, size_t* bytes_out);
+
+/* Paged decode attention ([T4] §2, Attention(Q,K,V) = softmax(QK^T/sqrt(d_k))V;
+ * paging per [T3] §2.2 and [T4] §3.2; tiling with an online softmax per
+ * [T4] §4.2): for every sequence s and query head h,
+ *   out[s][0][h] = softmax(scale * q[s][0][h] . K_t) V_t over t < context_lens[s],
+ * K_t / V_t gathered from the pools through block_tables[s][t / bs], row t % bs.
+ * fp16 in, fp32 accumulation, fp16 (round-to-nearest-even) out; a sequence of
+ * length 0 gives zeros.  Long contexts are split across CTAs and merged by
+ * log-sum-exp on the device.  Requirements: head_dim in {64, 128},
+ * block_size in {8, 16}, Hq % Hkv == 0, (Hq/Hkv)*q_len <= 32; workspace of at
+ * least paged_attention_workspace_size() bytes, 16-byte aligned. */
+int paged_decode_attention(const void* q, const void* k_pool, const void* v_pool,
+                           const int32_t* block_tables, int32_t max_blocks_per_seq,
+                           const int32_t* context_lens, float scale, void* out, int32_t B,
+                           int32_t Hq, int32_t Hkv, int32_t head_dim, int32_t block_size,
+                           int32_t num_blocks, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/* Causal verify window for speculative decoding ([T1] §"Speculative
+ * Decoding：用草稿模型加速": the target scores prompt + drafts in one pass;
+ * [T3] §6.2): q holds q_len rows per sequence, context_lens counts the drafts,
+ * and row j attends to tokens 0 .. context_lens[s] - q_len + j.  q_len = 1 is
+ * paged_decode_attention. */
+int paged_verify_attention(const void* q, const void* k_pool, const void* v_pool,
+                           const int32_t* block_tables, int32_t max_blocks_per_seq,
+                           const int32_t* context_lens, int32_t q_len, float scale, void* out,
+                           int32_t B, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                           int32_t block_size, int32_t num_blocks, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* Launch knobs for tuning and tests; zero fields mean "default".
+ *   grid_ctas        persistent CTAs (default: SMs x CTAs per SM);
+ *   min_split_blocks smallest run of blocks one CTA takes (default 16), lower
+ *                    values force more context splits (and merges);
+ *   use_pdl          1: launch the merge with programmatic dependent launch
+ *                    (default), -1: plain launch. */
+typedef struct paged_attention_opts {
+    int32_t grid_ctas;
+    int32_t min_split_blocks;
+    int32_t use_pdl;
+    int32_t reserved[5];
+} paged_attention_opts;
+
+int paged_attention_ex(const void* q, const void* k_pool, const void* v_pool,
+                       const int32_t* block_tables, int32_t max_blocks_per_seq,
+                       const int32_t* context_lens, int32_t q_len, float scale, void* out,
+                       int32_t B, int32_t Hq, int32_t Hkv, int32_t head_dim, int32_t block_size,
+                       int32_t num_blocks, void* workspace, size_t workspace_bytes,
+                       const paged_attention_opts* opts, void* stream);
+
+/* Read the current device's error word (bits KV_DEV_*) after synchronizing
+ * `stream`; reset != 0 clears it. */
+int kv_device_error(int32_t* word_out, int32_t reset, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_KV_H */

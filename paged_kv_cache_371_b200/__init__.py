@@ -1,0 +1,252 @@
+"""B200 (sm_100a) paged KV cache: PagedAttention decode, cache append, CoW.
+
+A thin binding over the C ABI of ``libpaged_kv.so`` (include/paged_kv.h):
+argument checks and marshalling only; every step runs in the library's CUDA
+kernels or its C++ host bookkeeping.  PyTorch supplies device memory and
+streams.  Importing this package fails loudly if the library is not built.
+
+Layouts: pools fp16 [num_blocks][Hkv][block_size][D]; q / out fp16
+[B][q_len][Hq][D] ([B][Hq][D] accepted for decode); block_tables int32
+[B][max_blocks]; context_lens int32 [B]; slot_mapping int64 [T].
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+from . import _abi
+from ._abi import KVError, check
+
+__all__ = ["KVPool", "KVError", "pool_bytes", "paged_kv_append", "paged_kv_copy_blocks",
+           "workspace_size", "paged_decode_attention", "paged_verify_attention",
+           "paged_attention", "device_error", "lib"]
+
+_L = _abi.load()
+
+
+def lib() -> ctypes.CDLL:
+    return _L
+
+
+def _stream(device: torch.device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, device=None) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def _i32p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+# ---------------------------------------------------------------------------
+# sizing and host bookkeeping
+
+def _cfg(num_blocks, block_size, num_kv_heads, head_dim, num_layers=1, dtype_bytes=2):
+    return _abi.KvPoolConfig(num_blocks, block_size, num_kv_heads, head_dim, num_layers,
+                             dtype_bytes)
+
+
+def pool_bytes(num_blocks, block_size, num_kv_heads, head_dim, num_layers=1, dtype_bytes=2):
+    """(per-layer K+V bytes, total bytes) of a pool."""
+    per, tot = ctypes.c_uint64(), ctypes.c_uint64()
+    c = _cfg(num_blocks, block_size, num_kv_heads, head_dim, num_layers, dtype_bytes)
+    check(_L.kv_pool_bytes(ctypes.byref(c), ctypes.byref(per), ctypes.byref(tot)), "kv_pool_bytes")
+    return per.value, tot.value
+
+
+class KVPool:
+    """Refcounted block pool with copy-on-write (host bookkeeping, C++)."""
+
+    def __init__(self, num_blocks: int, block_size: int, num_kv_heads: int = 1, head_dim: int = 128,
+                 num_layers: int = 1, order: Optional[Sequence[int]] = None):
+        c = _cfg(num_blocks, block_size, num_kv_heads, head_dim, num_layers)
+        h = ctypes.c_void_p()
+        arr = None
+        if order is not None:
+            arr = np.ascontiguousarray(order, dtype=np.int32)
+            if arr.shape != (num_blocks,):
+                raise ValueError("order must list every block once")
+        check(_L.kv_pool_create(ctypes.byref(c), _i32p(arr) if arr is not None else None,
+                                ctypes.byref(h)), "kv_pool_create")
+        self._h = h
+        self._lib = _L  # kept so close() still works during interpreter shutdown
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.kv_pool_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+    def num_free(self) -> int:
+        n = ctypes.c_int32()
+        check(_L.kv_pool_num_free(self._h, ctypes.byref(n)), "kv_pool_num_free")
+        return n.value
+
+    def alloc(self, n: int) -> list:
+        ids = np.zeros(max(n, 1), np.int32)
+        check(_L.block_alloc(self._h, n, _i32p(ids)), "block_alloc")
+        return ids[:n].tolist()
+
+    def free(self, ids) -> None:
+        a = np.ascontiguousarray(ids, dtype=np.int32)
+        check(_L.block_free(self._h, _i32p(a), a.size), "block_free")
+
+    def fork(self, ids) -> None:
+        a = np.ascontiguousarray(ids, dtype=np.int32)
+        check(_L.block_fork(self._h, _i32p(a), a.size), "block_fork")
+
+    def refcount(self, i: int) -> int:
+        rc = ctypes.c_int32()
+        check(_L.block_refcount(self._h, i, ctypes.byref(rc)), "block_refcount")
+        return rc.value
+
+    def reserve_slot(self, table: np.ndarray, n_blocks: int, ctx_len: int):
+        """Reserve the slot of token ``ctx_len``; ``table`` (int32, capacity =
+        its length) is updated in place.  Returns (slot, n_blocks, cow_src, cow_dst)."""
+        assert table.dtype == np.int32 and table.flags["C_CONTIGUOUS"]
+        nb = ctypes.c_int32(n_blocks)
+        slot = ctypes.c_int64()
+        src, dst = ctypes.c_int32(), ctypes.c_int32()
+        check(_L.kv_seq_reserve_slot(self._h, _i32p(table), table.size, ctypes.byref(nb), ctx_len,
+                                     ctypes.byref(slot), ctypes.byref(src), ctypes.byref(dst)),
+              "kv_seq_reserve_slot")
+        return slot.value, nb.value, src.value, dst.value
+
+    def reserve_slots(self, tables: np.ndarray, n_blocks: np.ndarray, ctx_lens: np.ndarray):
+        """Batched reserve_slot over B sequences (tables [B][cap] and n_blocks
+        [B] updated in place).  Returns (slots int64 [B], cow pairs int32 [k][2])."""
+        assert tables.dtype == np.int32 and tables.flags["C_CONTIGUOUS"] and tables.ndim == 2
+        assert n_blocks.dtype == np.int32 and n_blocks.flags["C_CONTIGUOUS"]
+        B, cap = tables.shape
+        cl = np.ascontiguousarray(ctx_lens, dtype=np.int32)
+        slots = np.zeros(B, np.int64)
+        pairs = np.zeros((max(B, 1), 2), np.int32)
+        ncow, ndone = ctypes.c_int32(), ctypes.c_int32()
+        check(_L.kv_batch_reserve_slots(self._h, B, _i32p(tables), cap, _i32p(n_blocks), _i32p(cl),
+                                        slots.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                        _i32p(pairs), ctypes.byref(ncow), ctypes.byref(ndone)),
+              "kv_batch_reserve_slots")
+        return slots, pairs[:ncow.value].copy()
+
+
+# ---------------------------------------------------------------------------
+# device calls
+
+def paged_kv_append(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor,
+                    k_pool: torch.Tensor, v_pool: torch.Tensor) -> None:
+    dev = k_pool.device
+    for t, n in ((k_pool, "k_pool"), (v_pool, "v_pool"), (k_new, "k_new"), (v_new, "v_new")):
+        _need(t, n, torch.float16, dev)
+    _need(slot_mapping, "slot_mapping", torch.int64, dev)
+    nb, Hkv, bs, D = k_pool.shape
+    T = slot_mapping.numel()
+    if k_new.numel() != T * Hkv * D or v_new.numel() != T * Hkv * D or v_pool.shape != k_pool.shape:
+        raise ValueError("paged_kv_append: shape mismatch")
+    check(_L.paged_kv_append(k_new.data_ptr(), v_new.data_ptr(), slot_mapping.data_ptr(),
+                             k_pool.data_ptr(), v_pool.data_ptr(), T, Hkv, D, bs, nb, _stream(dev)),
+          "paged_kv_append")
+
+
+def paged_kv_copy_blocks(k_pool: torch.Tensor, v_pool: torch.Tensor, pairs: torch.Tensor) -> None:
+    dev = k_pool.device
+    _need(k_pool, "k_pool", torch.float16, dev)
+    _need(v_pool, "v_pool", torch.float16, dev)
+    _need(pairs, "pairs", torch.int32, dev)
+    nb, Hkv, bs, D = k_pool.shape
+    n = pairs.numel() // 2
+    check(_L.paged_kv_copy_blocks(k_pool.data_ptr(), v_pool.data_ptr(), pairs.data_ptr(), n, Hkv, D,
+                                  bs, nb, _stream(dev)), "paged_kv_copy_blocks")
+
+
+def workspace_size(Hq: int, Hkv: int, q_len: int, head_dim: int, grid_ctas: int = 0) -> int:
+    n = ctypes.c_size_t()
+    check(_L.paged_attention_workspace_size(Hq, Hkv, q_len, head_dim, grid_ctas, ctypes.byref(n)),
+          "paged_attention_workspace_size")
+    return n.value
+
+
+def _attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len, out, workspace,
+               grid_ctas, min_split_blocks, use_pdl, entry):
+    dev = k_pool.device
+    for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool")):
+        _need(t, n, torch.float16, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(context_lens, "context_lens", torch.int32, dev)
+    nb, Hkv, bs, D = k_pool.shape
+    B = context_lens.numel()
+    Hq = q.shape[-2]
+    if q.shape[-1] != D or q.numel() != B * q_len * Hq * D:
+        raise ValueError("q must be [B][q_len][Hq][D]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B:
+        raise ValueError("block_tables must be [B][max_blocks]")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.float16, dev)
+    if out.shape != q.shape:
+        raise ValueError("out must have q's shape")
+    need = workspace_size(Hq, Hkv, q_len, D, grid_ctas)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, dev)
+    mb = block_tables.shape[1]
+    args = (q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_tables.data_ptr(), mb,
+            context_lens.data_ptr())
+    tail = (float(scale), out.data_ptr(), B, Hq, Hkv, D, bs, nb, workspace.data_ptr(),
+            workspace.numel())
+    if entry == "decode":
+        rc = _L.paged_decode_attention(*args, *tail, _stream(dev))
+    elif entry == "verify":
+        rc = _L.paged_verify_attention(*args, q_len, *tail, _stream(dev))
+    else:
+        o = _abi.PagedAttentionOpts(grid_ctas, min_split_blocks, use_pdl)
+        rc = _L.paged_attention_ex(*args, q_len, *tail, ctypes.byref(o), _stream(dev))
+    check(rc, f"paged attention ({entry})")
+    return out
+
+
+def paged_decode_attention(q, k_pool, v_pool, block_tables, context_lens, scale, out=None,
+                           workspace=None):
+    """out[s][h] = softmax(scale q K^T) V over the first context_lens[s] tokens."""
+    return _attention(q, k_pool, v_pool, block_tables, context_lens, scale, 1, out, workspace,
+                      0, 0, 0, "decode")
+
+
+def paged_verify_attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len, out=None,
+                           workspace=None):
+    """Causal verify window: row j sees tokens 0 .. context_lens[s] - q_len + j."""
+    return _attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len, out, workspace,
+                      0, 0, 0, "verify")
+
+
+def paged_attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len=1, out=None,
+                    workspace=None, grid_ctas=0, min_split_blocks=0, use_pdl=0):
+    """Decode / verify with launch knobs (grid size, smallest split, PDL)."""
+    return _attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len, out, workspace,
+                      grid_ctas, min_split_blocks, use_pdl, "ex")
+
+
+def device_error(reset: bool = True, device=None) -> int:
+    """Synchronise the current stream and return (optionally clear) the
+    device error word (bits KV_DEV_*)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    w = ctypes.c_int32()
+    check(_L.kv_device_error(ctypes.byref(w), 1 if reset else 0, _stream(dev)), "kv_device_error")
+    return w.value

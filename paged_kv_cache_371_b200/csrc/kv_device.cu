@@ -1,0 +1,169 @@
+// Device-side helpers of the paged KV library: the per-device error word, the
+// cache-append scatter and the copy-on-write block copy.
+//
+// Cache append: each decode step writes the new token's K and V into the slot
+// the host reserved for it ("LLM 推理优化：KV Cache、PagedAttention 与量化"
+// §2.3 (1): blocks are filled on write).  Block copy: the copy-on-write step of
+// §2.3 (2) of the same page (the block a beam writes into is copied first).
+// Both are plain byte moves: 16-byte vector loads/stores, fully coalesced
+// within each (token, head) row and each block.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/paged_kv.h"
+#include "kv_device.h"
+#include "kv_status.h"
+
+namespace {
+
+__device__ int g_kv_error_word;
+
+constexpr int kMaxDevices = 64;
+int* g_word_ptr[kMaxDevices];
+std::mutex g_word_mu;
+
+__global__ void append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                              const int64_t* __restrict__ slot_mapping, uint4* __restrict__ k_pool,
+                              uint4* __restrict__ v_pool, int32_t T, int32_t Hkv,
+                              int32_t chunks_per_row, int32_t bs, int64_t num_slots, int* err)
+{
+    // one thread per 16-byte chunk of one (token, head) row, K and V together
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t per_tok = (int64_t)Hkv * chunks_per_row;
+    if (i >= (int64_t)T * per_tok) return;
+    const int32_t t = (int32_t)(i / per_tok);
+    const int32_t rem = (int32_t)(i % per_tok);
+    const int32_t h = rem / chunks_per_row;
+    const int32_t c = rem % chunks_per_row;
+    const int64_t slot = __ldg(slot_mapping + t);
+    if (slot < 0) return;
+    if (slot >= num_slots) {
+        if (rem == 0) atomicOr(err, KV_DEV_BAD_SLOT);
+        return;
+    }
+    const int64_t blk = slot / bs;
+    const int32_t off = (int32_t)(slot % bs);
+    const int64_t dst = ((blk * Hkv + h) * bs + off) * chunks_per_row + c;
+    k_pool[dst] = __ldg(k_new + i);
+    v_pool[dst] = __ldg(v_new + i);
+}
+
+__global__ void copy_blocks_kernel(uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
+                                   const int32_t* __restrict__ pairs, int32_t n,
+                                   int64_t chunks_per_block, int32_t num_blocks, int* err)
+{
+    const int32_t pair = blockIdx.y;
+    const int32_t src = __ldg(pairs + 2 * pair);
+    const int32_t dst = __ldg(pairs + 2 * pair + 1);
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(err, KV_DEV_BAD_BLOCK);
+        return;
+    }
+    const uint4* ks = k_pool + (int64_t)src * chunks_per_block;
+    const uint4* vs = v_pool + (int64_t)src * chunks_per_block;
+    uint4* kd = k_pool + (int64_t)dst * chunks_per_block;
+    uint4* vd = v_pool + (int64_t)dst * chunks_per_block;
+    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < chunks_per_block;
+         c += (int64_t)gridDim.x * blockDim.x) {
+        kd[c] = ks[c];
+        vd[c] = vs[c];
+    }
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+int* kv_error_word_ptr()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_word_mu);
+    if (!g_word_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_kv_error_word) != cudaSuccess) return nullptr;
+        g_word_ptr[dev] = static_cast<int*>(p);
+    }
+    return g_word_ptr[dev];
+}
+
+int kv_cuda_check(cudaError_t e, const char* where)
+{
+    if (e == cudaSuccess) return KV_OK;
+    static thread_local char buf[256];
+    snprintf(buf, sizeof(buf), "%s: %s", where, cudaGetErrorString(e));
+    return kv_fail(KV_ERR_CUDA, buf);
+}
+
+extern "C" {
+
+int paged_kv_append(const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                    void* k_pool, void* v_pool, int32_t T, int32_t Hkv, int32_t head_dim,
+                    int32_t block_size, int32_t num_blocks, void* stream)
+{
+    if (T < 0 || Hkv <= 0 || head_dim <= 0 || head_dim % 8 != 0 || block_size <= 0 ||
+        num_blocks <= 0)
+        return kv_fail(KV_ERR_INVALID, "paged_kv_append: bad sizes");
+    if (T == 0) return KV_OK;
+    if (!k_new || !v_new || !slot_mapping || !k_pool || !v_pool)
+        return kv_fail(KV_ERR_INVALID, "paged_kv_append: null pointer");
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool))
+        return kv_fail(KV_ERR_INVALID, "paged_kv_append: buffers must be 16-byte aligned");
+    int* err = kv_error_word_ptr();
+    if (!err) return kv_fail(KV_ERR_CUDA, "paged_kv_append: no device error word");
+    const int32_t cpr = head_dim / 8;
+    const int64_t total = (int64_t)T * Hkv * cpr;
+    const int threads = 256;
+    const int64_t blocks = (total + threads - 1) / threads;
+    append_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), slot_mapping,
+        static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), T, Hkv, cpr, block_size,
+        (int64_t)num_blocks * block_size, err);
+    return kv_cuda_check(cudaGetLastError(), "paged_kv_append");
+}
+
+int paged_kv_copy_blocks(void* k_pool, void* v_pool, const int32_t* pairs, int32_t n, int32_t Hkv,
+                         int32_t head_dim, int32_t block_size, int32_t num_blocks, void* stream)
+{
+    if (n < 0 || Hkv <= 0 || head_dim <= 0 || head_dim % 8 != 0 || block_size <= 0 ||
+        num_blocks <= 0 || n > 65535)
+        return kv_fail(KV_ERR_INVALID, "paged_kv_copy_blocks: bad sizes");
+    if (n == 0) return KV_OK;
+    if (!k_pool || !v_pool || !pairs)
+        return kv_fail(KV_ERR_INVALID, "paged_kv_copy_blocks: null pointer");
+    if (!aligned16(k_pool) || !aligned16(v_pool))
+        return kv_fail(KV_ERR_INVALID, "paged_kv_copy_blocks: pools must be 16-byte aligned");
+    int* err = kv_error_word_ptr();
+    if (!err) return kv_fail(KV_ERR_CUDA, "paged_kv_copy_blocks: no device error word");
+    const int64_t cpb = (int64_t)Hkv * block_size * head_dim / 8;
+    const int threads = 256;
+    int64_t bx = (cpb + threads - 1) / threads;
+    if (bx > 64) bx = 64;
+    dim3 grid((unsigned)bx, (unsigned)n);
+    copy_blocks_kernel<<<grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), pairs, n, cpb, num_blocks, err);
+    return kv_cuda_check(cudaGetLastError(), "paged_kv_copy_blocks");
+}
+
+int kv_device_error(int32_t* word_out, int32_t reset, void* stream)
+{
+    if (!word_out) return kv_fail(KV_ERR_INVALID, "kv_device_error: null output");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = kv_cuda_check(cudaMemcpyFromSymbolAsync(word_out, g_kv_error_word, sizeof(int32_t), 0,
+                                                     cudaMemcpyDeviceToHost, st),
+                           "kv_device_error");
+    if (rc != KV_OK) return rc;
+    if (reset) {
+        const int32_t zero = 0;
+        rc = kv_cuda_check(cudaMemcpyToSymbolAsync(g_kv_error_word, &zero, sizeof(int32_t), 0,
+                                                   cudaMemcpyHostToDevice, st),
+                           "kv_device_error");
+        if (rc != KV_OK) return rc;
+    }
+    return kv_cuda_check(cudaStreamSynchronize(st), "kv_device_error");
+}
+
+}  // extern "C"

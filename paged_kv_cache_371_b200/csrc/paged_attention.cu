@@ -1,0 +1,1056 @@
+// Paged decode / verify attention for sm_100a.
+//
+// What is computed ("大模型推理加速与显存黑科技 (Inference Acceleration & KV Cache)"
+// §2, the Attention(Q,K,V) formula): for every sequence s, window row j and
+// query head h,  out = softmax(scale * q . K_t) V_t  over the visible tokens t,
+// K_t / V_t read through the sequence's block table ("LLM 推理优化：KV Cache、
+// PagedAttention 与量化" §2.2; the same §3.2 figure of the first page with
+// 16-token blocks).  The softmax is streamed: tiles of K/V are staged on chip
+// and a running maximum and denominator are kept ("大模型推理加速与显存黑科技"
+// §4.2, tiling with an online softmax).  Query heads form contiguous groups
+// that share one KV head ("大模型推理加速：从 KV Cache 到投机采样的工程实践"
+// §"主流优化策略", GQA).  Row j of a verify window sees tokens up to
+// L - q_len + j ("LLM推理优化实战：从KV Cache到Speculative Decoding" §"Speculative
+// Decoding：用草稿模型加速", verify in one target pass).
+//
+// Design (B200):
+//  * Work is the flattened space of (sequence, kv-head, block) units.  Each
+//    persistent CTA takes one equal contiguous run of units, so CTAs stay
+//    balanced for any length mix; a (sequence, kv-head) that straddles CTAs
+//    yields partial results (o/l, log2-sum-exp) that a second kernel merges
+//    (split-context log-sum-exp merge).  The schedule is computed on the
+//    device from context_lens: no host planning, no per-step copies.
+//  * One producer warp streams K and V tiles with 2-D TMA (128-byte swizzle)
+//    into a ring of shared-memory stages (mbarrier complete_tx), plus the
+//    query rows with a 1-D bulk copy at each segment start.  Consumer warps
+//    take 16 tokens each per 64-token stage.
+//  * When the rows sharing a KV head (GQA group x window) make the products a
+//    dense contraction (rows > 1), q K^T and P V run on tensor cores
+//    (mma.sync m16n8k16, fp16 in, fp32 accumulate), fed by conflict-free
+//    ldmatrix from the swizzled tiles.  With one row (MHA decode) the work is
+//    a matrix-vector product and runs on the FMA pipes with warp shuffles.
+//  * Every wait is bounded; a timeout or a bad block id sets a bit in the
+//    device error word and the kernel returns without trapping.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/paged_kv.h"
+#include "kv_device.h"
+#include "kv_ptx.cuh"
+#include "kv_status.h"
+
+namespace pkv {
+
+constexpr int kTS = 64;                     // tokens per pipeline stage
+constexpr int kTokWarps = 4;                // consumer warps along the tokens of a stage
+constexpr int kMaxMT = 2;                   // m16 tiles of rows per KV head (rows <= 32)
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr int kSmemBudget = 225 * 1024;
+constexpr float kNegInf = -__builtin_huge_valf();
+
+enum : int32_t { F_FIRST = 1, F_LAST = 2, F_WHOLE = 4, F_END = 8 };
+
+struct StageMeta {
+    int32_t s, kvh, t0, ntok, L, flags, slot, pad;
+};
+
+struct Params {
+    const __half* q;
+    __half* out;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    float* part_o;    // [grid][2][RP][D]
+    float* part_lse;  // [grid][2][RP]
+    int4* meta;       // [grid]: {s, kvh, first cta, slot in first cta} or s = -1
+    int* err;
+    int32_t max_blocks, B, q_len, Hq, Hkv, G, rows, num_blocks, min_share;
+    float scale_log2;
+};
+
+template <int D_, int BS_, int MT_, bool FMA_>
+struct Cfg {
+    static constexpr int D = D_, BS = BS_, MT = MT_;
+    static constexpr bool FMA = FMA_;
+    static constexpr int NH = D / 64;                       // 64-column halves per row
+    static constexpr int NBS = kTS / BS;                    // blocks per stage
+    static constexpr int RP = FMA ? 1 : 16 * MT;            // padded rows
+    static constexpr int NCW = FMA ? kTokWarps : kTokWarps * MT;
+    static constexpr int THREADS = (NCW + 1) * 32;
+    static constexpr int KV_BYTES = kTS * D * 2;            // K (or V) bytes per stage
+    static constexpr int Q_BYTES = (RP * D * 2 + 1023) / 1024 * 1024;
+    static constexpr int STAGE_BYTES = 2 * KV_BYTES + Q_BYTES;
+    static constexpr int OB_STRIDE = D + 8;                 // floats per obuf row
+    static constexpr int OBUF_BYTES = RP * OB_STRIDE * 4;
+    static constexpr int ML_BYTES = kTokWarps * RP * 2 * 4;
+    static constexpr int FIXED = OBUF_BYTES + ML_BYTES + 128 + 16 * 64;
+    static constexpr int STAGES_RAW = (kSmemBudget - FIXED) / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+    static_assert(STAGES >= 2, "not enough shared memory for two stages");
+    static constexpr int META_OFF = STAGES * STAGE_BYTES;   // StageMeta[STAGES]
+    static constexpr int BAR_OFF = META_OFF + STAGES * 32;  // full[S], empty[S]
+    static constexpr int ZERO_OFF = BAR_OFF + STAGES * 16;  // 128 zero bytes
+    static constexpr int ML_OFF = ZERO_OFF + 128;
+    static constexpr int OBUF_OFF = ML_OFF + ML_BYTES;
+    static constexpr int SMEM_USED = OBUF_OFF + OBUF_BYTES;
+    static constexpr int SMEM_ALLOC = SMEM_USED + 1024;    // room to align the base
+};
+
+__device__ __forceinline__ int32_t nblk_of(int32_t L, int32_t bs, int32_t max_blocks)
+{
+    int32_t nb = L <= 0 ? 1 : (L + bs - 1) / bs;
+    return nb > max_blocks ? max_blocks : nb;
+}
+
+__device__ __forceinline__ int32_t clamp_len(int32_t L, int32_t bs, int32_t max_blocks)
+{
+    if (L < 0) return 0;
+    const int32_t cap = max_blocks * bs;
+    return L > cap ? cap : L;
+}
+
+__device__ __forceinline__ int64_t warp_sum64(int64_t v)
+{
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ int64_t warp_incl_scan64(int64_t v, int lane)
+{
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int64_t n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    return v;
+}
+
+// Swizzled address of 16-byte chunk `c` (0..7) of row `row` in a TMA box of
+// 64 fp16 columns written with 128-byte swizzle (box base 1024-aligned).
+__device__ __forceinline__ uint32_t swz(uint32_t box_base, int row, int c)
+{
+    return box_base + row * 128 + ((c ^ (row & 7)) << 4);
+}
+
+// ---------------------------------------------------------------------------
+// Producer warp: walks this CTA's run of units and feeds the stage ring.
+template <class C>
+__device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const Params& p,
+                         uint8_t* smem, volatile int* abort_flag)
+{
+    const int lane = threadIdx.x & 31;
+    const uint32_t sbase = smem_u32(smem);
+    StageMeta* smeta = reinterpret_cast<StageMeta*>(smem + C::META_OFF);
+    const uint32_t full0 = sbase + C::BAR_OFF;
+    const uint32_t empty0 = full0 + C::STAGES * 8;
+    const uint64_t pol = l2_policy_evict_first();
+    if (lane == 0) {
+        prefetch_tmap(tmK);
+        prefetch_tmap(tmV);
+    }
+
+    // Pass 1: total units.
+    int64_t total = 0;
+    for (int base = 0; base < p.B; base += 32) {
+        const int s = base + lane;
+        int64_t u = 0;
+        if (s < p.B) u = (int64_t)nblk_of(__ldg(p.context_lens + s), C::BS, p.max_blocks) * p.Hkv;
+        total += warp_sum64(u);
+    }
+    const int64_t G = gridDim.x;
+    int64_t share = (total + G - 1) / G;
+    if (share < p.min_share) share = p.min_share;
+    const int64_t u0 = (int64_t)blockIdx.x * share;
+    const int64_t u1 = u0 + share < total ? u0 + share : total;
+
+    int4 my_meta = make_int4(-1, 0, 0, 0);
+    int k_issued = 0;  // stages issued so far
+    bool ok = true;
+
+    if (u0 < u1) {
+        // Pass 2: the sequence holding unit u0.
+        int s = -1;
+        int64_t seq_start = 0, run = 0;
+        for (int base = 0; base < p.B && s < 0; base += 32) {
+            const int sl = base + lane;
+            int64_t u = 0;
+            if (sl < p.B) u = (int64_t)nblk_of(__ldg(p.context_lens + sl), C::BS, p.max_blocks) * p.Hkv;
+            const int64_t incl = warp_incl_scan64(u, lane);
+            const bool hit = sl < p.B && run + incl > u0 && run + incl - u <= u0;
+            const unsigned m = __ballot_sync(0xffffffffu, hit);
+            if (m) {
+                const int src = __ffs(m) - 1;
+                s = base + src;
+                seq_start = run + __shfl_sync(0xffffffffu, incl - u, src);
+            }
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (s < 0) {  // unreachable when u0 < total; keeps the walk well defined
+            s = 0;
+            ok = false;
+        }
+        int32_t Lraw = __ldg(p.context_lens + s);
+        int32_t L = clamp_len(Lraw, C::BS, p.max_blocks);
+        if (lane == 0 && Lraw > L) atomicOr(p.err, KV_DEV_BAD_BLOCK);
+        int32_t nb = nblk_of(Lraw, C::BS, p.max_blocks);
+        int64_t u = u0;
+        bool first_seg = true;
+        while (u < u1 && ok) {
+            const int64_t local = u - seq_start;
+            const int32_t kvh = (int32_t)(local / nb);
+            const int32_t b0 = (int32_t)(local % nb);
+            const int64_t kv_end = seq_start + (int64_t)(kvh + 1) * nb;
+            const int64_t seg_end = u1 < kv_end ? u1 : kv_end;
+            const int32_t b1 = b0 + (int32_t)(seg_end - u);
+            const bool whole = b0 == 0 && b1 == nb;
+            const int32_t slot = first_seg ? 0 : 1;
+            if (first_seg && b0 > 0 && b1 == nb) {
+                const int64_t gstart = seq_start + (int64_t)kvh * nb;
+                my_meta = make_int4(s, kvh, (int32_t)(gstart / share), (gstart % share) ? 1 : 0);
+            }
+            for (int32_t b = b0; b < b1; b += C::NBS) {
+                const int32_t nbl = (b1 - b) < C::NBS ? (b1 - b) : C::NBS;
+                const int32_t t0 = b * C::BS;
+                int32_t tend = (b + nbl) * C::BS;
+                if (tend > L) tend = L;
+                const int32_t ntok = tend > t0 ? tend - t0 : 0;
+                const int stage = k_issued % C::STAGES;
+                const int round = k_issued / C::STAGES;
+                if (round > 0) {
+                    if (!mbar_wait_bounded(empty0 + stage * 8, (round - 1) & 1, kWaitLimitNs) ||
+                        *abort_flag) {
+                        ok = false;
+                        break;
+                    }
+                }
+                // block ids of this stage, one per lane
+                int32_t id = -1;
+                const bool has_tok = lane < nbl && t0 + lane * C::BS < L;
+                if (has_tok) id = __ldg(p.block_tables + (int64_t)s * p.max_blocks + b + lane);
+                const bool bad = has_tok && (id < 0 || id >= p.num_blocks);
+                const bool load = has_tok && !bad;
+                const unsigned lmask = __ballot_sync(0xffffffffu, load);
+                if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, KV_DEV_BAD_BLOCK);
+                const bool firstst = b == b0;
+                const uint32_t qbytes = (uint32_t)(p.G * C::D * 2);
+                uint32_t bytes = (uint32_t)__popc(lmask) * (uint32_t)(2 * C::BS * C::D * 2);
+                if (firstst) bytes += qbytes * (uint32_t)p.q_len;
+                const uint32_t full = full0 + stage * 8;
+                if (lane == 0) {
+                    StageMeta& md = smeta[stage];
+                    md.s = s;
+                    md.kvh = kvh;
+                    md.t0 = t0;
+                    md.ntok = ntok;
+                    md.L = L;
+                    md.flags = (firstst ? F_FIRST : 0) | (b + C::NBS >= b1 ? F_LAST : 0) |
+                               (whole ? F_WHOLE : 0);
+                    md.slot = slot;
+                    mbar_arrive_expect_tx(full, bytes);
+                }
+                __syncwarp();
+                const uint32_t st = sbase + stage * C::STAGE_BYTES;
+                if (load) {
+                    const int32_t y = (id * p.Hkv + kvh) * C::BS;
+#pragma unroll
+                    for (int h = 0; h < C::NH; ++h) {
+                        const uint32_t off = (uint32_t)((lane * C::NH + h) * C::BS * 128);
+                        tma_load_2d(st + off, tmK, h * 64, y, full, pol);
+                        tma_load_2d(st + C::KV_BYTES + off, tmV, h * 64, y, full, pol);
+                    }
+                }
+                if (firstst && lane < p.q_len) {
+                    const __half* src =
+                        p.q + (((int64_t)s * p.q_len + lane) * p.Hq + (int64_t)kvh * p.G) * C::D;
+                    bulk_load(st + 2 * C::KV_BYTES + lane * qbytes, src, qbytes, full);
+                }
+                ++k_issued;
+            }
+            first_seg = false;
+            u = seg_end;
+            if (u < u1 && u == seq_start + (int64_t)nb * p.Hkv) {
+                seq_start = u;
+                ++s;
+                Lraw = __ldg(p.context_lens + s);
+                L = clamp_len(Lraw, C::BS, p.max_blocks);
+                if (lane == 0 && Lraw > L) atomicOr(p.err, KV_DEV_BAD_BLOCK);
+                nb = nblk_of(Lraw, C::BS, p.max_blocks);
+            }
+        }
+    }
+    if (lane == 0) p.meta[blockIdx.x] = my_meta;
+
+    // End marker.
+    if (ok) {
+        const int stage = k_issued % C::STAGES;
+        const int round = k_issued / C::STAGES;
+        if (round > 0 && !mbar_wait_bounded(empty0 + stage * 8, (round - 1) & 1, kWaitLimitNs))
+            ok = false;
+        if (ok) {
+            if (lane == 0) {
+                smeta[stage].flags = F_END;
+                mbar_arrive(full0 + stage * 8);
+            }
+            ++k_issued;
+        }
+    }
+    if (!ok) {
+        if (lane == 0) {
+            atomicOr(p.err, KV_DEV_TIMEOUT);
+            *abort_flag = 1;
+        }
+    }
+    // Drain: every issued stage's copies must have landed before the CTA may
+    // exit (consumers normally wait for them anyway).
+    for (int i = lane; i < C::STAGES && i < k_issued; i += 32) {
+        const int n_i = (k_issued - i + C::STAGES - 1) / C::STAGES;  // issues into slot i
+        if (!mbar_wait_bounded(full0 + i * 8, (n_i - 1) & 1, kWaitLimitNs))
+            atomicOr(p.err, KV_DEV_TIMEOUT);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Output of a finished segment: `obuf` rows hold the normalised o; `mlb`
+// holds per token-warp (m, l).  Writes fp16 output or fp32 partials.
+template <class C>
+__device__ void store_segment(const Params& p, const StageMeta& md, const float* obuf,
+                              const float* mlb, int tid)
+{
+    const int rows = p.rows;
+    if (md.flags & F_WHOLE) {
+        for (int idx = tid; idx < rows * (C::D / 8); idx += C::NCW * 32) {
+            const int R = idx / (C::D / 8);
+            const int d0 = (idx % (C::D / 8)) * 8;
+            const int j = R / p.G, g = R % p.G;
+            const float* src = obuf + R * C::OB_STRIDE + d0;
+            uint4 v;
+            v.x = pack_half2(src[0], src[1]);
+            v.y = pack_half2(src[2], src[3]);
+            v.z = pack_half2(src[4], src[5]);
+            v.w = pack_half2(src[6], src[7]);
+            __half* dst = p.out + (((int64_t)md.s * p.q_len + j) * p.Hq + (int64_t)md.kvh * p.G + g) *
+                                      C::D + d0;
+            *reinterpret_cast<uint4*>(dst) = v;
+        }
+    } else {
+        const int64_t pbase = ((int64_t)blockIdx.x * 2 + md.slot) * C::RP;
+        for (int idx = tid; idx < rows * (C::D / 8); idx += C::NCW * 32) {
+            const int R = idx / (C::D / 8);
+            const int d0 = (idx % (C::D / 8)) * 8;
+            const float* src = obuf + R * C::OB_STRIDE + d0;
+            float4* dst = reinterpret_cast<float4*>(p.part_o + (pbase + R) * C::D + d0);
+            dst[0] = make_float4(src[0], src[1], src[2], src[3]);
+            dst[1] = make_float4(src[4], src[5], src[6], src[7]);
+        }
+        for (int R = tid; R < rows; R += C::NCW * 32) {
+            float M = kNegInf;
+#pragma unroll
+            for (int w = 0; w < kTokWarps; ++w) M = fmaxf(M, mlb[(w * C::RP + R) * 2]);
+            const float Mu = M == kNegInf ? 0.f : M;
+            float Ls = 0.f;
+#pragma unroll
+            for (int w = 0; w < kTokWarps; ++w)
+                Ls += mlb[(w * C::RP + R) * 2 + 1] * ex2(mlb[(w * C::RP + R) * 2] - Mu);
+            p.part_lse[pbase + R] = Ls > 0.f ? Mu + lg2(Ls) : kNegInf;
+        }
+    }
+}
+
+// Combine the token-warps' (m, l) for row R; returns this warp's factor
+// 2^(m_w - M) / sum.
+template <class C>
+__device__ __forceinline__ float row_factor(const float* mlb, int R, float m_w)
+{
+    float M = kNegInf;
+#pragma unroll
+    for (int w = 0; w < kTokWarps; ++w) M = fmaxf(M, mlb[(w * C::RP + R) * 2]);
+    const float Mu = M == kNegInf ? 0.f : M;
+    float Ls = 0.f;
+#pragma unroll
+    for (int w = 0; w < kTokWarps; ++w)
+        Ls += mlb[(w * C::RP + R) * 2 + 1] * ex2(mlb[(w * C::RP + R) * 2] - Mu);
+    return Ls > 0.f ? ex2(m_w - Mu) / Ls : 0.f;
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core consumer: rows = GQA group x window (1 < rows <= 16*MT).
+template <class C>
+__device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort_flag)
+{
+    const int cw = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int mt = cw / kTokWarps, qw = cw % kTokWarps;
+    const int gid = lane >> 2, tig = lane & 3;
+    const uint32_t sbase = smem_u32(smem);
+    const StageMeta* smeta = reinterpret_cast<const StageMeta*>(smem + C::META_OFF);
+    const uint32_t full0 = sbase + C::BAR_OFF;
+    const uint32_t empty0 = full0 + C::STAGES * 8;
+    const uint32_t zero_row = sbase + C::ZERO_OFF;
+    float* mlb = reinterpret_cast<float*>(smem + C::ML_OFF);
+    float* obuf = reinterpret_cast<float*>(smem + C::OBUF_OFF);
+    const float sl2 = p.scale_log2;
+
+    // per-lane ldmatrix geometry
+    const int k_tok = qw * 16 + (lane >> 4) * 8 + (lane & 7);   // K: token of this lane's row
+    const int k_sel = (lane >> 3) & 1;                          // K: chunk select
+    const int v_i = ((lane >> 3) & 1) * 8 + (lane & 7);         // V: token within my 16
+    const int v_tok = qw * 16 + v_i;
+    const int v_sel = lane >> 4;
+    const uint32_t k_row_off = (uint32_t)(((k_tok / C::BS) * C::NH * C::BS + (k_tok % C::BS)) * 128);
+    const uint32_t v_row_off = (uint32_t)(((v_tok / C::BS) * C::NH * C::BS + (v_tok % C::BS)) * 128);
+    const int k_x = k_tok % C::BS & 7;
+    const int v_x = v_tok % C::BS & 7;
+
+    float O[C::D / 8][4];
+    uint32_t qa[C::D / 16][4];
+    float m[2], l[2];
+    int lim[2];
+
+    int stage = 0;
+    uint32_t phase = 0;
+    for (;;) {
+        if (!mbar_wait_bounded(full0 + stage * 8, phase, kWaitLimitNs)) {
+            *abort_flag = 1;
+            break;
+        }
+        const StageMeta md = smeta[stage];
+        if (md.flags & F_END) break;
+        const uint32_t st = sbase + stage * C::STAGE_BYTES;
+        if (md.flags & F_FIRST) {
+            const uint8_t* qs = smem + stage * C::STAGE_BYTES + 2 * C::KV_BYTES;
+            const int r0 = mt * 16 + gid, r1 = r0 + 8;
+#pragma unroll
+            for (int ks = 0; ks < C::D / 16; ++ks) {
+                const int c0 = ks * 16 + tig * 2;
+                qa[ks][0] = *reinterpret_cast<const uint32_t*>(qs + (r0 * C::D + c0) * 2);
+                qa[ks][1] = *reinterpret_cast<const uint32_t*>(qs + (r1 * C::D + c0) * 2);
+                qa[ks][2] = *reinterpret_cast<const uint32_t*>(qs + (r0 * C::D + c0 + 8) * 2);
+                qa[ks][3] = *reinterpret_cast<const uint32_t*>(qs + (r1 * C::D + c0 + 8) * 2);
+            }
+#pragma unroll
+            for (int n = 0; n < C::D / 8; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.f;
+            m[0] = m[1] = kNegInf;
+            l[0] = l[1] = 0.f;
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int R = r0 + rr * 8;
+                lim[rr] = R < p.rows ? md.L - p.q_len + R / p.G + 1 : md.L;
+            }
+        }
+        const int nv = md.ntok - qw * 16;
+        if (nv > 0) {
+            // S = q K^T for my 16 tokens (two n8 tiles)
+            float S[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int ks = 0; ks < C::D / 16; ++ks) {
+                const int h = ks / 4;
+                const int c = (2 * ks) % 8 + k_sel;
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(st + k_row_off + h * C::BS * 128 + ((c ^ k_x) << 4), b0, b1, b2, b3);
+                mma_16816(S[0], qa[ks], b0, b1);
+                mma_16816(S[1], qa[ks], b2, b3);
+            }
+            const int pos0 = md.t0 + qw * 16 + tig * 2;
+            float mx[2] = {kNegInf, kNegInf};
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int pos = pos0 + nt * 8 + (c & 1);
+                    const float v = pos < lim[c >> 1] ? S[nt][c] * sl2 : kNegInf;
+                    S[nt][c] = v;
+                    mx[c >> 1] = fmaxf(mx[c >> 1], v);
+                }
+            float alpha[2], mu[2];
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
+                mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
+                const float mn = fmaxf(m[rr], mx[rr]);
+                mu[rr] = mn == kNegInf ? 0.f : mn;
+                alpha[rr] = ex2(m[rr] - mu[rr]);
+                m[rr] = mn;
+            }
+            float ps[2] = {0.f, 0.f};
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float e = ex2(S[nt][c] - mu[c >> 1]);
+                    S[nt][c] = e;
+                    ps[c >> 1] += e;
+                }
+            l[0] = l[0] * alpha[0] + ps[0];
+            l[1] = l[1] * alpha[1] + ps[1];
+            if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
+#pragma unroll
+                for (int n = 0; n < C::D / 8; ++n) {
+                    O[n][0] *= alpha[0];
+                    O[n][1] *= alpha[0];
+                    O[n][2] *= alpha[1];
+                    O[n][3] *= alpha[1];
+                }
+            }
+            uint32_t pa[4];
+            pa[0] = pack_half2(S[0][0], S[0][1]);
+            pa[1] = pack_half2(S[0][2], S[0][3]);
+            pa[2] = pack_half2(S[1][0], S[1][1]);
+            pa[3] = pack_half2(S[1][2], S[1][3]);
+            // rows of V past the valid tokens read a zero row instead
+            const bool v_ok = v_i < nv;
+#pragma unroll
+            for (int np = 0; np < C::D / 16; ++np) {
+                const int h = np / 4;
+                const int c = (2 * np) % 8 + v_sel;
+                const uint32_t addr =
+                    v_ok ? st + C::KV_BYTES + v_row_off + h * C::BS * 128 + ((c ^ v_x) << 4)
+                         : zero_row;
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_trans(addr, b0, b1, b2, b3);
+                mma_16816(O[2 * np], pa, b0, b1);
+                mma_16816(O[2 * np + 1], pa, b2, b3);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + stage * 8);
+
+        if (md.flags & F_LAST) {
+            // merge the token-warps of each m-tile, then store
+            const int tid = threadIdx.x;
+            for (int i = tid; i < C::RP * C::OB_STRIDE; i += C::NCW * 32) obuf[i] = 0.f;
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                float lr = l[rr];
+                lr += __shfl_xor_sync(0xffffffffu, lr, 1);
+                lr += __shfl_xor_sync(0xffffffffu, lr, 2);
+                if (tig == 0) {
+                    const int R = mt * 16 + gid + rr * 8;
+                    mlb[(qw * C::RP + R) * 2] = m[rr];
+                    mlb[(qw * C::RP + R) * 2 + 1] = lr;
+                }
+            }
+            named_bar_sync(1, C::NCW * 32);
+            float f[2];
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) f[rr] = row_factor<C>(mlb, mt * 16 + gid + rr * 8, m[rr]);
+#pragma unroll
+            for (int n = 0; n < C::D / 8; ++n) {
+                const int col = n * 8 + tig * 2;
+                float* o0 = obuf + (mt * 16 + gid) * C::OB_STRIDE + col;
+                float* o1 = obuf + (mt * 16 + gid + 8) * C::OB_STRIDE + col;
+                atomicAdd(o0, O[n][0] * f[0]);
+                atomicAdd(o0 + 1, O[n][1] * f[0]);
+                atomicAdd(o1, O[n][2] * f[1]);
+                atomicAdd(o1 + 1, O[n][3] * f[1]);
+            }
+            named_bar_sync(1, C::NCW * 32);
+            store_segment<C>(p, md, obuf, mlb, tid);
+            named_bar_sync(1, C::NCW * 32);
+        }
+        if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// FMA consumer: one query row per KV head (MHA decode).  Lane = (token, half
+// of the head dimension) for q . k; lane = D/32 columns for P V.
+template <class C>
+__device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort_flag)
+{
+    constexpr int D = C::D;
+    constexpr int DPL = D / 2;    // q . k columns per lane
+    constexpr int CPL = DPL / 8;  // 16-byte chunks per lane
+    constexpr int DPT = D / 32;   // P V columns per lane
+    const int cw = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int qw = cw;
+    const uint32_t sbase = smem_u32(smem);
+    const StageMeta* smeta = reinterpret_cast<const StageMeta*>(smem + C::META_OFF);
+    const uint32_t full0 = sbase + C::BAR_OFF;
+    const uint32_t empty0 = full0 + C::STAGES * 8;
+    float* mlb = reinterpret_cast<float*>(smem + C::ML_OFF);
+    float* obuf = reinterpret_cast<float*>(smem + C::OBUF_OFF);
+    const float sl2 = p.scale_log2;
+
+    const int tk = lane & 15, hf = lane >> 4;
+    const int k_tok = qw * 16 + tk;
+    const uint32_t k_row = (uint32_t)(((k_tok / C::BS) * C::NH * C::BS + (k_tok % C::BS)) * 128);
+    const int k_x = (k_tok % C::BS) & 7;
+    const int k_box = (hf * DPL) / 64;         // which 64-column box
+    const int k_c0 = ((hf * DPL) % 64) / 8;    // first chunk inside it
+    const int v_col = lane * DPT;
+    const int v_box = v_col / 64;
+    const int v_c = (v_col % 64) / 8;
+    const int v_byte = (v_col % 8) * 2;
+
+    uint32_t qh[DPL / 2];
+    float o[DPT];
+    float m = kNegInf, l = 0.f;
+
+    int stage = 0;
+    uint32_t phase = 0;
+    for (;;) {
+        if (!mbar_wait_bounded(full0 + stage * 8, phase, kWaitLimitNs)) {
+            *abort_flag = 1;
+            break;
+        }
+        const StageMeta md = smeta[stage];
+        if (md.flags & F_END) break;
+        const uint8_t* st = smem + stage * C::STAGE_BYTES;
+        if (md.flags & F_FIRST) {
+            const uint4* qs = reinterpret_cast<const uint4*>(st + 2 * C::KV_BYTES + hf * DPL * 2);
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                const uint4 v = qs[c];
+                qh[4 * c] = v.x;
+                qh[4 * c + 1] = v.y;
+                qh[4 * c + 2] = v.z;
+                qh[4 * c + 3] = v.w;
+            }
+#pragma unroll
+            for (int i = 0; i < DPT; ++i) o[i] = 0.f;
+            m = kNegInf;
+            l = 0.f;
+        }
+        const int nv = md.ntok - qw * 16;
+        if (nv > 0) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            if (tk < nv) {
+                const uint8_t* kb = st + k_row + k_box * C::BS * 128;
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+                    const uint4 kv = *reinterpret_cast<const uint4*>(
+                        kb + (((k_c0 + c) ^ k_x) << 4));
+                    const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t qq = qh[4 * c + e];
+                        acc[e] = fma_h((uint16_t)(qq & 0xffff), (uint16_t)(kw[e] & 0xffff), acc[e]);
+                        acc[e] = fma_h((uint16_t)(qq >> 16), (uint16_t)(kw[e] >> 16), acc[e]);
+                    }
+                }
+            }
+            float sdot = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            sdot += __shfl_xor_sync(0xffffffffu, sdot, 16);
+            const float s = tk < nv ? sdot * sl2 : kNegInf;
+            float mx = s;
+#pragma unroll
+            for (int off = 1; off < 16; off <<= 1)
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            const float mn = fmaxf(m, mx);
+            const float mu = mn == kNegInf ? 0.f : mn;
+            const float alpha = ex2(m - mu);
+            m = mn;
+            const float pe = ex2(s - mu);
+            l = l * alpha + (hf == 0 ? pe : 0.f);
+#pragma unroll
+            for (int i = 0; i < DPT; ++i) o[i] *= alpha;
+            const __half ph = __float2half_rn(pe);
+            const uint16_t phu = __half_as_ushort(ph);
+            const uint8_t* vb = st + C::KV_BYTES + v_box * C::BS * 128;
+            const int lim = nv < 16 ? nv : 16;
+            for (int t = 0; t < lim; ++t) {
+                const uint16_t pt = (uint16_t)__shfl_sync(0xffffffffu, (uint32_t)phu, t);
+                const int vt = qw * 16 + t;
+                const uint8_t* vr = vb + ((vt / C::BS) * C::NH * C::BS + (vt % C::BS)) * 128 +
+                                    ((v_c ^ ((vt % C::BS) & 7)) << 4) + v_byte;
+                if constexpr (DPT == 4) {
+                    const uint2 vv = *reinterpret_cast<const uint2*>(vr);
+                    o[0] = fma_h(pt, (uint16_t)(vv.x & 0xffff), o[0]);
+                    o[1] = fma_h(pt, (uint16_t)(vv.x >> 16), o[1]);
+                    o[2] = fma_h(pt, (uint16_t)(vv.y & 0xffff), o[2]);
+                    o[3] = fma_h(pt, (uint16_t)(vv.y >> 16), o[3]);
+                } else {
+                    const uint32_t vv = *reinterpret_cast<const uint32_t*>(vr);
+                    o[0] = fma_h(pt, (uint16_t)(vv & 0xffff), o[0]);
+                    o[1] = fma_h(pt, (uint16_t)(vv >> 16), o[1]);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + stage * 8);
+
+        if (md.flags & F_LAST) {
+            const int tid = threadIdx.x;
+            for (int i = tid; i < C::RP * C::OB_STRIDE; i += C::NCW * 32) obuf[i] = 0.f;
+            float lr = l;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) lr += __shfl_xor_sync(0xffffffffu, lr, off);
+            if (lane == 0) {
+                mlb[(qw * C::RP) * 2] = m;
+                mlb[(qw * C::RP) * 2 + 1] = lr;
+            }
+            named_bar_sync(1, C::NCW * 32);
+            const float f = row_factor<C>(mlb, 0, m);
+#pragma unroll
+            for (int i = 0; i < DPT; ++i) atomicAdd(obuf + v_col + i, o[i] * f);
+            named_bar_sync(1, C::NCW * 32);
+            store_segment<C>(p, md, obuf, mlb, tid);
+            named_bar_sync(1, C::NCW * 32);
+        }
+        if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+        }
+    }
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    paged_attention_kernel(const __grid_constant__ CUtensorMap tmK,
+                           const __grid_constant__ CUtensorMap tmV, const Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ int abort_flag;
+    const uint32_t sbase = smem_u32(smem);
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        for (int i = 0; i < C::STAGES; ++i) {
+            mbar_init(sbase + C::BAR_OFF + i * 8, 1);
+            mbar_init(sbase + C::BAR_OFF + (C::STAGES + i) * 8, C::NCW);
+        }
+        fence_barrier_init();
+    }
+    // zero the padded query rows of every stage and the zero row
+    if constexpr (!C::FMA) {
+        const int used = p.rows * C::D * 2;
+        for (int st = 0; st < C::STAGES; ++st) {
+            uint8_t* qa = smem + st * C::STAGE_BYTES + 2 * C::KV_BYTES;
+            for (int i = used + threadIdx.x * 16; i < C::RP * C::D * 2; i += C::THREADS * 16)
+                *reinterpret_cast<uint4*>(qa + i) = make_uint4(0, 0, 0, 0);
+        }
+    }
+    if (threadIdx.x < 8)
+        reinterpret_cast<uint4*>(smem + C::ZERO_OFF)[threadIdx.x] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async();
+    __syncthreads();
+    pdl_launch_dependents();
+    const int warp = threadIdx.x >> 5;
+    if (warp == C::NCW) {
+        producer<C>(&tmK, &tmV, p, smem, &abort_flag);
+    } else if constexpr (C::FMA) {
+        consumer_fma<C>(p, smem, &abort_flag);
+    } else {
+        consumer_mma<C>(p, smem, &abort_flag);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Split-context merge: CTA c merges the (sequence, kv-head) whose last piece
+// it computed, from the partials of CTAs meta.first .. c:
+//   lse* = log2 sum_i 2^(lse_i),  out = sum_i 2^(lse_i - lse*) o_i.
+template <int D, int RP>
+__global__ void __launch_bounds__(128) lse_merge_kernel(const Params p)
+{
+    pdl_wait();
+    const int c = blockIdx.x;
+    const int4 md = p.meta[c];
+    if (md.x < 0) return;
+    const int s = md.x, kvh = md.y, a = md.z, slot_a = md.w;
+    for (int idx = threadIdx.x; idx < p.rows * (D / 8); idx += blockDim.x) {
+        const int R = idx / (D / 8);
+        const int d0 = (idx % (D / 8)) * 8;
+        float M = kNegInf;
+        for (int i = a; i <= c; ++i) {
+            const int slot = i == a ? slot_a : 0;
+            M = fmaxf(M, p.part_lse[((int64_t)i * 2 + slot) * RP + R]);
+        }
+        const float Mu = M == kNegInf ? 0.f : M;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float W = 0.f;
+        for (int i = a; i <= c; ++i) {
+            const int slot = i == a ? slot_a : 0;
+            const int64_t pr = ((int64_t)i * 2 + slot) * RP + R;
+            const float w = ex2(p.part_lse[pr] - Mu);
+            W += w;
+            const float4* src = reinterpret_cast<const float4*>(p.part_o + pr * D + d0);
+            const float4 x = src[0], y = src[1];
+            acc[0] += w * x.x;
+            acc[1] += w * x.y;
+            acc[2] += w * x.z;
+            acc[3] += w * x.w;
+            acc[4] += w * y.x;
+            acc[5] += w * y.y;
+            acc[6] += w * y.z;
+            acc[7] += w * y.w;
+        }
+        const float inv = W > 0.f ? 1.f / W : 0.f;
+        const int j = R / p.G, g = R % p.G;
+        uint4 v;
+        v.x = pack_half2(acc[0] * inv, acc[1] * inv);
+        v.y = pack_half2(acc[2] * inv, acc[3] * inv);
+        v.z = pack_half2(acc[4] * inv, acc[5] * inv);
+        v.w = pack_half2(acc[6] * inv, acc[7] * inv);
+        __half* dst = p.out + (((int64_t)s * p.q_len + j) * p.Hq + (int64_t)kvh * p.G + g) * D + d0;
+        *reinterpret_cast<uint4*>(dst) = v;
+    }
+}
+
+}  // namespace pkv
+
+// ===========================================================================
+// Host side
+namespace {
+
+using namespace pkv;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::mutex g_mu;
+
+struct TmapEntry {
+    const void* ptr;
+    uint64_t rows;
+    int D, BS, dev;
+    CUtensorMap map;
+};
+constexpr int kTmapCache = 32;
+TmapEntry g_tmaps[kTmapCache];
+int g_tmap_next = 0;
+
+int get_encoder()
+{
+    if (g_encode) return KV_OK;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+        return kv_fail(KV_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return KV_OK;
+}
+
+// Tensor map of a pool viewed as [num_blocks*Hkv*BS rows][D] fp16, box
+// [BS rows][64 columns], 128-byte swizzle.  Cached by (pointer, shape, device).
+int pool_tmap(const void* pool, uint64_t rows, int D, int BS, CUtensorMap* out)
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (auto& e : g_tmaps)
+        if (e.ptr == pool && e.rows == rows && e.D == D && e.BS == BS && e.dev == dev) {
+            *out = e.map;
+            return KV_OK;
+        }
+    int rc = get_encoder();
+    if (rc != KV_OK) return rc;
+    CUtensorMap m;
+    const cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)BS};
+    const cuuint32_t estride[2] = {1, 1};
+    CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(pool), gdim,
+                          gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return kv_fail(KV_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    TmapEntry& e = g_tmaps[g_tmap_next];
+    g_tmap_next = (g_tmap_next + 1) % kTmapCache;
+    e = {pool, rows, D, BS, dev, m};
+    *out = m;
+    return KV_OK;
+}
+
+int device_sms()
+{
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms > 0 ? sms : 1;
+}
+
+int rows_padded(int rows) { return rows == 1 ? 1 : 16 * ((rows + 15) / 16); }
+
+size_t workspace_bytes_for(int grid, int rp, int D)
+{
+    size_t meta = (size_t)grid * 16;
+    size_t lse = (size_t)grid * 2 * rp * 4;
+    lse = (lse + 15) / 16 * 16;
+    size_t po = (size_t)grid * 2 * rp * D * 4;
+    return meta + lse + po;
+}
+
+template <class C>
+int launch(const CUtensorMap& tk, const CUtensorMap& tv, const Params& prm, int grid, bool pdl,
+           cudaStream_t stream)
+{
+    static std::mutex mu;
+    static unsigned long long configured = 0;  // bit per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (dev < 64 && !(configured & (1ull << dev))) {
+            int rc = kv_cuda_check(
+                cudaFuncSetAttribute(paged_attention_kernel<C>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC),
+                "cudaFuncSetAttribute");
+            if (rc != KV_OK) return rc;
+            configured |= 1ull << dev;
+        }
+    }
+    paged_attention_kernel<C><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(tk, tv, prm);
+    int rc = kv_cuda_check(cudaGetLastError(), "paged_attention_kernel launch");
+    if (rc != KV_OK) return rc;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return kv_cuda_check(cudaLaunchKernelEx(&cfg, lse_merge_kernel<C::D, C::RP>, prm),
+                         "lse_merge_kernel launch");
+}
+
+template <int D, int BS>
+int dispatch_rows(int rows, const CUtensorMap& tk, const CUtensorMap& tv, const Params& prm,
+                  int grid, bool pdl, cudaStream_t st)
+{
+    if (rows == 1) return launch<Cfg<D, BS, 1, true>>(tk, tv, prm, grid, pdl, st);
+    if (rows <= 16) return launch<Cfg<D, BS, 1, false>>(tk, tv, prm, grid, pdl, st);
+    return launch<Cfg<D, BS, 2, false>>(tk, tv, prm, grid, pdl, st);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int attention_impl(const void* q, const void* k_pool, const void* v_pool,
+                   const int32_t* block_tables, int32_t max_blocks_per_seq,
+                   const int32_t* context_lens, int32_t q_len, float scale, void* out, int32_t B,
+                   int32_t Hq, int32_t Hkv, int32_t D, int32_t BS, int32_t num_blocks,
+                   void* workspace, size_t ws_bytes, const paged_attention_opts* opts,
+                   void* stream)
+{
+    if (B < 0 || q_len < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || num_blocks < 1 ||
+        max_blocks_per_seq < 1)
+        return kv_fail(KV_ERR_INVALID, "paged attention: bad sizes");
+    if (D != 64 && D != 128) return kv_fail(KV_ERR_INVALID, "paged attention: head_dim must be 64 or 128");
+    if (BS != 8 && BS != 16) return kv_fail(KV_ERR_INVALID, "paged attention: block_size must be 8 or 16");
+    const int G = Hq / Hkv;
+    const int rows = G * q_len;
+    if (rows > 16 * kMaxMT)
+        return kv_fail(KV_ERR_INVALID, "paged attention: (Hq/Hkv)*q_len must be <= 32");
+    if ((uint64_t)num_blocks * Hkv * BS >= (1ull << 31))
+        return kv_fail(KV_ERR_INVALID, "paged attention: pool too large for 32-bit row coordinates");
+    if (B == 0) return KV_OK;
+    if (!q || !k_pool || !v_pool || !block_tables || !context_lens || !out || !workspace)
+        return kv_fail(KV_ERR_INVALID, "paged attention: null pointer");
+    if (!aligned16(q) || !aligned16(out) || !aligned16(k_pool) || !aligned16(v_pool) ||
+        !aligned16(workspace))
+        return kv_fail(KV_ERR_INVALID, "paged attention: buffers must be 16-byte aligned");
+    const int sms = device_sms();
+    int grid = sms;
+    if (opts && opts->grid_ctas > 0) grid = opts->grid_ctas;
+    const int rp = rows_padded(rows);
+    if (ws_bytes < workspace_bytes_for(grid, rp, D))
+        return kv_fail(KV_ERR_INVALID, "paged attention: workspace too small");
+    int* err = kv_error_word_ptr();
+    if (!err) return kv_fail(KV_ERR_CUDA, "paged attention: no device error word");
+
+    CUtensorMap tk, tv;
+    const uint64_t prow = (uint64_t)num_blocks * Hkv * BS;
+    int rc = pool_tmap(k_pool, prow, D, BS, &tk);
+    if (rc != KV_OK) return rc;
+    rc = pool_tmap(v_pool, prow, D, BS, &tv);
+    if (rc != KV_OK) return rc;
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    Params prm;
+    prm.q = static_cast<const __half*>(q);
+    prm.out = static_cast<__half*>(out);
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    prm.meta = reinterpret_cast<int4*>(ws);
+    size_t off = (size_t)grid * 16;
+    prm.part_lse = reinterpret_cast<float*>(ws + off);
+    off += ((size_t)grid * 2 * rp * 4 + 15) / 16 * 16;
+    prm.part_o = reinterpret_cast<float*>(ws + off);
+    prm.err = err;
+    prm.max_blocks = max_blocks_per_seq;
+    prm.B = B;
+    prm.q_len = q_len;
+    prm.Hq = Hq;
+    prm.Hkv = Hkv;
+    prm.G = G;
+    prm.rows = rows;
+    prm.num_blocks = num_blocks;
+    prm.min_share = (opts && opts->min_split_blocks > 0) ? opts->min_split_blocks : 16;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    const bool pdl = !(opts && opts->use_pdl < 0);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (D == 64) {
+        return BS == 8 ? dispatch_rows<64, 8>(rows, tk, tv, prm, grid, pdl, st)
+                       : dispatch_rows<64, 16>(rows, tk, tv, prm, grid, pdl, st);
+    }
+    return BS == 8 ? dispatch_rows<128, 8>(rows, tk, tv, prm, grid, pdl, st)
+                   : dispatch_rows<128, 16>(rows, tk, tv, prm, grid, pdl, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int paged_attention_workspace_size(int32_t Hq, int32_t Hkv, int32_t q_len, int32_t head_dim,
+                                   int32_t grid_ctas, size_t* bytes_out)
+{
+    if (!bytes_out || Hq < 1 || Hkv < 1 || Hq % Hkv || q_len < 1 ||
+        (head_dim != 64 && head_dim != 128))
+        return kv_fail(KV_ERR_INVALID, "paged_attention_workspace_size: bad arguments");
+    const int rows = (Hq / Hkv) * q_len;
+    if (rows > 16 * kMaxMT)
+        return kv_fail(KV_ERR_INVALID, "paged_attention_workspace_size: rows must be <= 32");
+    const int grid = grid_ctas > 0 ? grid_ctas : device_sms();
+    *bytes_out = workspace_bytes_for(grid, rows_padded(rows), head_dim);
+    return KV_OK;
+}
+
+int paged_decode_attention(const void* q, const void* k_pool, const void* v_pool,
+                           const int32_t* block_tables, int32_t max_blocks_per_seq,
+                           const int32_t* context_lens, float scale, void* out, int32_t B,
+                           int32_t Hq, int32_t Hkv, int32_t head_dim, int32_t block_size,
+                           int32_t num_blocks, void* workspace, size_t workspace_bytes,
+                           void* stream)
+{
+    return attention_impl(q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens, 1,
+                          scale, out, B, Hq, Hkv, head_dim, block_size, num_blocks, workspace,
+                          workspace_bytes, nullptr, stream);
+}
+
+int paged_verify_attention(const void* q, const void* k_pool, const void* v_pool,
+                           const int32_t* block_tables, int32_t max_blocks_per_seq,
+                           const int32_t* context_lens, int32_t q_len, float scale, void* out,
+                           int32_t B, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                           int32_t block_size, int32_t num_blocks, void* workspace,
+                           size_t workspace_bytes, void* stream)
+{
+    return attention_impl(q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens, q_len,
+                          scale, out, B, Hq, Hkv, head_dim, block_size, num_blocks, workspace,
+                          workspace_bytes, nullptr, stream);
+}
+
+int paged_attention_ex(const void* q, const void* k_pool, const void* v_pool,
+                       const int32_t* block_tables, int32_t max_blocks_per_seq,
+                       const int32_t* context_lens, int32_t q_len, float scale, void* out,
+                       int32_t B, int32_t Hq, int32_t Hkv, int32_t head_dim, int32_t block_size,
+                       int32_t num_blocks, void* workspace, size_t workspace_bytes,
+                       const paged_attention_opts* opts, void* stream)
+{
+    return attention_impl(q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens, q_len,
+                          scale, out, B, Hq, Hkv, head_dim, block_size, num_blocks, workspace,
+                          workspace_bytes, opts, stream);
+}
+
+}  // extern "C"

@@ -10,8 +10,20 @@ if ROOT not in sys.path:
 GOLDEN = os.path.join(ROOT, "tests", "golden")
 
 
+def _build_library():
+    """Compile libpaged_kv.so in-tree if it is missing or older than its
+    sources (nvcc cross-compiles; no GPU needed)."""
+    import importlib.util
+    path = os.path.join(ROOT, "paged_kv_cache_371_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_pkv_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
+    _build_library()
 
 
 def read_golden(name):

@@ -1,0 +1,313 @@
+"""CUDA path vs the fp64 oracle on the same seeded inputs (needs a B200).
+
+Attention: |gpu - ref| <= 2e-3 + 1e-2 |ref| elementwise; append, block copy
+and all bookkeeping: bit-exact.  Full-size configs run in the launch
+configuration the benchmark times and are checked on a sample of sequences;
+smaller cases (forced context splits, edge cases) are checked in full.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle.block_spec import BlockPoolSpec
+from paged_helpers import assert_close, device_inputs, oracle_subset
+from workloads import make_workload, normal_fp16, random_distinct_slots
+
+pytestmark = pytest.mark.gpu
+
+pkv = pytest.importorskip("paged_kv_cache_371_b200")
+
+
+@pytest.fixture(autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    pkv.device_error(reset=True)
+    yield
+    torch.cuda.synchronize()
+
+
+def _u16(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+# ----------------------------------------------------------------------------- append / copy
+
+@pytest.mark.parametrize("shape", [(16, 4, 16, 64, 2), (300, 8, 16, 128, 128), (97, 8, 8, 128, 33)])
+def test_append_bit_exact(shape):
+    nb, Hkv, bs, D, T = shape
+    K = normal_fp16((nb, Hkv, bs, D), 11, "cuda")
+    V = normal_fp16((nb, Hkv, bs, D), 12, "cuda")
+    kn = normal_fp16((T, Hkv, D), 13, "cuda")
+    vn = normal_fp16((T, Hkv, D), 14, "cuda")
+    slots = random_distinct_slots(T, nb * bs, 15)
+    slots[::5] = -1  # padding tokens
+    ref_k, ref_v = oracle.append(K.cpu().numpy(), V.cpu().numpy(), kn.cpu().numpy(),
+                                 vn.cpu().numpy(), slots)
+    pkv.paged_kv_append(kn, vn, torch.as_tensor(slots, device="cuda"), K, V)
+    assert pkv.device_error() == 0
+    assert np.array_equal(_u16(K), ref_k.view(np.uint16))
+    assert np.array_equal(_u16(V), ref_v.view(np.uint16))
+
+
+def test_append_bad_slot_is_flagged_and_skipped():
+    nb, Hkv, bs, D = 8, 2, 16, 64
+    K = normal_fp16((nb, Hkv, bs, D), 1, "cuda")
+    V = normal_fp16((nb, Hkv, bs, D), 2, "cuda")
+    K0, V0 = K.clone(), V.clone()
+    kn = normal_fp16((2, Hkv, D), 3, "cuda")
+    slots = torch.tensor([nb * bs, 3], dtype=torch.int64, device="cuda")
+    pkv.paged_kv_append(kn, kn, slots, K, V)
+    err = pkv.device_error()
+    assert err & pkv._abi.KV_DEV_BAD_SLOT
+    assert torch.equal(K.view(torch.int16)[0, :, 3], kn.view(torch.int16)[1])
+    K[0, :, 3] = K0[0, :, 3]
+    V[0, :, 3] = V0[0, :, 3]
+    assert torch.equal(K.view(torch.int16), K0.view(torch.int16))
+
+
+def test_copy_blocks_bit_exact():
+    nb, Hkv, bs, D = 64, 8, 16, 128
+    K = normal_fp16((nb, Hkv, bs, D), 21, "cuda")
+    V = normal_fp16((nb, Hkv, bs, D), 22, "cuda")
+    rng = np.random.Generator(np.random.PCG64(23))
+    perm = rng.permutation(nb)
+    pairs = np.stack([perm[:10], perm[10:20]], 1).astype(np.int32)
+    ref_k, ref_v = oracle.copy_blocks(K.cpu().numpy(), V.cpu().numpy(), pairs)
+    pkv.paged_kv_copy_blocks(K, V, torch.as_tensor(pairs, device="cuda"))
+    assert pkv.device_error() == 0
+    assert np.array_equal(_u16(K), ref_k.view(np.uint16))
+    assert np.array_equal(_u16(V), ref_v.view(np.uint16))
+
+
+# ----------------------------------------------------------------------------- decode / verify
+
+def _run(wl, q_len=1, **kw):
+    bt, cl = device_inputs(wl)
+    if kw:
+        out = pkv.paged_attention(wl.q, wl.k_pool, wl.v_pool, bt, cl, wl.scale, q_len=q_len, **kw)
+    elif q_len == 1:
+        out = pkv.paged_decode_attention(wl.q, wl.k_pool, wl.v_pool, bt, cl, wl.scale)
+    else:
+        out = pkv.paged_verify_attention(wl.q, wl.k_pool, wl.v_pool, bt, cl, wl.scale, q_len)
+    assert pkv.device_error() == 0
+    return out
+
+
+def _sample(lens, n, seed=0):
+    order = np.argsort(lens)
+    picks = {int(order[0]), int(order[-1])}
+    rng = np.random.Generator(np.random.PCG64(seed))
+    while len(picks) < min(n, len(lens)):
+        picks.add(int(rng.integers(len(lens))))
+    return sorted(picks)
+
+
+@pytest.mark.parametrize("name,n_sample", [("llama7b_mha", 6), ("llama70b_gqa", 10),
+                                           ("llama70b_gqa_bs8", 6), ("prefix_beam", 4),
+                                           ("long_decode", 2), ("long_verify", 2)])
+def test_full_size_config_sampled(name, n_sample):
+    wl = make_workload(name, "cuda")
+    q_len = wl.spec.q_len
+    out = _run(wl, q_len)
+    seqs = _sample(wl.lens, n_sample)
+    ref = oracle_subset(wl, seqs, q_len)
+    assert_close(out[torch.as_tensor(seqs, device="cuda")], ref, name)
+
+
+def test_tiny_config_full_with_append():
+    """Config 1: decode, then append one token per sequence through the block
+    manager and the append kernel, then decode again."""
+    wl = make_workload("tiny", "cuda")
+    out = _run(wl)
+    assert_close(out, oracle_subset(wl, [0, 1]), "tiny")
+
+    bs = wl.spec.bs
+    cap = wl.block_tables.shape[1] + 1
+    impl = pkv.KVPool(wl.num_blocks, bs, order=wl.order)
+    spec = BlockPoolSpec(wl.num_blocks, bs, wl.order)
+    tables = np.full((wl.B, cap), -1, np.int32)
+    nblk = np.zeros(wl.B, np.int32)
+    spec_tables = [[] for _ in range(wl.B)]
+    for s in range(wl.B):  # rebuild the existing sequences token by token
+        for t in range(int(wl.lens[s])):
+            spec.reserve_slot(spec_tables[s], t)
+            nblk[s] = impl.reserve_slot(tables[s], int(nblk[s]), t)[1]
+        assert tables[s, :nblk[s]].tolist() == wl.block_tables[s][wl.block_tables[s] >= 0].tolist()
+    slots, pairs = impl.reserve_slots(tables, nblk, wl.lens)
+    spec_slots = [spec.reserve_slot(spec_tables[s], int(wl.lens[s]))[1] for s in range(wl.B)]
+    assert slots.tolist() == spec_slots and len(pairs) == 0
+    Hkv, D = wl.spec.Hkv, wl.spec.D
+    kn = normal_fp16((wl.B, Hkv, D), 31, "cuda")
+    vn = normal_fp16((wl.B, Hkv, D), 32, "cuda")
+    ref_k, ref_v = oracle.append(wl.k_pool.cpu().numpy(), wl.v_pool.cpu().numpy(),
+                                 kn.cpu().numpy(), vn.cpu().numpy(), np.array(spec_slots))
+    pkv.paged_kv_append(kn, vn, torch.as_tensor(slots, device="cuda"), wl.k_pool, wl.v_pool)
+    assert np.array_equal(_u16(wl.k_pool), ref_k.view(np.uint16))
+    new_lens = (wl.lens + 1).astype(np.int32)
+    bt = torch.as_tensor(tables, device="cuda")
+    out2 = pkv.paged_decode_attention(wl.q, wl.k_pool, wl.v_pool, bt,
+                                      torch.as_tensor(new_lens, device="cuda"), wl.scale)
+    spec_tab = np.full((wl.B, cap), -1, np.int32)
+    for s in range(wl.B):
+        spec_tab[s, :len(spec_tables[s])] = spec_tables[s]
+    ref2 = oracle.paged_attention(wl.q.cpu().numpy(), ref_k, ref_v, spec_tab, new_lens,
+                                  scale=wl.scale)
+    assert_close(out2, ref2, "tiny after append")
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,bs,q_len", [
+    (4, 4, 64, 16, 1), (8, 8, 128, 8, 1),           # FMA path (one row per KV head)
+    (8, 2, 64, 16, 1), (64, 8, 128, 16, 1),          # tensor-core path, one m16 tile
+    (32, 8, 128, 8, 5), (16, 2, 128, 16, 4),         # verify windows, two m16 tiles
+    (4, 4, 128, 16, 3), (6, 2, 64, 8, 1)])
+@pytest.mark.parametrize("grid,min_split", [(0, 0), (300, 1), (7, 1)])
+def test_forced_splits_full_compare(Hq, Hkv, D, bs, q_len, grid, min_split):
+    """Oracle-sized problems over several tiles and ragged tails, with the
+    context split across many CTAs (merge path) or few CTAs (long runs)."""
+    rng = np.random.Generator(np.random.PCG64(Hq * 131 + D + bs + q_len))
+    B = 5
+    lens = np.array([1, bs, 3 * bs + 1, 200, 411], dtype=np.int32)
+    lens = np.maximum(lens, q_len)
+    wl = make_workload("llama70b_gqa", "cuda", lens=lens, bs=bs, q_len=q_len, Hq=Hq, Hkv=Hkv, D=D,
+                       seed=int(rng.integers(1 << 30)))
+    out = _run(wl, q_len, grid_ctas=grid, min_split_blocks=min_split)
+    ref = oracle_subset(wl, list(range(B)), q_len)
+    assert_close(out, ref, f"Hq{Hq} Hkv{Hkv} D{D} bs{bs} q{q_len} grid{grid}")
+
+
+def test_edge_cases():
+    """Empty context (zeros), one token (exactly V), exact block multiples,
+    a window longer than the context (zeros for rows that see nothing)."""
+    lens = np.array([0, 1, 16, 17, 32, 2], dtype=np.int32)
+    wl = make_workload("llama70b_gqa", "cuda", lens=lens, q_len=1, seed=77, Hq=8, Hkv=2, D=128)
+    out = _run(wl, 1, grid_ctas=5, min_split_blocks=1)
+    ref = oracle_subset(wl, list(range(len(lens))))
+    assert_close(out, ref, "edge decode")
+    assert not out[0].any()
+    # one token: softmax weight exactly 1, output bit-exactly V (fp16)
+    v0 = wl.v_pool[int(wl.block_tables[1, 0]), :, 0, :]  # [Hkv][D]
+    G = 8 // 2
+    exp = v0.repeat_interleave(G, dim=0)
+    assert torch.equal(out[1, 0].view(torch.int16), exp.view(torch.int16))
+    # verify window of 3 over contexts of 2 and 1 tokens: rows past the context see nothing
+    wl.q = normal_fp16((len(lens), 3, 8, 128), 5, "cuda")
+    out3 = _run(wl, 3, grid_ctas=3)
+    ref3 = oracle_subset(wl, list(range(len(lens))), q_len=3)
+    assert_close(out3, ref3, "edge verify")
+
+
+def test_permutation_invariance_bit_exact():
+    """Moving blocks to other physical ids (same work split) changes no bit."""
+    wl = make_workload("llama70b_gqa", "cuda", B=24, max_len=700, seed=5)
+    out = _run(wl).clone()
+    rng = np.random.Generator(np.random.PCG64(6))
+    perm = rng.permutation(wl.num_blocks)
+    pt = torch.as_tensor(perm, device="cuda", dtype=torch.long)
+    k2 = torch.empty_like(wl.k_pool)
+    v2 = torch.empty_like(wl.v_pool)
+    k2[pt] = wl.k_pool
+    v2[pt] = wl.v_pool
+    t2 = np.where(wl.block_tables >= 0, perm[np.maximum(wl.block_tables, 0)], -1).astype(np.int32)
+    wl.k_pool, wl.v_pool, wl.block_tables = k2, v2, t2
+    out2 = _run(wl)
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+
+
+def test_bad_block_id_is_flagged_without_fault():
+    wl = make_workload("llama70b_gqa", "cuda", B=6, max_len=300, seed=8)
+    wl.block_tables[2, 1] = wl.num_blocks + 5
+    bt, cl = device_inputs(wl)
+    out = pkv.paged_decode_attention(wl.q, wl.k_pool, wl.v_pool, bt, cl, wl.scale)
+    err = pkv.device_error()
+    assert err & pkv._abi.KV_DEV_BAD_BLOCK
+    others = [0, 1, 3, 4, 5]
+    assert_close(out[torch.as_tensor(others, device="cuda")], oracle_subset(wl, others),
+                 "untouched sequences")
+
+
+# ----------------------------------------------------------------------------- prefix + beams
+
+@pytest.mark.parametrize("fork_len", [1024, 1030])
+def test_prefix_sharing_and_beam_copy_on_write(fork_len):
+    """Config 4: 64 requests share a 2048-token prefix (refcount 64); 4 beams
+    forked at fork_len each append one token; a shared partial last block is
+    copied on write.  Bookkeeping and pools bit-exact, attention within
+    tolerance."""
+    wl = make_workload("prefix_beam", "cuda", spare_blocks=600)
+    bs, Hkv, D = wl.spec.bs, wl.spec.Hkv, wl.spec.D
+    nb = wl.num_blocks
+    cap = wl.block_tables.shape[1] + 2
+    impl = pkv.KVPool(nb, bs, order=wl.order)
+    spec = BlockPoolSpec(nb, bs, wl.order)
+    P = wl.extra["prefix_blocks"]
+    # request 0 builds the prefix, the others fork it, then each grows its suffix
+    t_impl = np.full((wl.B, cap), -1, np.int32)
+    n_impl = np.zeros(wl.B, np.int32)
+    t_spec = [[] for _ in range(wl.B)]
+    for t in range(P * bs):
+        spec.reserve_slot(t_spec[0], t)
+        n_impl[0] = impl.reserve_slot(t_impl[0], int(n_impl[0]), t)[1]
+    for s in range(1, wl.B):
+        spec.fork(t_spec[0][:P])
+        impl.fork(t_impl[0, :P])
+        t_spec[s] = list(t_spec[0][:P])
+        t_impl[s, :P] = t_impl[0, :P]
+        n_impl[s] = P
+    for s in range(wl.B):
+        for t in range(P * bs, int(wl.lens[s])):
+            spec.reserve_slot(t_spec[s], t)
+            n_impl[s] = impl.reserve_slot(t_impl[s], int(n_impl[s]), t)[1]
+        assert t_impl[s, :n_impl[s]].tolist() == t_spec[s]
+        assert t_spec[s] == wl.block_tables[s][wl.block_tables[s] >= 0].tolist()
+    assert impl.refcount(t_spec[0][0]) == wl.B == spec.refcount[t_spec[0][0]]
+    out = _run(wl)
+    seqs = [0, 17, 63]
+    assert_close(out[torch.as_tensor(seqs, device="cuda")], oracle_subset(wl, seqs), "prefix")
+
+    # beams: a parent of fork_len tokens, 3 forks -> 4 beams sharing every block
+    parent_spec, parent_impl = [], np.full(cap, -1, np.int32)
+    npar = 0
+    for t in range(fork_len):
+        spec.reserve_slot(parent_spec, t)
+        npar = impl.reserve_slot(parent_impl, npar, t)[1]
+    # the parent's blocks came off the free list (poisoned): give them data
+    pid = torch.as_tensor(parent_impl[:npar], device="cuda", dtype=torch.long)
+    wl.k_pool[pid] = normal_fp16((npar, Hkv, bs, D), 44, "cuda")
+    wl.v_pool[pid] = normal_fp16((npar, Hkv, bs, D), 45, "cuda")
+    beams_spec = [parent_spec] + [list(parent_spec) for _ in range(3)]
+    beams_impl = np.full((4, cap), -1, np.int32)
+    for b in range(4):
+        beams_impl[b, :npar] = parent_impl[:npar]
+        if b:
+            spec.fork(parent_spec)
+            impl.fork(parent_impl[:npar])
+    nbeam = np.full(4, npar, np.int32)
+    lens4 = np.full(4, fork_len, np.int32)
+    slots, pairs = impl.reserve_slots(beams_impl, nbeam, lens4)
+    exp = [spec.reserve_slot(beams_spec[b], fork_len) for b in range(4)]
+    assert slots.tolist() == [e[1] for e in exp]
+    exp_pairs = [(e[2], e[3]) for e in exp if e[2] >= 0]
+    assert [tuple(p) for p in pairs.tolist()] == exp_pairs
+    assert len(exp_pairs) == (0 if fork_len % bs == 0 else 3)
+    kn = normal_fp16((4, Hkv, D), 41, "cuda")
+    vn = normal_fp16((4, Hkv, D), 42, "cuda")
+    Kh, Vh = wl.k_pool.cpu().numpy(), wl.v_pool.cpu().numpy()
+    if exp_pairs:
+        Kh, Vh = oracle.copy_blocks(Kh, Vh, np.array(exp_pairs, np.int32))
+        pkv.paged_kv_copy_blocks(wl.k_pool, wl.v_pool, torch.as_tensor(pairs, device="cuda"))
+    Kh, Vh = oracle.append(Kh, Vh, kn.cpu().numpy(), vn.cpu().numpy(), np.array([e[1] for e in exp]))
+    pkv.paged_kv_append(kn, vn, torch.as_tensor(slots, device="cuda"), wl.k_pool, wl.v_pool)
+    assert pkv.device_error() == 0
+    assert np.array_equal(_u16(wl.k_pool), Kh.view(np.uint16))
+    assert np.array_equal(_u16(wl.v_pool), Vh.view(np.uint16))
+    qb = normal_fp16((4, 1, wl.spec.Hq, D), 43, "cuda")
+    L4 = lens4 + 1
+    outb = pkv.paged_decode_attention(qb, wl.k_pool, wl.v_pool, torch.as_tensor(beams_impl, device="cuda"),
+                                      torch.as_tensor(L4, device="cuda"), wl.scale)
+    tb = np.full((4, cap), -1, np.int32)
+    for b in range(4):
+        tb[b, :len(beams_spec[b])] = beams_spec[b]
+    ref = oracle.paged_attention(qb.cpu().numpy(), Kh, Vh, tb, L4, scale=wl.scale)
+    assert_close(outb, ref, f"beams forked at {fork_len}")

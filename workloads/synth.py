@@ -142,8 +142,10 @@ def _ceil_div(a, b):
 def make_workload(name: str, device="cpu", *, B: Optional[int] = None,
                   max_len: Optional[int] = None, lens=None, bs: Optional[int] = None,
                   q_len: Optional[int] = None, seed: Optional[int] = None,
+                  Hq: Optional[int] = None, Hkv: Optional[int] = None, D: Optional[int] = None,
                   spare_blocks: int = 0, poison: bool = True) -> Workload:
-    """Build config ``name``; the keyword overrides shrink it for oracle-sized runs.
+    """Build config ``name``; the keyword overrides shrink or reshape it for
+    oracle-sized runs.
 
     ``spare_blocks`` adds free blocks beyond the config's pool (room to append).
     """
@@ -186,7 +188,9 @@ def make_workload(name: str, device="cpu", *, B: Optional[int] = None,
         nxt += private[s]
 
     dev = torch.device(device)
-    Hq, Hkv, D = spec.Hq, spec.Hkv, spec.D
+    Hq = spec.Hq if Hq is None else Hq
+    Hkv = spec.Hkv if Hkv is None else Hkv
+    D = spec.D if D is None else D
     q = normal_fp16((B, q_len, Hq, D), seed * 1000 + 1, dev)
     k_pool = torch.empty((num_blocks, Hkv, bs, D), dtype=torch.float16, device=dev)
     v_pool = torch.empty_like(k_pool)
