@@ -42,13 +42,15 @@ CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.ac
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="use only the first B sequences of the workload (profiling runs)")
     return ap.parse_args(argv)
 
 
@@ -112,50 +114,68 @@ def ncu_traffic(workload):
 
 
 class ClockSampler:
-    def __init__(self, gpu_index):
-        self.proc = None
-        self.gpu = gpu_index
+    """Samples SM clock, max clock and throttle reasons every ~1 ms through
+    NVML while the timed region runs (nvidia-smi's 200 ms period is longer
+    than a short timed region)."""
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.samples = []
+        self.max_mhz = None
+        self._stop = None
+
+    def _handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            idx = int(vis.split(",")[self.dev]) if vis else self.dev
+            return pynvml.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self, h):
+        import pynvml
+        while not self._stop.is_set():
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, rs))
+            except Exception:
+                pass
+            time.sleep(0.001)
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={CLOCK_QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import pynvml
+            h = self._handle()
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self._stop = threading.Event()
+            self._t = threading.Thread(target=self._run, args=(h,), daemon=True)
+            self._t.start()
         except Exception:
-            self.proc = None
+            self._stop = None
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except Exception:
-                self.proc.kill()
-                out = ""
-            self.lines = [l for l in out.splitlines() if l.strip()]
+        if self._stop is not None:
+            self._stop.set()
+            self._t.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in getattr(self, "lines", []):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "source": "nvml"}
+        reasons = sorted(n for n, bit in self.REASONS.items()
+                         if any(r & bit for _, r in self.samples))
+        return {"sm_mhz": statistics.median(sm for sm, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples),
+                "source": "nvml, 1 ms polling during the timed steps"}
 
 
 # ---------------------------------------------------------------------------
@@ -234,7 +254,7 @@ def run_ours(args):
     from workloads.synth import CONFIGS
     spec = CONFIGS[args.workload]
     seed = rank_seed(spec.seed, rank)
-    wl = make_workload(args.workload, device, seed=seed)
+    wl = make_workload(args.workload, device, seed=seed, B=args.batch or None)
     q_len = spec.q_len
     Hq, Hkv, D, bs = spec.Hq, spec.Hkv, spec.D, spec.bs
     n_distinct = min(args.warmup + args.steps, 64)
@@ -274,9 +294,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
-    phys = vis.split(",")[local] if vis and len(vis.split(",")) > local else str(local)
-    with ClockSampler(phys) as clk:
+    with ClockSampler(local) as clk:
         for k in range(args.steps):
             i = args.warmup + k
             st = steps[i % n_distinct]
@@ -325,7 +343,8 @@ def run_ours(args):
             "ms_per_step": round(t_all / args.steps, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
             "config": {
-                "workload": args.workload, "description": spec.description, "B": wl.B,
+                "workload": args.workload + (f"[B={wl.B}]" if args.batch else ""),
+                "description": spec.description, "B": wl.B,
                 "Hq": Hq, "Hkv": Hkv, "head_dim": D, "block_size": bs, "q_len": q_len,
                 "mean_context": float(np.mean(wl.lens)),
                 "step": "copy-on-write copies + append 1 token/sequence + paged attention + merge",
@@ -344,8 +363,10 @@ def run_ours(args):
         }
         if e2e:
             result["e2e"] = e2e
-        if world == 1:
-            result["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
+        if world == 1 and args.cpu_seconds > 0:
+            # the timed appends only wrote slots past each sequence's original
+            # length, so the workload's original tokens are still in the pools
+            result["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
     if world > 1:
         dist.destroy_process_group()
     return result
@@ -435,16 +456,38 @@ def time_oracle(wl):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(workload, target_s):
+def host_copy(wl):
+    """The workload's inputs as host arrays: only the blocks the tables use,
+    renumbered (plain data movement)."""
+    import numpy as np
+    import torch
+    tables = wl.block_tables
+    ids = np.unique(tables[tables >= 0])
+    idx = torch.as_tensor(ids, device=wl.k_pool.device, dtype=torch.long)
+    K = wl.k_pool[idx].cpu().numpy()
+    V = wl.v_pool[idx].cpu().numpy()
+    t2 = np.where(tables >= 0, np.searchsorted(ids, np.maximum(tables, 0)), -1).astype(np.int32)
+    return wl.q.cpu().numpy(), K, V, t2
+
+
+def cpu_baseline(wl, target_s):
+    """The oracle, as it stands, over the whole workload of this run (its
+    sequences, blocks and queries copied to the host), repeated until about
+    target_s seconds of CPU time have been spent."""
     import oracle
-    wl = oracle_sample(workload, target_s)
-    dt = time_oracle(wl)
+    q, K, V, t2 = host_copy(wl)
     s = wl.spec
-    kvb = algorithmic_bytes(wl.lens, s.Hq, s.Hkv, s.D, s.bs, s.q_len)[0]
-    return {"value": round(kvb / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
-            "sample": f"{wl.B} of {s.B} sequences of {workload} (same length recipe), "
-                      f"{int(wl.lens.sum())} tokens, fp64 C oracle, {dt:.2f} s"}
+    reps, spent = 0, 0.0
+    while reps == 0 or spent < target_s:
+        t0 = time.perf_counter()
+        oracle.paged_attention(q, K, V, t2, wl.lens, scale=wl.scale, q_len=q.shape[1])
+        spent += time.perf_counter() - t0
+        reps += 1
+    kvb = algorithmic_bytes(wl.lens, q.shape[2], s.Hkv, q.shape[3], s.bs, q.shape[1])[0]
+    return {"value": round(kvb * reps / spent / 1e9, 4), "unit": "GB/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"whole workload of this run ({wl.B} sequences, {int(wl.lens.sum())} "
+                      f"tokens) x {reps} repeat(s), fp64 C oracle, {spent:.2f} s"}
 
 
 def run_reference(args):

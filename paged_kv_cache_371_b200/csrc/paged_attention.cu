@@ -81,20 +81,27 @@ struct Cfg {
     static constexpr int RP = FMA ? 1 : 16 * MT;            // padded rows
     static constexpr int NCW = FMA ? kTokWarps : kTokWarps * MT;
     static constexpr int THREADS = (NCW + 1) * 32;
+    // registers per thread for one CTA per SM: warps are spread over the 4
+    // SM sub-partitions, each with a 16K-register file
+    static constexpr int WARPS_PER_SUBPART = (THREADS / 32 + 3) / 4;
+    static constexpr int MAXREG_RAW = (16384 / (32 * WARPS_PER_SUBPART)) / 8 * 8;
+    static constexpr int MAXREG = MAXREG_RAW > 255 ? 255 : MAXREG_RAW;
+    static constexpr int TILE_BYTES = BS * D * 2;           // one (block, kv-head) tile
     static constexpr int KV_BYTES = kTS * D * 2;            // K (or V) bytes per stage
     static constexpr int Q_BYTES = (RP * D * 2 + 1023) / 1024 * 1024;
     static constexpr int STAGE_BYTES = 2 * KV_BYTES + Q_BYTES;
     static constexpr int OB_STRIDE = D + 8;                 // floats per obuf row
     static constexpr int OBUF_BYTES = RP * OB_STRIDE * 4;
     static constexpr int ML_BYTES = kTokWarps * RP * 2 * 4;
-    static constexpr int FIXED = OBUF_BYTES + ML_BYTES + 128 + 16 * 64;
+    static constexpr int FIXED = OBUF_BYTES + ML_BYTES + 256 + 16 * 64;
     static constexpr int STAGES_RAW = (kSmemBudget - FIXED) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
     static_assert(STAGES >= 2, "not enough shared memory for two stages");
     static constexpr int META_OFF = STAGES * STAGE_BYTES;   // StageMeta[STAGES]
     static constexpr int BAR_OFF = META_OFF + STAGES * 32;  // full[S], empty[S]
     static constexpr int ZERO_OFF = BAR_OFF + STAGES * 16;  // 128 zero bytes
-    static constexpr int ML_OFF = ZERO_OFF + 128;
+    static constexpr int PB_OFF = ZERO_OFF + 128;           // per-warp fp16 weights (FMA path)
+    static constexpr int ML_OFF = PB_OFF + 128;
     static constexpr int OBUF_OFF = ML_OFF + ML_BYTES;
     static constexpr int SMEM_USED = OBUF_OFF + OBUF_BYTES;
     static constexpr int SMEM_ALLOC = SMEM_USED + 1024;    // room to align the base
@@ -130,15 +137,128 @@ __device__ __forceinline__ int64_t warp_incl_scan64(int64_t v, int lane)
     return v;
 }
 
-// Swizzled address of 16-byte chunk `c` (0..7) of row `row` in a TMA box of
-// 64 fp16 columns written with 128-byte swizzle (box base 1024-aligned).
-__device__ __forceinline__ uint32_t swz(uint32_t box_base, int row, int c)
+// Shared-memory layout of a staged tile: one (block, kv-head) tile is its
+// BS rows of D fp16, i.e. BS * NH units of 128 bytes in global order (one TMA
+// copy of the contiguous tile).  The 128-byte swizzle stores 16-byte chunk c
+// of unit u at chunk position c ^ (u mod 8).  Byte offset, inside a stage's K
+// (or V) area, of chunk cg (0 .. D/8-1) of stage token `tok`:
+template <class C>
+__device__ __forceinline__ uint32_t tile_chunk(int tok, int cg)
 {
-    return box_base + row * 128 + ((c ^ (row & 7)) << 4);
+    const int r = tok % C::BS;
+    const int u = r * C::NH + (cg >> 3);
+    return (uint32_t)((tok / C::BS) * C::TILE_BYTES + u * 128 + (((cg & 7) ^ (u & 7)) << 4));
+}
+
+// One TMA copy of the tile whose first row is `y` in the pool's row space.
+template <int NH>
+__device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap* tm, int32_t y,
+                                              uint32_t bar, uint64_t pol)
+{
+    if constexpr (NH == 1)
+        tma_load_2d(dst, tm, 0, y, bar, pol);
+    else
+        tma_load_3d(dst, tm, 0, 0, y, bar, pol);
 }
 
 // ---------------------------------------------------------------------------
 // Producer warp: walks this CTA's run of units and feeds the stage ring.
+//
+// Block-table entries are loaded one batch of kLA stages ahead of the stage
+// being issued, so the table's load latency overlaps the copies in flight
+// instead of sitting in front of every TMA issue.
+constexpr int kLA = 4;  // stages per look-ahead batch
+
+struct StageDesc {
+    int32_t s, kvh, b, nbl, t0, ntok, L, flags, slot;
+};
+
+// Walks (sequence, kv-head, block) units of one CTA's run and cuts them into
+// stages of at most NBS blocks that never cross a (sequence, kv-head).
+template <class C>
+struct UnitWalker {
+    const Params* p;
+    int lane;
+    int64_t u, u1, share, seq_start;
+    int32_t s, L, nb;
+    int32_t kvh, b, b1, slot;
+    bool whole, in_seg, first_seg, seg_first_stage;
+    int32_t win_base, win_len;  // lane i holds context_lens[win_base + i]
+    int4 merge_meta;            // what the merge kernel needs from this CTA
+
+    __device__ int32_t len_of(int32_t seq)
+    {
+        if (seq >= win_base + 32 || seq < win_base) {
+            win_base = seq;
+            win_len = seq + lane < p->B ? __ldg(p->context_lens + seq + lane) : 0;
+        }
+        return __shfl_sync(0xffffffffu, win_len, seq - win_base);
+    }
+
+    __device__ void enter_sequence(int32_t seq)
+    {
+        s = seq;
+        const int32_t Lraw = len_of(seq);
+        L = clamp_len(Lraw, C::BS, p->max_blocks);
+        nb = nblk_of(Lraw, C::BS, p->max_blocks);
+        if (lane == 0 && Lraw > L) atomicOr(p->err, KV_DEV_BAD_BLOCK);
+    }
+
+    // Next stage of the run; false when the run is exhausted.
+    __device__ bool next(StageDesc& d)
+    {
+        if (!in_seg) {
+            if (u >= u1) return false;
+            const int64_t local = u - seq_start;
+            kvh = (int32_t)(local / nb);
+            b = (int32_t)(local % nb);
+            const int64_t kv_end = seq_start + (int64_t)(kvh + 1) * nb;
+            const int64_t seg_end = u1 < kv_end ? u1 : kv_end;
+            b1 = b + (int32_t)(seg_end - u);
+            whole = b == 0 && b1 == nb;
+            slot = first_seg ? 0 : 1;
+            if (first_seg && b > 0 && b1 == nb) {
+                const int64_t gstart = seq_start + (int64_t)kvh * nb;
+                merge_meta = make_int4(s, kvh, (int32_t)(gstart / share), (gstart % share) ? 1 : 0);
+            }
+            first_seg = false;
+            in_seg = true;
+            seg_first_stage = true;
+        }
+        const int32_t nbl = (b1 - b) < C::NBS ? (b1 - b) : C::NBS;
+        d.s = s;
+        d.kvh = kvh;
+        d.b = b;
+        d.nbl = nbl;
+        d.t0 = b * C::BS;
+        int32_t tend = (b + nbl) * C::BS;
+        if (tend > L) tend = L;
+        d.ntok = tend > d.t0 ? tend - d.t0 : 0;
+        d.L = L;
+        d.flags = (seg_first_stage ? F_FIRST : 0) | (b + nbl >= b1 ? F_LAST : 0) |
+                  (whole ? F_WHOLE : 0);
+        d.slot = slot;
+        seg_first_stage = false;
+        b += nbl;
+        u += nbl;
+        if (b >= b1) {
+            in_seg = false;
+            if (u < u1 && u == seq_start + (int64_t)nb * p->Hkv) {
+                seq_start = u;
+                enter_sequence(s + 1);
+            }
+        }
+        return true;
+    }
+};
+
+// Number of units (blocks x KV heads) of sequence s.
+template <class C>
+__device__ __forceinline__ int64_t units_of(const Params& p, int32_t Lraw)
+{
+    return (int64_t)nblk_of(Lraw, C::BS, p.max_blocks) * p.Hkv;
+}
+
 template <class C>
 __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const Params& p,
                          uint8_t* smem, volatile int* abort_flag)
@@ -154,13 +274,17 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
         prefetch_tmap(tmV);
     }
 
-    // Pass 1: total units.
+    // Pass 1: total units.  Each lane takes 8 consecutive sequences of a
+    // 256-sequence chunk; all loads of a chunk are in flight together.
     int64_t total = 0;
-    for (int base = 0; base < p.B; base += 32) {
-        const int s = base + lane;
-        int64_t u = 0;
-        if (s < p.B) u = (int64_t)nblk_of(__ldg(p.context_lens + s), C::BS, p.max_blocks) * p.Hkv;
-        total += warp_sum64(u);
+    for (int base = 0; base < p.B; base += 256) {
+        int64_t sum = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int s = base + lane * 8 + j;
+            if (s < p.B) sum += units_of<C>(p, __ldg(p.context_lens + s));
+        }
+        total += warp_sum64(sum);
     }
     const int64_t G = gridDim.x;
     int64_t share = (total + G - 1) / G;
@@ -168,57 +292,89 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
     const int64_t u0 = (int64_t)blockIdx.x * share;
     const int64_t u1 = u0 + share < total ? u0 + share : total;
 
-    int4 my_meta = make_int4(-1, 0, 0, 0);
-    int k_issued = 0;  // stages issued so far
+    UnitWalker<C> w;
+    w.p = &p;
+    w.lane = lane;
+    w.merge_meta = make_int4(-1, 0, 0, 0);
+    w.win_base = -64;
+    w.win_len = 0;
     bool ok = true;
+    int k_issued = 0;  // stages issued so far (the end marker included)
 
     if (u0 < u1) {
         // Pass 2: the sequence holding unit u0.
-        int s = -1;
-        int64_t seq_start = 0, run = 0;
-        for (int base = 0; base < p.B && s < 0; base += 32) {
-            const int sl = base + lane;
-            int64_t u = 0;
-            if (sl < p.B) u = (int64_t)nblk_of(__ldg(p.context_lens + sl), C::BS, p.max_blocks) * p.Hkv;
-            const int64_t incl = warp_incl_scan64(u, lane);
-            const bool hit = sl < p.B && run + incl > u0 && run + incl - u <= u0;
+        int s0 = -1;
+        int64_t start0 = 0, run = 0;
+        for (int base = 0; base < p.B && s0 < 0; base += 256) {
+            int64_t uu[8];
+            int64_t sum = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int s = base + lane * 8 + j;
+                uu[j] = s < p.B ? units_of<C>(p, __ldg(p.context_lens + s)) : 0;
+                sum += uu[j];
+            }
+            const int64_t incl = warp_incl_scan64(sum, lane);
+            const int64_t excl = run + incl - sum;
+            const bool hit = excl <= u0 && u0 < excl + sum;
             const unsigned m = __ballot_sync(0xffffffffu, hit);
             if (m) {
                 const int src = __ffs(m) - 1;
-                s = base + src;
-                seq_start = run + __shfl_sync(0xffffffffu, incl - u, src);
+                int64_t acc = excl;
+                int found = -1;
+                int64_t fstart = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (found < 0 && uu[j] > 0 && acc <= u0 && u0 < acc + uu[j]) {
+                        found = base + lane * 8 + j;
+                        fstart = acc;
+                    }
+                    acc += uu[j];
+                }
+                s0 = __shfl_sync(0xffffffffu, found, src);
+                start0 = __shfl_sync(0xffffffffu, fstart, src);
             }
             run += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (s < 0) {  // unreachable when u0 < total; keeps the walk well defined
-            s = 0;
+        if (s0 < 0) {  // unreachable when u0 < total; keeps the walk well defined
+            s0 = 0;
             ok = false;
         }
-        int32_t Lraw = __ldg(p.context_lens + s);
-        int32_t L = clamp_len(Lraw, C::BS, p.max_blocks);
-        if (lane == 0 && Lraw > L) atomicOr(p.err, KV_DEV_BAD_BLOCK);
-        int32_t nb = nblk_of(Lraw, C::BS, p.max_blocks);
-        int64_t u = u0;
-        bool first_seg = true;
-        while (u < u1 && ok) {
-            const int64_t local = u - seq_start;
-            const int32_t kvh = (int32_t)(local / nb);
-            const int32_t b0 = (int32_t)(local % nb);
-            const int64_t kv_end = seq_start + (int64_t)(kvh + 1) * nb;
-            const int64_t seg_end = u1 < kv_end ? u1 : kv_end;
-            const int32_t b1 = b0 + (int32_t)(seg_end - u);
-            const bool whole = b0 == 0 && b1 == nb;
-            const int32_t slot = first_seg ? 0 : 1;
-            if (first_seg && b0 > 0 && b1 == nb) {
-                const int64_t gstart = seq_start + (int64_t)kvh * nb;
-                my_meta = make_int4(s, kvh, (int32_t)(gstart / share), (gstart % share) ? 1 : 0);
+        w.u = u0;
+        w.u1 = ok ? u1 : u0;
+        w.share = share;
+        w.seq_start = start0;
+        w.in_seg = false;
+        w.first_seg = true;
+        w.seg_first_stage = false;
+        w.enter_sequence(s0);
+
+        // block id of block `lane` of a stage (-1: nothing to load)
+        auto load_id = [&](const StageDesc& d) -> int32_t {
+            if (lane < d.nbl && d.t0 + lane * C::BS < d.L)
+                return __ldg(p.block_tables + (int64_t)d.s * p.max_blocks + d.b + lane);
+            return -1;
+        };
+        StageDesc cur[kLA], nxt[kLA];
+        int32_t cid[kLA], nid[kLA];
+        int ncur = 0, nnxt = 0;
+#pragma unroll
+        for (int k = 0; k < kLA; ++k)
+            if (ncur == k && w.next(cur[k])) {
+                cid[k] = load_id(cur[k]);
+                ++ncur;
             }
-            for (int32_t b = b0; b < b1; b += C::NBS) {
-                const int32_t nbl = (b1 - b) < C::NBS ? (b1 - b) : C::NBS;
-                const int32_t t0 = b * C::BS;
-                int32_t tend = (b + nbl) * C::BS;
-                if (tend > L) tend = L;
-                const int32_t ntok = tend > t0 ? tend - t0 : 0;
+#pragma unroll
+        for (int k = 0; k < kLA; ++k)
+            if (nnxt == k && w.next(nxt[k])) {
+                nid[k] = load_id(nxt[k]);
+                ++nnxt;
+            }
+        while (ncur > 0 && ok) {
+#pragma unroll
+            for (int k = 0; k < kLA; ++k) {
+                if (k >= ncur || !ok) break;
+                const StageDesc& d = cur[k];
                 const int stage = k_issued % C::STAGES;
                 const int round = k_issued / C::STAGES;
                 if (round > 0) {
@@ -228,62 +384,59 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
                         break;
                     }
                 }
-                // block ids of this stage, one per lane
-                int32_t id = -1;
-                const bool has_tok = lane < nbl && t0 + lane * C::BS < L;
-                if (has_tok) id = __ldg(p.block_tables + (int64_t)s * p.max_blocks + b + lane);
+                const int32_t id = cid[k];
+                const bool has_tok = lane < d.nbl && d.t0 + lane * C::BS < d.L;
                 const bool bad = has_tok && (id < 0 || id >= p.num_blocks);
                 const bool load = has_tok && !bad;
                 const unsigned lmask = __ballot_sync(0xffffffffu, load);
                 if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, KV_DEV_BAD_BLOCK);
-                const bool firstst = b == b0;
+                const bool firstst = (d.flags & F_FIRST) != 0;
                 const uint32_t qbytes = (uint32_t)(p.G * C::D * 2);
                 uint32_t bytes = (uint32_t)__popc(lmask) * (uint32_t)(2 * C::BS * C::D * 2);
                 if (firstst) bytes += qbytes * (uint32_t)p.q_len;
                 const uint32_t full = full0 + stage * 8;
                 if (lane == 0) {
                     StageMeta& md = smeta[stage];
-                    md.s = s;
-                    md.kvh = kvh;
-                    md.t0 = t0;
-                    md.ntok = ntok;
-                    md.L = L;
-                    md.flags = (firstst ? F_FIRST : 0) | (b + C::NBS >= b1 ? F_LAST : 0) |
-                               (whole ? F_WHOLE : 0);
-                    md.slot = slot;
+                    md.s = d.s;
+                    md.kvh = d.kvh;
+                    md.t0 = d.t0;
+                    md.ntok = d.ntok;
+                    md.L = d.L;
+                    md.flags = d.flags;
+                    md.slot = d.slot;
                     mbar_arrive_expect_tx(full, bytes);
                 }
                 __syncwarp();
                 const uint32_t st = sbase + stage * C::STAGE_BYTES;
                 if (load) {
-                    const int32_t y = (id * p.Hkv + kvh) * C::BS;
-#pragma unroll
-                    for (int h = 0; h < C::NH; ++h) {
-                        const uint32_t off = (uint32_t)((lane * C::NH + h) * C::BS * 128);
-                        tma_load_2d(st + off, tmK, h * 64, y, full, pol);
-                        tma_load_2d(st + C::KV_BYTES + off, tmV, h * 64, y, full, pol);
-                    }
+                    const int32_t y = (id * p.Hkv + d.kvh) * C::BS;
+                    const uint32_t off = (uint32_t)(lane * C::TILE_BYTES);
+                    tma_load_tile<C::NH>(st + off, tmK, y, full, pol);
+                    tma_load_tile<C::NH>(st + C::KV_BYTES + off, tmV, y, full, pol);
                 }
                 if (firstst && lane < p.q_len) {
                     const __half* src =
-                        p.q + (((int64_t)s * p.q_len + lane) * p.Hq + (int64_t)kvh * p.G) * C::D;
+                        p.q + (((int64_t)d.s * p.q_len + lane) * p.Hq + (int64_t)d.kvh * p.G) * C::D;
                     bulk_load(st + 2 * C::KV_BYTES + lane * qbytes, src, qbytes, full);
                 }
                 ++k_issued;
             }
-            first_seg = false;
-            u = seg_end;
-            if (u < u1 && u == seq_start + (int64_t)nb * p.Hkv) {
-                seq_start = u;
-                ++s;
-                Lraw = __ldg(p.context_lens + s);
-                L = clamp_len(Lraw, C::BS, p.max_blocks);
-                if (lane == 0 && Lraw > L) atomicOr(p.err, KV_DEV_BAD_BLOCK);
-                nb = nblk_of(Lraw, C::BS, p.max_blocks);
+#pragma unroll
+            for (int k = 0; k < kLA; ++k) {
+                cur[k] = nxt[k];
+                cid[k] = nid[k];
             }
+            ncur = nnxt;
+            nnxt = 0;
+#pragma unroll
+            for (int k = 0; k < kLA; ++k)
+                if (nnxt == k && w.next(nxt[k])) {
+                    nid[k] = load_id(nxt[k]);
+                    ++nnxt;
+                }
         }
     }
-    if (lane == 0) p.meta[blockIdx.x] = my_meta;
+    if (lane == 0) p.meta[blockIdx.x] = w.merge_meta;
 
     // End marker.
     if (ok) {
@@ -401,10 +554,6 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
     const int v_i = ((lane >> 3) & 1) * 8 + (lane & 7);         // V: token within my 16
     const int v_tok = qw * 16 + v_i;
     const int v_sel = lane >> 4;
-    const uint32_t k_row_off = (uint32_t)(((k_tok / C::BS) * C::NH * C::BS + (k_tok % C::BS)) * 128);
-    const uint32_t v_row_off = (uint32_t)(((v_tok / C::BS) * C::NH * C::BS + (v_tok % C::BS)) * 128);
-    const int k_x = k_tok % C::BS & 7;
-    const int v_x = v_tok % C::BS & 7;
 
     float O[C::D / 8][4];
     uint32_t qa[C::D / 16][4];
@@ -448,21 +597,23 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
             float S[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
             for (int ks = 0; ks < C::D / 16; ++ks) {
-                const int h = ks / 4;
-                const int c = (2 * ks) % 8 + k_sel;
                 uint32_t b0, b1, b2, b3;
-                ldsm_x4(st + k_row_off + h * C::BS * 128 + ((c ^ k_x) << 4), b0, b1, b2, b3);
+                ldsm_x4(st + tile_chunk<C>(k_tok, 2 * ks + k_sel), b0, b1, b2, b3);
                 mma_16816(S[0], qa[ks], b0, b1);
                 mma_16816(S[1], qa[ks], b2, b3);
             }
+            // a token counts if its row may see it and this stage loaded it
+            // (with 8-token blocks a warp's second block can lie past the run)
             const int pos0 = md.t0 + qw * 16 + tig * 2;
+            const int st_end = md.t0 + md.ntok;
+            const int lim0 = min(lim[0], st_end), lim1 = min(lim[1], st_end);
             float mx[2] = {kNegInf, kNegInf};
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const int pos = pos0 + nt * 8 + (c & 1);
-                    const float v = pos < lim[c >> 1] ? S[nt][c] * sl2 : kNegInf;
+                    const float v = pos < ((c >> 1) ? lim1 : lim0) ? S[nt][c] * sl2 : kNegInf;
                     S[nt][c] = v;
                     mx[c >> 1] = fmaxf(mx[c >> 1], v);
                 }
@@ -505,11 +656,8 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
             const bool v_ok = v_i < nv;
 #pragma unroll
             for (int np = 0; np < C::D / 16; ++np) {
-                const int h = np / 4;
-                const int c = (2 * np) % 8 + v_sel;
                 const uint32_t addr =
-                    v_ok ? st + C::KV_BYTES + v_row_off + h * C::BS * 128 + ((c ^ v_x) << 4)
-                         : zero_row;
+                    v_ok ? st + C::KV_BYTES + tile_chunk<C>(v_tok, 2 * np + v_sel) : zero_row;
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4_trans(addr, b0, b1, b2, b3);
                 mma_16816(O[2 * np], pa, b0, b1);
@@ -520,9 +668,8 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
         if (lane == 0) mbar_arrive(empty0 + stage * 8);
 
         if (md.flags & F_LAST) {
-            // merge the token-warps of each m-tile, then store
+            // merge the token-warps of each m-tile (fixed order), then store
             const int tid = threadIdx.x;
-            for (int i = tid; i < C::RP * C::OB_STRIDE; i += C::NCW * 32) obuf[i] = 0.f;
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
                 float lr = l[rr];
@@ -538,17 +685,28 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
             float f[2];
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) f[rr] = row_factor<C>(mlb, mt * 16 + gid + rr * 8, m[rr]);
+            for (int w = 0; w < kTokWarps; ++w) {
+                if (qw == w) {
 #pragma unroll
-            for (int n = 0; n < C::D / 8; ++n) {
-                const int col = n * 8 + tig * 2;
-                float* o0 = obuf + (mt * 16 + gid) * C::OB_STRIDE + col;
-                float* o1 = obuf + (mt * 16 + gid + 8) * C::OB_STRIDE + col;
-                atomicAdd(o0, O[n][0] * f[0]);
-                atomicAdd(o0 + 1, O[n][1] * f[0]);
-                atomicAdd(o1, O[n][2] * f[1]);
-                atomicAdd(o1 + 1, O[n][3] * f[1]);
+                    for (int n = 0; n < C::D / 8; ++n) {
+                        const int col = n * 8 + tig * 2;
+                        float2* o0 = reinterpret_cast<float2*>(obuf + (mt * 16 + gid) * C::OB_STRIDE + col);
+                        float2* o1 =
+                            reinterpret_cast<float2*>(obuf + (mt * 16 + gid + 8) * C::OB_STRIDE + col);
+                        const float2 a = make_float2(O[n][0] * f[0], O[n][1] * f[0]);
+                        const float2 b = make_float2(O[n][2] * f[1], O[n][3] * f[1]);
+                        if (w == 0) {
+                            *o0 = a;
+                            *o1 = b;
+                        } else {
+                            const float2 x = *o0, y = *o1;
+                            *o0 = make_float2(x.x + a.x, x.y + a.y);
+                            *o1 = make_float2(y.x + b.x, y.y + b.y);
+                        }
+                    }
+                }
+                named_bar_sync(1, C::NCW * 32);
             }
-            named_bar_sync(1, C::NCW * 32);
             store_segment<C>(p, md, obuf, mlb, tid);
             named_bar_sync(1, C::NCW * 32);
         }
@@ -560,15 +718,18 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
 }
 
 // ---------------------------------------------------------------------------
-// FMA consumer: one query row per KV head (MHA decode).  Lane = (token, half
-// of the head dimension) for q . k; lane = D/32 columns for P V.
+// FMA consumer: one query row per KV head (MHA decode), a matrix-vector
+// product, so no tensor cores.  q . k: the 8 lanes of group g = lane / 8 each
+// take one 16-byte chunk per 128-byte unit of the rows of tokens g, g+4, g+8,
+// g+12 (a warp-wide 16-byte load reads whole units: no bank conflicts), then
+// sum over the group with shuffles.  P V: lane = D/32 output columns; the
+// fp16 weights of the warp's 16 tokens are broadcast through shared memory.
 template <class C>
 __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort_flag)
 {
     constexpr int D = C::D;
-    constexpr int DPL = D / 2;    // q . k columns per lane
-    constexpr int CPL = DPL / 8;  // 16-byte chunks per lane
-    constexpr int DPT = D / 32;   // P V columns per lane
+    constexpr int NH = C::NH;
+    constexpr int DPT = D / 32;  // P V columns per lane
     const int cw = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int qw = cw;
@@ -578,20 +739,20 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
     const uint32_t empty0 = full0 + C::STAGES * 8;
     float* mlb = reinterpret_cast<float*>(smem + C::ML_OFF);
     float* obuf = reinterpret_cast<float*>(smem + C::OBUF_OFF);
+    __half* pbuf = reinterpret_cast<__half*>(smem + C::PB_OFF) + qw * 16;
     const float sl2 = p.scale_log2;
 
-    const int tk = lane & 15, hf = lane >> 4;
-    const int k_tok = qw * 16 + tk;
-    const uint32_t k_row = (uint32_t)(((k_tok / C::BS) * C::NH * C::BS + (k_tok % C::BS)) * 128);
-    const int k_x = (k_tok % C::BS) & 7;
-    const int k_box = (hf * DPL) / 64;         // which 64-column box
-    const int k_c0 = ((hf * DPL) % 64) / 8;    // first chunk inside it
+    const int c = lane & 7, grp = lane >> 3;
+    uint32_t koff[4][NH];  // chunk c of each unit of tokens grp + 4i
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int h = 0; h < NH; ++h) koff[i][h] = tile_chunk<C>(qw * 16 + grp + 4 * i, h * 8 + c);
     const int v_col = lane * DPT;
-    const int v_box = v_col / 64;
-    const int v_c = (v_col % 64) / 8;
-    const int v_byte = (v_col % 8) * 2;
+    const int v_cg = v_col / 8;          // chunk holding my output columns
+    const int v_byte = (v_col % 8) * 2;  // byte offset inside that chunk
 
-    uint32_t qh[DPL / 2];
+    uint32_t qh[NH][4];  // q columns h*64 + c*8 .. +8 as fp16 pairs
     float o[DPT];
     float m = kNegInf, l = 0.f;
 
@@ -606,14 +767,13 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
         if (md.flags & F_END) break;
         const uint8_t* st = smem + stage * C::STAGE_BYTES;
         if (md.flags & F_FIRST) {
-            const uint4* qs = reinterpret_cast<const uint4*>(st + 2 * C::KV_BYTES + hf * DPL * 2);
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-                const uint4 v = qs[c];
-                qh[4 * c] = v.x;
-                qh[4 * c + 1] = v.y;
-                qh[4 * c + 2] = v.z;
-                qh[4 * c + 3] = v.w;
+            for (int h = 0; h < NH; ++h) {
+                const uint4 v = *reinterpret_cast<const uint4*>(st + 2 * C::KV_BYTES + (h * 64 + c * 8) * 2);
+                qh[h][0] = v.x;
+                qh[h][1] = v.y;
+                qh[h][2] = v.z;
+                qh[h][3] = v.w;
             }
 #pragma unroll
             for (int i = 0; i < DPT; ++i) o[i] = 0.f;
@@ -622,56 +782,75 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
         }
         const int nv = md.ntok - qw * 16;
         if (nv > 0) {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            if (tk < nv) {
-                const uint8_t* kb = st + k_row + k_box * C::BS * 128;
+            // partial dots of tokens grp + 4i over my chunk of every unit
+            float acc[4];
 #pragma unroll
-                for (int c = 0; c < CPL; ++c) {
-                    const uint4 kv = *reinterpret_cast<const uint4*>(
-                        kb + (((k_c0 + c) ^ k_x) << 4));
+            for (int i = 0; i < 4; ++i) {
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                    const uint4 kv = *reinterpret_cast<const uint4*>(st + koff[i][h]);
                     const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const uint32_t qq = qh[4 * c + e];
-                        acc[e] = fma_h((uint16_t)(qq & 0xffff), (uint16_t)(kw[e] & 0xffff), acc[e]);
-                        acc[e] = fma_h((uint16_t)(qq >> 16), (uint16_t)(kw[e] >> 16), acc[e]);
+                        a0 = fma_h((uint16_t)(qh[h][e] & 0xffff), (uint16_t)(kw[e] & 0xffff), a0);
+                        a1 = fma_h((uint16_t)(qh[h][e] >> 16), (uint16_t)(kw[e] >> 16), a1);
                     }
                 }
+                acc[i] = a0 + a1;
             }
-            float sdot = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-            sdot += __shfl_xor_sync(0xffffffffu, sdot, 16);
-            const float s = tk < nv ? sdot * sl2 : kNegInf;
-            float mx = s;
 #pragma unroll
-            for (int off = 1; off < 16; off <<= 1)
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            for (int off = 1; off < 8; off <<= 1)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+            float s[4], mx = kNegInf;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                s[i] = grp + 4 * i < nv ? acc[i] * sl2 : kNegInf;
+                mx = fmaxf(mx, s[i]);
+            }
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
             const float mn = fmaxf(m, mx);
             const float mu = mn == kNegInf ? 0.f : mn;
             const float alpha = ex2(m - mu);
             m = mn;
-            const float pe = ex2(s - mu);
-            l = l * alpha + (hf == 0 ? pe : 0.f);
+            float psum = 0.f;
 #pragma unroll
-            for (int i = 0; i < DPT; ++i) o[i] *= alpha;
-            const __half ph = __float2half_rn(pe);
-            const uint16_t phu = __half_as_ushort(ph);
-            const uint8_t* vb = st + C::KV_BYTES + v_box * C::BS * 128;
-            const int lim = nv < 16 ? nv : 16;
-            for (int t = 0; t < lim; ++t) {
-                const uint16_t pt = (uint16_t)__shfl_sync(0xffffffffu, (uint32_t)phu, t);
-                const int vt = qw * 16 + t;
-                const uint8_t* vr = vb + ((vt / C::BS) * C::NH * C::BS + (vt % C::BS)) * 128 +
-                                    ((v_c ^ ((vt % C::BS) & 7)) << 4) + v_byte;
-                if constexpr (DPT == 4) {
-                    const uint2 vv = *reinterpret_cast<const uint2*>(vr);
-                    o[0] = fma_h(pt, (uint16_t)(vv.x & 0xffff), o[0]);
-                    o[1] = fma_h(pt, (uint16_t)(vv.x >> 16), o[1]);
-                    o[2] = fma_h(pt, (uint16_t)(vv.y & 0xffff), o[2]);
-                    o[3] = fma_h(pt, (uint16_t)(vv.y >> 16), o[3]);
-                } else {
-                    const uint32_t vv = *reinterpret_cast<const uint32_t*>(vr);
-                    o[0] = fma_h(pt, (uint16_t)(vv & 0xffff), o[0]);
-                    o[1] = fma_h(pt, (uint16_t)(vv >> 16), o[1]);
+            for (int i = 0; i < 4; ++i) {
+                s[i] = ex2(s[i] - mu);
+                psum += s[i];
+            }
+            l = l * alpha + (c == 0 ? psum : 0.f);
+            if (alpha != 1.f) {
+#pragma unroll
+                for (int i = 0; i < DPT; ++i) o[i] *= alpha;
+            }
+            if (c == 0) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) pbuf[grp + 4 * i] = __float2half_rn(s[i]);
+            }
+            __syncwarp();
+            const uint4 pw0 = reinterpret_cast<const uint4*>(pbuf)[0];
+            const uint4 pw1 = reinterpret_cast<const uint4*>(pbuf)[1];
+            const uint32_t pw[8] = {pw0.x, pw0.y, pw0.z, pw0.w, pw1.x, pw1.y, pw1.z, pw1.w};
+            const uint8_t* vb = st + C::KV_BYTES + v_byte;
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+                if (t < nv) {
+                    const uint16_t pt = (uint16_t)(t & 1 ? pw[t >> 1] >> 16 : pw[t >> 1] & 0xffff);
+                    const uint8_t* vr = vb + tile_chunk<C>(qw * 16 + t, v_cg);
+                    if constexpr (DPT == 4) {
+                        const uint2 vv = *reinterpret_cast<const uint2*>(vr);
+                        o[0] = fma_h(pt, (uint16_t)(vv.x & 0xffff), o[0]);
+                        o[1] = fma_h(pt, (uint16_t)(vv.x >> 16), o[1]);
+                        o[2] = fma_h(pt, (uint16_t)(vv.y & 0xffff), o[2]);
+                        o[3] = fma_h(pt, (uint16_t)(vv.y >> 16), o[3]);
+                    } else {
+                        const uint32_t vv = *reinterpret_cast<const uint32_t*>(vr);
+                        o[0] = fma_h(pt, (uint16_t)(vv & 0xffff), o[0]);
+                        o[1] = fma_h(pt, (uint16_t)(vv >> 16), o[1]);
+                    }
                 }
             }
         }
@@ -680,7 +859,6 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
 
         if (md.flags & F_LAST) {
             const int tid = threadIdx.x;
-            for (int i = tid; i < C::RP * C::OB_STRIDE; i += C::NCW * 32) obuf[i] = 0.f;
             float lr = l;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) lr += __shfl_xor_sync(0xffffffffu, lr, off);
@@ -690,9 +868,14 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
             }
             named_bar_sync(1, C::NCW * 32);
             const float f = row_factor<C>(mlb, 0, m);
+            for (int w = 0; w < kTokWarps; ++w) {  // fixed order: deterministic sums
+                if (qw == w) {
 #pragma unroll
-            for (int i = 0; i < DPT; ++i) atomicAdd(obuf + v_col + i, o[i] * f);
-            named_bar_sync(1, C::NCW * 32);
+                    for (int i = 0; i < DPT; ++i)
+                        obuf[v_col + i] = (w == 0 ? 0.f : obuf[v_col + i]) + o[i] * f;
+                }
+                named_bar_sync(1, C::NCW * 32);
+            }
             store_segment<C>(p, md, obuf, mlb, tid);
             named_bar_sync(1, C::NCW * 32);
         }
@@ -704,7 +887,7 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
 }
 
 template <class C>
-__global__ void __launch_bounds__(C::THREADS, 1)
+__global__ void __maxnreg__(C::MAXREG)
     paged_attention_kernel(const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, const Params p)
 {
@@ -829,8 +1012,9 @@ int get_encoder()
     return KV_OK;
 }
 
-// Tensor map of a pool viewed as [num_blocks*Hkv*BS rows][D] fp16, box
-// [BS rows][64 columns], 128-byte swizzle.  Cached by (pointer, shape, device).
+// Tensor map of a pool viewed as [num_blocks*Hkv*BS rows][D] fp16 whose box
+// is one (block, kv-head) tile, 128-byte swizzle.  Cached by (pointer, shape,
+// device).
 int pool_tmap(const void* pool, uint64_t rows, int D, int BS, CUtensorMap* out)
 {
     int dev = 0;
@@ -843,12 +1027,16 @@ int pool_tmap(const void* pool, uint64_t rows, int D, int BS, CUtensorMap* out)
         }
     int rc = get_encoder();
     if (rc != KV_OK) return rc;
+    // The pool as [rows][D/64][64] fp16: a box of BS rows is one whole
+    // contiguous (block, kv-head) tile, written with the 128-byte swizzle.
     CUtensorMap m;
-    const cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    const cuuint64_t gstride[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)BS};
-    const cuuint32_t estride[2] = {1, 1};
-    CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(pool), gdim,
+    const cuuint32_t rank = D == 64 ? 2 : 3;
+    const cuuint64_t gdim[3] = {64, D == 64 ? (cuuint64_t)rows : (cuuint64_t)(D / 64),
+                                (cuuint64_t)rows};
+    const cuuint64_t gstride[2] = {D == 64 ? (cuuint64_t)128 : (cuuint64_t)128, (cuuint64_t)D * 2};
+    const cuuint32_t box[3] = {64, D == 64 ? (cuuint32_t)BS : (cuuint32_t)(D / 64), (cuuint32_t)BS};
+    const cuuint32_t estride[3] = {1, 1, 1};
+    CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, rank, const_cast<void*>(pool), gdim,
                           gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

@@ -215,6 +215,23 @@ def test_permutation_invariance_bit_exact():
     assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
 
 
+@pytest.mark.parametrize("name,kw", [("llama70b_gqa_bs8", {"B": 40, "max_len": 900}),
+                                     ("llama7b_mha", {"B": 12, "max_len": 1500}),
+                                     ("long_verify", {"B": 2, "max_len": 3000})])
+def test_deterministic_across_runs_and_splits(name, kw):
+    """Same inputs and launch -> the same bits; a different split of the
+    context -> within tolerance of the first."""
+    wl = make_workload(name, "cuda", **kw)
+    q_len = wl.spec.q_len
+    a = _run(wl, q_len).clone()
+    b = _run(wl, q_len).clone()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    c = _run(wl, q_len, grid_ctas=37, min_split_blocks=3)
+    ref = oracle_subset(wl, list(range(wl.B)), q_len)
+    assert_close(a, ref, name)
+    assert_close(c, ref, name + " resplit")
+
+
 def test_bad_block_id_is_flagged_without_fault():
     wl = make_workload("llama70b_gqa", "cuda", B=6, max_len=300, seed=8)
     wl.block_tables[2, 1] = wl.num_blocks + 5
