@@ -192,15 +192,19 @@ int paged_verify_attention(const void* q, const void* k_pool, const void* v_pool
 
 /* Launch knobs for tuning and tests; zero fields mean "default".
  *   grid_ctas        persistent CTAs (default: SMs x CTAs per SM);
- *   min_split_blocks smallest run of blocks one CTA takes (default 16), lower
- *                    values force more context splits (and merges);
+ *   min_split_blocks smallest run of work units one CTA takes (default 16),
+ *                    lower values force more context splits (and merges);
  *   use_pdl          1: launch the merge with programmatic dependent launch
- *                    (default), -1: plain launch. */
+ *                    (default), -1: plain launch;
+ *   seg_cost_blocks  fixed cost, in blocks, charged to every (sequence,
+ *                    kv-head) when work is divided among CTAs (default 8;
+ *                    -1 for none). */
 typedef struct paged_attention_opts {
     int32_t grid_ctas;
     int32_t min_split_blocks;
     int32_t use_pdl;
-    int32_t reserved[5];
+    int32_t seg_cost_blocks;
+    int32_t reserved[4];
 } paged_attention_opts;
 
 int paged_attention_ex(const void* q, const void* k_pool, const void* v_pool,

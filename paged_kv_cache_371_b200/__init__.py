@@ -184,7 +184,7 @@ def workspace_size(Hq: int, Hkv: int, q_len: int, head_dim: int, grid_ctas: int 
 
 
 def _attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len, out, workspace,
-               grid_ctas, min_split_blocks, use_pdl, entry):
+               grid_ctas, min_split_blocks, use_pdl, entry, seg_cost_blocks=0):
     dev = k_pool.device
     for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool")):
         _need(t, n, torch.float16, dev)
@@ -216,7 +216,7 @@ def _attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len, out,
     elif entry == "verify":
         rc = _L.paged_verify_attention(*args, q_len, *tail, _stream(dev))
     else:
-        o = _abi.PagedAttentionOpts(grid_ctas, min_split_blocks, use_pdl)
+        o = _abi.PagedAttentionOpts(grid_ctas, min_split_blocks, use_pdl, seg_cost_blocks)
         rc = _L.paged_attention_ex(*args, q_len, *tail, ctypes.byref(o), _stream(dev))
     check(rc, f"paged attention ({entry})")
     return out
@@ -237,10 +237,11 @@ def paged_verify_attention(q, k_pool, v_pool, block_tables, context_lens, scale,
 
 
 def paged_attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len=1, out=None,
-                    workspace=None, grid_ctas=0, min_split_blocks=0, use_pdl=0):
-    """Decode / verify with launch knobs (grid size, smallest split, PDL)."""
+                    workspace=None, grid_ctas=0, min_split_blocks=0, use_pdl=0, seg_cost_blocks=0):
+    """Decode / verify with launch knobs (grid size, smallest split, PDL,
+    per-segment cost used to balance CTAs)."""
     return _attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len, out, workspace,
-                      grid_ctas, min_split_blocks, use_pdl, "ex")
+                      grid_ctas, min_split_blocks, use_pdl, "ex", seg_cost_blocks)
 
 
 def device_error(reset: bool = True, device=None) -> int:

@@ -25,7 +25,8 @@ class KvPoolConfig(ctypes.Structure):
 
 class PagedAttentionOpts(ctypes.Structure):
     _fields_ = [("grid_ctas", ctypes.c_int32), ("min_split_blocks", ctypes.c_int32),
-                ("use_pdl", ctypes.c_int32), ("reserved", ctypes.c_int32 * 5)]
+                ("use_pdl", ctypes.c_int32), ("seg_cost_blocks", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 4)]
 
 
 _P = ctypes.c_void_p

@@ -51,6 +51,7 @@ constexpr int kTokWarps = 4;                // consumer warps along the tokens o
 constexpr int kMaxMT = 2;                   // m16 tiles of rows per KV head (rows <= 32)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kSmemBudget = 225 * 1024;
+constexpr int kDefaultSegCost = 8;          // virtual blocks per segment (balance)
 constexpr float kNegInf = -__builtin_huge_valf();
 
 enum : int32_t { F_FIRST = 1, F_LAST = 2, F_WHOLE = 4, F_END = 8 };
@@ -69,6 +70,7 @@ struct Params {
     int4* meta;       // [grid]: {s, kvh, first cta, slot in first cta} or s = -1
     int* err;
     int32_t max_blocks, B, q_len, Hq, Hkv, G, rows, num_blocks, min_share;
+    int32_t seg_cost;  // virtual blocks charged per (sequence, kv-head) segment
     float scale_log2;
 };
 
@@ -88,10 +90,13 @@ struct Cfg {
     static constexpr int MAXREG = MAXREG_RAW > 255 ? 255 : MAXREG_RAW;
     static constexpr int TILE_BYTES = BS * D * 2;           // one (block, kv-head) tile
     static constexpr int KV_BYTES = kTS * D * 2;            // K (or V) bytes per stage
-    static constexpr int Q_BYTES = (RP * D * 2 + 1023) / 1024 * 1024;
+    // query rows of a segment, one per 16-byte-padded row (conflict-free ldmatrix)
+    static constexpr int QROW = D * 2 + 16;
+    static constexpr int Q_BYTES = (RP * QROW + 1023) / 1024 * 1024;
     static constexpr int STAGE_BYTES = 2 * KV_BYTES + Q_BYTES;
     static constexpr int OB_STRIDE = D + 8;                 // floats per obuf row
-    static constexpr int OBUF_BYTES = RP * OB_STRIDE * 4;
+    static constexpr int OBUF_SLICE = RP * OB_STRIDE;               // floats
+    static constexpr int OBUF_BYTES = 2 * OBUF_SLICE * 4;           // two merge slices
     static constexpr int ML_BYTES = kTokWarps * RP * 2 * 4;
     static constexpr int FIXED = OBUF_BYTES + ML_BYTES + 256 + 16 * 64;
     static constexpr int STAGES_RAW = (kSmemBudget - FIXED) / STAGE_BYTES;
@@ -205,21 +210,34 @@ struct UnitWalker {
     }
 
     // Next stage of the run; false when the run is exhausted.
+    // Each (sequence, kv-head) spans seg_cost virtual units (its fixed cost:
+    // query load, merge, partial last stage) followed by its nb blocks, so
+    // equal runs of units also even out the number of segments per CTA.
     __device__ bool next(StageDesc& d)
     {
         if (!in_seg) {
             if (u >= u1) return false;
+            const int64_t span = (int64_t)nb + p->seg_cost;
             const int64_t local = u - seq_start;
-            kvh = (int32_t)(local / nb);
-            b = (int32_t)(local % nb);
-            const int64_t kv_end = seq_start + (int64_t)(kvh + 1) * nb;
+            kvh = (int32_t)(local / span);
+            const int64_t off = local % span;
+            if (off < p->seg_cost) {  // skip the virtual units
+                u += p->seg_cost - off;
+                if (u >= u1) return false;
+            }
+            b = (int32_t)((u - seq_start) % span - p->seg_cost);
+            const int64_t kv_end = seq_start + (int64_t)(kvh + 1) * span;
             const int64_t seg_end = u1 < kv_end ? u1 : kv_end;
             b1 = b + (int32_t)(seg_end - u);
             whole = b == 0 && b1 == nb;
             slot = first_seg ? 0 : 1;
             if (first_seg && b > 0 && b1 == nb) {
-                const int64_t gstart = seq_start + (int64_t)kvh * nb;
-                merge_meta = make_int4(s, kvh, (int32_t)(gstart / share), (gstart % share) ? 1 : 0);
+                // first CTA of this (sequence, kv-head): the one holding its
+                // first block; its piece is that CTA's first segment exactly
+                // when the CTA's run starts at or after the virtual units
+                const int64_t gstart = seq_start + (int64_t)kvh * span + p->seg_cost;
+                const int64_t a = gstart / share;
+                merge_meta = make_int4(s, kvh, (int32_t)a, a * share >= gstart - p->seg_cost ? 0 : 1);
             }
             first_seg = false;
             in_seg = true;
@@ -243,7 +261,7 @@ struct UnitWalker {
         u += nbl;
         if (b >= b1) {
             in_seg = false;
-            if (u < u1 && u == seq_start + (int64_t)nb * p->Hkv) {
+            if (u < u1 && u == seq_start + ((int64_t)nb + p->seg_cost) * p->Hkv) {
                 seq_start = u;
                 enter_sequence(s + 1);
             }
@@ -252,11 +270,11 @@ struct UnitWalker {
     }
 };
 
-// Number of units (blocks x KV heads) of sequence s.
+// Work units of sequence s: (blocks + the per-segment cost) x KV heads.
 template <class C>
 __device__ __forceinline__ int64_t units_of(const Params& p, int32_t Lraw)
 {
-    return (int64_t)nblk_of(Lraw, C::BS, p.max_blocks) * p.Hkv;
+    return ((int64_t)nblk_of(Lraw, C::BS, p.max_blocks) + p.seg_cost) * p.Hkv;
 }
 
 template <class C>
@@ -391,7 +409,7 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
                 const unsigned lmask = __ballot_sync(0xffffffffu, load);
                 if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, KV_DEV_BAD_BLOCK);
                 const bool firstst = (d.flags & F_FIRST) != 0;
-                const uint32_t qbytes = (uint32_t)(p.G * C::D * 2);
+                const uint32_t qbytes = (uint32_t)(p.G * C::D * 2);  // query bytes per window row
                 uint32_t bytes = (uint32_t)__popc(lmask) * (uint32_t)(2 * C::BS * C::D * 2);
                 if (firstst) bytes += qbytes * (uint32_t)p.q_len;
                 const uint32_t full = full0 + stage * 8;
@@ -414,10 +432,11 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
                     tma_load_tile<C::NH>(st + off, tmK, y, full, pol);
                     tma_load_tile<C::NH>(st + C::KV_BYTES + off, tmV, y, full, pol);
                 }
-                if (firstst && lane < p.q_len) {
+                if (firstst && lane < p.rows) {  // row R = j*G + g of the segment's queries
+                    const int j = lane / p.G, g = lane % p.G;
                     const __half* src =
-                        p.q + (((int64_t)d.s * p.q_len + lane) * p.Hq + (int64_t)d.kvh * p.G) * C::D;
-                    bulk_load(st + 2 * C::KV_BYTES + lane * qbytes, src, qbytes, full);
+                        p.q + (((int64_t)d.s * p.q_len + j) * p.Hq + (int64_t)d.kvh * p.G + g) * C::D;
+                    bulk_load(st + 2 * C::KV_BYTES + lane * C::QROW, src, C::D * 2, full);
                 }
                 ++k_issued;
             }
@@ -468,8 +487,9 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
 }
 
 // ---------------------------------------------------------------------------
-// Output of a finished segment: `obuf` rows hold the normalised o; `mlb`
-// holds per token-warp (m, l).  Writes fp16 output or fp32 partials.
+// Output of a finished segment: the two `obuf` slices hold the token-warps'
+// rescaled o (summed here, always in the same order); `mlb` holds per
+// token-warp (m, l).  Writes fp16 output or fp32 partials.
 template <class C>
 __device__ void store_segment(const Params& p, const StageMeta& md, const float* obuf,
                               const float* mlb, int tid)
@@ -480,12 +500,14 @@ __device__ void store_segment(const Params& p, const StageMeta& md, const float*
             const int R = idx / (C::D / 8);
             const int d0 = (idx % (C::D / 8)) * 8;
             const int j = R / p.G, g = R % p.G;
-            const float* src = obuf + R * C::OB_STRIDE + d0;
+            const float4* a = reinterpret_cast<const float4*>(obuf + R * C::OB_STRIDE + d0);
+            const float4* b = reinterpret_cast<const float4*>(obuf + C::OBUF_SLICE + R * C::OB_STRIDE + d0);
+            const float4 a0 = a[0], a1 = a[1], b0 = b[0], b1 = b[1];
             uint4 v;
-            v.x = pack_half2(src[0], src[1]);
-            v.y = pack_half2(src[2], src[3]);
-            v.z = pack_half2(src[4], src[5]);
-            v.w = pack_half2(src[6], src[7]);
+            v.x = pack_half2(a0.x + b0.x, a0.y + b0.y);
+            v.y = pack_half2(a0.z + b0.z, a0.w + b0.w);
+            v.z = pack_half2(a1.x + b1.x, a1.y + b1.y);
+            v.w = pack_half2(a1.z + b1.z, a1.w + b1.w);
             __half* dst = p.out + (((int64_t)md.s * p.q_len + j) * p.Hq + (int64_t)md.kvh * p.G + g) *
                                       C::D + d0;
             *reinterpret_cast<uint4*>(dst) = v;
@@ -495,10 +517,12 @@ __device__ void store_segment(const Params& p, const StageMeta& md, const float*
         for (int idx = tid; idx < rows * (C::D / 8); idx += C::NCW * 32) {
             const int R = idx / (C::D / 8);
             const int d0 = (idx % (C::D / 8)) * 8;
-            const float* src = obuf + R * C::OB_STRIDE + d0;
+            const float4* a = reinterpret_cast<const float4*>(obuf + R * C::OB_STRIDE + d0);
+            const float4* b = reinterpret_cast<const float4*>(obuf + C::OBUF_SLICE + R * C::OB_STRIDE + d0);
+            const float4 a0 = a[0], a1 = a[1], b0 = b[0], b1 = b[1];
             float4* dst = reinterpret_cast<float4*>(p.part_o + (pbase + R) * C::D + d0);
-            dst[0] = make_float4(src[0], src[1], src[2], src[3]);
-            dst[1] = make_float4(src[4], src[5], src[6], src[7]);
+            dst[0] = make_float4(a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w);
+            dst[1] = make_float4(a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w);
         }
         for (int R = tid; R < rows; R += C::NCW * 32) {
             float M = kNegInf;
@@ -571,16 +595,15 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
         if (md.flags & F_END) break;
         const uint32_t st = sbase + stage * C::STAGE_BYTES;
         if (md.flags & F_FIRST) {
-            const uint8_t* qs = smem + stage * C::STAGE_BYTES + 2 * C::KV_BYTES;
-            const int r0 = mt * 16 + gid, r1 = r0 + 8;
+            // A fragments of this warp's 16 query rows: matrices (rows 0-7 | 8-15)
+            // x (columns 16ks.. | 16ks+8..), one padded row address per lane
+            const uint32_t qrow = st + 2 * C::KV_BYTES +
+                                  (mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * C::QROW;
+            const int r0 = mt * 16 + gid;
 #pragma unroll
-            for (int ks = 0; ks < C::D / 16; ++ks) {
-                const int c0 = ks * 16 + tig * 2;
-                qa[ks][0] = *reinterpret_cast<const uint32_t*>(qs + (r0 * C::D + c0) * 2);
-                qa[ks][1] = *reinterpret_cast<const uint32_t*>(qs + (r1 * C::D + c0) * 2);
-                qa[ks][2] = *reinterpret_cast<const uint32_t*>(qs + (r0 * C::D + c0 + 8) * 2);
-                qa[ks][3] = *reinterpret_cast<const uint32_t*>(qs + (r1 * C::D + c0 + 8) * 2);
-            }
+            for (int ks = 0; ks < C::D / 16; ++ks)
+                ldsm_x4(qrow + ((2 * ks + (lane >> 4)) << 4), qa[ks][0], qa[ks][1], qa[ks][2],
+                        qa[ks][3]);
 #pragma unroll
             for (int n = 0; n < C::D / 8; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.f;
             m[0] = m[1] = kNegInf;
@@ -594,14 +617,25 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
         const int nv = md.ntok - qw * 16;
         if (nv > 0) {
             // S = q K^T for my 16 tokens (two n8 tiles)
+            // (even and odd k-steps accumulate separately: half the chain length)
             float S[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            float T[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
             for (int ks = 0; ks < C::D / 16; ++ks) {
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4(st + tile_chunk<C>(k_tok, 2 * ks + k_sel), b0, b1, b2, b3);
-                mma_16816(S[0], qa[ks], b0, b1);
-                mma_16816(S[1], qa[ks], b2, b3);
+                if (ks & 1) {
+                    mma_16816(T[0], qa[ks], b0, b1);
+                    mma_16816(T[1], qa[ks], b2, b3);
+                } else {
+                    mma_16816(S[0], qa[ks], b0, b1);
+                    mma_16816(S[1], qa[ks], b2, b3);
+                }
             }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) S[nt][c] += T[nt][c];
             // a token counts if its row may see it and this stage loaded it
             // (with 8-token blocks a warp's second block can lie past the run)
             const int pos0 = md.t0 + qw * 16 + tig * 2;
@@ -685,24 +719,31 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
             float f[2];
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) f[rr] = row_factor<C>(mlb, mt * 16 + gid + rr * 8, m[rr]);
-            for (int w = 0; w < kTokWarps; ++w) {
-                if (qw == w) {
+            // token-warps 0 and 1 write slices 0 and 1, then 2 and 3 add to them
+            const bool row0 = mt * 16 + gid < p.rows, row1 = mt * 16 + gid + 8 < p.rows;
+            float* slice = obuf + (qw & 1) * C::OBUF_SLICE;
+            for (int round = 0; round < 2; ++round) {
+                if ((qw >> 1) == round) {
 #pragma unroll
                     for (int n = 0; n < C::D / 8; ++n) {
                         const int col = n * 8 + tig * 2;
-                        float2* o0 = reinterpret_cast<float2*>(obuf + (mt * 16 + gid) * C::OB_STRIDE + col);
+                        float2* o0 = reinterpret_cast<float2*>(slice + (mt * 16 + gid) * C::OB_STRIDE + col);
                         float2* o1 =
-                            reinterpret_cast<float2*>(obuf + (mt * 16 + gid + 8) * C::OB_STRIDE + col);
-                        const float2 a = make_float2(O[n][0] * f[0], O[n][1] * f[0]);
-                        const float2 b = make_float2(O[n][2] * f[1], O[n][3] * f[1]);
-                        if (w == 0) {
-                            *o0 = a;
-                            *o1 = b;
-                        } else {
-                            const float2 x = *o0, y = *o1;
-                            *o0 = make_float2(x.x + a.x, x.y + a.y);
-                            *o1 = make_float2(y.x + b.x, y.y + b.y);
+                            reinterpret_cast<float2*>(slice + (mt * 16 + gid + 8) * C::OB_STRIDE + col);
+                        float2 a = make_float2(O[n][0] * f[0], O[n][1] * f[0]);
+                        float2 b = make_float2(O[n][2] * f[1], O[n][3] * f[1]);
+                        if (round) {
+                            if (row0) {
+                                const float2 x = *o0;
+                                a = make_float2(x.x + a.x, x.y + a.y);
+                            }
+                            if (row1) {
+                                const float2 y = *o1;
+                                b = make_float2(y.x + b.x, y.y + b.y);
+                            }
                         }
+                        if (row0) *o0 = a;
+                        if (row1) *o1 = b;
                     }
                 }
                 named_bar_sync(1, C::NCW * 32);
@@ -868,11 +909,12 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
             }
             named_bar_sync(1, C::NCW * 32);
             const float f = row_factor<C>(mlb, 0, m);
-            for (int w = 0; w < kTokWarps; ++w) {  // fixed order: deterministic sums
-                if (qw == w) {
+            float* slice = obuf + (qw & 1) * C::OBUF_SLICE;
+            for (int round = 0; round < 2; ++round) {  // fixed order: deterministic sums
+                if ((qw >> 1) == round) {
 #pragma unroll
                     for (int i = 0; i < DPT; ++i)
-                        obuf[v_col + i] = (w == 0 ? 0.f : obuf[v_col + i]) + o[i] * f;
+                        slice[v_col + i] = (round ? slice[v_col + i] : 0.f) + o[i] * f;
                 }
                 named_bar_sync(1, C::NCW * 32);
             }
@@ -906,10 +948,10 @@ __global__ void __maxnreg__(C::MAXREG)
     }
     // zero the padded query rows of every stage and the zero row
     if constexpr (!C::FMA) {
-        const int used = p.rows * C::D * 2;
+        const int used = p.rows * C::QROW;
         for (int st = 0; st < C::STAGES; ++st) {
             uint8_t* qa = smem + st * C::STAGE_BYTES + 2 * C::KV_BYTES;
-            for (int i = used + threadIdx.x * 16; i < C::RP * C::D * 2; i += C::THREADS * 16)
+            for (int i = used + threadIdx.x * 16; i < C::RP * C::QROW; i += C::THREADS * 16)
                 *reinterpret_cast<uint4*>(qa + i) = make_uint4(0, 0, 0, 0);
         }
     }
@@ -1176,6 +1218,8 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
     prm.rows = rows;
     prm.num_blocks = num_blocks;
     prm.min_share = (opts && opts->min_split_blocks > 0) ? opts->min_split_blocks : 16;
+    prm.seg_cost = (opts && opts->seg_cost_blocks != 0) ? (opts->seg_cost_blocks > 0 ? opts->seg_cost_blocks : 0)
+                                                        : kDefaultSegCost;
     prm.scale_log2 = scale * 1.4426950408889634f;
     const bool pdl = !(opts && opts->use_pdl < 0);
     cudaStream_t st = static_cast<cudaStream_t>(stream);

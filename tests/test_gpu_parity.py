@@ -177,6 +177,18 @@ def test_forced_splits_full_compare(Hq, Hkv, D, bs, q_len, grid, min_split):
     assert_close(out, ref, f"Hq{Hq} Hkv{Hkv} D{D} bs{bs} q{q_len} grid{grid}")
 
 
+@pytest.mark.parametrize("seg_cost", [-1, 1, 4, 13])
+@pytest.mark.parametrize("grid", [0, 61])
+def test_segment_cost_partition(seg_cost, grid):
+    """Many short sequences: CTA runs that start or end inside a segment's
+    virtual cost units, splits and merges all give the oracle's result."""
+    rng = np.random.Generator(np.random.PCG64(17))
+    lens = rng.integers(1, 120, size=40).astype(np.int32)
+    wl = make_workload("llama70b_gqa", "cuda", lens=lens, seed=19, Hq=16, Hkv=4, D=128)
+    out = _run(wl, 1, grid_ctas=grid, min_split_blocks=1, seg_cost_blocks=seg_cost)
+    assert_close(out, oracle_subset(wl, list(range(wl.B))), f"seg_cost {seg_cost} grid {grid}")
+
+
 def test_edge_cases():
     """Empty context (zeros), one token (exactly V), exact block multiples,
     a window longer than the context (zeros for rows that see nothing)."""
