@@ -214,6 +214,30 @@ int paged_attention_ex(const void* q, const void* k_pool, const void* v_pool,
                        int32_t num_blocks, void* workspace, size_t workspace_bytes,
                        const paged_attention_opts* opts, void* stream);
 
+/* paged_decode_attention without a workspace argument: for callers that may
+ * not allocate device memory themselves (their device memory is owned by
+ * another allocator, they receive tensors but no way to allocate, or a
+ * cudaMalloc on their hot path is not allowed).  The pages have no
+ * counterpart to this call; it exists for those callers only.
+ *   - Scratch for context splits comes from a fixed 8 MiB array inside the
+ *     library, present on every device that loads it until process exit.
+ *     Shapes that would need more return KV_ERR_INVALID (use
+ *     paged_decode_attention with a workspace instead).
+ *   - The call allocates nothing.  Its first call on each device looks up the
+ *     array's device address (a host-side runtime query, done once per
+ *     device with that device current); make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     contents; nothing in it needs to start at zero.  Calls that overlap on
+ *     the GPU (different streams running at the same time) race on it:
+ *     serialise them.
+ * Arguments and results are those of paged_decode_attention. */
+int paged_decode_attention_static_ws(const void* q, const void* k_pool, const void* v_pool,
+                                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                     const int32_t* context_lens, float scale, void* out,
+                                     int32_t B, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                                     int32_t block_size, int32_t num_blocks, void* stream);
+
 /* Read the current device's error word (bits KV_DEV_*) after synchronizing
  * `stream`; reset != 0 clears it. */
 int kv_device_error(int32_t* word_out, int32_t reset, void* stream);

@@ -1286,3 +1286,73 @@ int paged_attention_ex(const void* q, const void* k_pool, const void* v_pool,
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// Decode attention with library-owned scratch.
+//
+// The ordinary entry points take a caller-allocated workspace.  Some callers
+// cannot provide one: code that runs where every device byte is handed out by
+// someone else's allocator and a stray cudaMalloc is not allowed, plugins that
+// get tensors from a host framework but no allocation hook, and latency-
+// critical paths where a cudaMalloc (which may synchronise the device) must
+// never happen after start-up.  For them the split-context scratch lives in
+// this fixed array, loaded with the library: every GPU that loads the library
+// holds kStaticScratchBytes of it until the process exits.
+namespace {
+
+constexpr size_t kStaticScratchBytes = 8u << 20;  // 8 MiB
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxScratchDevices = 64;
+void* g_static_scratch_ptr[kMaxScratchDevices];
+std::mutex g_static_scratch_mu;
+
+// Device address of this device's copy of the array.  In host code the
+// array's name is only a host-side stand-in; the real address comes from the
+// runtime, looked up once per device with that device current.
+int static_scratch_address(void** out)
+{
+    int dev = 0;
+    int rc = kv_cuda_check(cudaGetDevice(&dev), "paged_decode_attention_static_ws");
+    if (rc != KV_OK) return rc;
+    if (dev < 0 || dev >= kMaxScratchDevices)
+        return kv_fail(KV_ERR_INVALID, "paged_decode_attention_static_ws: device index too large");
+    std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+    if (!g_static_scratch_ptr[dev]) {
+        void* p = nullptr;
+        rc = kv_cuda_check(cudaGetSymbolAddress(&p, g_static_scratch),
+                           "paged_decode_attention_static_ws: cudaGetSymbolAddress");
+        if (rc != KV_OK) return rc;
+        g_static_scratch_ptr[dev] = p;
+    }
+    *out = g_static_scratch_ptr[dev];
+    return KV_OK;
+}
+
+}  // namespace
+
+extern "C" int paged_decode_attention_static_ws(const void* q, const void* k_pool,
+                                                const void* v_pool, const int32_t* block_tables,
+                                                int32_t max_blocks_per_seq,
+                                                const int32_t* context_lens, float scale,
+                                                void* out, int32_t B, int32_t Hq, int32_t Hkv,
+                                                int32_t head_dim, int32_t block_size,
+                                                int32_t num_blocks, void* stream)
+{
+    if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || (head_dim != 64 && head_dim != 128))
+        return kv_fail(KV_ERR_INVALID, "paged_decode_attention_static_ws: bad sizes");
+    const int rows = Hq / Hkv;
+    if (rows > 16 * kMaxMT)
+        return kv_fail(KV_ERR_INVALID, "paged_decode_attention_static_ws: Hq/Hkv must be <= 32");
+    const size_t need = workspace_bytes_for(device_sms(), rows_padded(rows), head_dim);
+    if (need > kStaticScratchBytes)
+        return kv_fail(KV_ERR_INVALID,
+                       "paged_decode_attention_static_ws: this shape needs more scratch than the "
+                       "library's fixed 8 MiB; use paged_decode_attention with a workspace");
+    void* scratch = nullptr;
+    const int rc = static_scratch_address(&scratch);
+    if (rc != KV_OK) return rc;
+    return attention_impl(q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens, 1,
+                          scale, out, B, Hq, Hkv, head_dim, block_size, num_blocks, scratch,
+                          kStaticScratchBytes, nullptr, stream);
+}
