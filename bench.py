@@ -178,6 +178,21 @@ class ClockSampler:
                 "source": "nvml, 1 ms polling during the timed steps"}
 
 
+def aggregate(kv_bytes, tokens_heads, total_ms, world, device):
+    """Whole-job totals: bytes and tokens of all ranks, time of the slowest
+    rank (each rank times its own replica on the device).  Host-side only;
+    no data-path collective."""
+    import torch
+    import torch.distributed as dist
+    tot = torch.tensor([float(kv_bytes), float(tokens_heads)], dtype=torch.float64, device=device)
+    tmax = torch.tensor([float(total_ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+    kv_all, th_all = tot.tolist()
+    return kv_all, th_all, tmax.item()
+
+
 # ---------------------------------------------------------------------------
 # our arm
 
@@ -316,14 +331,7 @@ def run_ours(args):
     assert err == 0, f"device error word {err}"
     total_ms = sum(step_ms)
 
-    # whole-job aggregate: bytes of all ranks / slowest rank's time
-    tot = torch.tensor([kv_bytes_total, th_tokens], dtype=torch.float64, device=device)
-    tmax = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-    kv_all, th_all = tot.tolist()
-    t_all = tmax.item()
+    kv_all, th_all, t_all = aggregate(kv_bytes_total, th_tokens, total_ms, world, device)
     value = kv_all / (t_all * 1e-3) / 1e9
 
     # e2e: same steps through the public API with pinned host buffers
