@@ -81,7 +81,7 @@ struct Cfg {
     static constexpr int NH = D / 64;                       // 64-column halves per row
     static constexpr int NBS = kTS / BS;                    // blocks per stage
     static constexpr int RP = FMA ? 1 : 16 * MT;            // padded rows
-    static constexpr int NCW = FMA ? kTokWarps : kTokWarps * MT;
+    static constexpr int NCW = kTokWarps;                   // consumer warps
     static constexpr int THREADS = (NCW + 1) * 32;
     // registers per thread for one CTA per SM: warps are spread over the 4
     // SM sub-partitions, each with a 16K-register file
@@ -98,7 +98,8 @@ struct Cfg {
     static constexpr int OBUF_SLICE = RP * OB_STRIDE;               // floats
     static constexpr int OBUF_BYTES = 2 * OBUF_SLICE * 4;           // two merge slices
     static constexpr int ML_BYTES = kTokWarps * RP * 2 * 4;
-    static constexpr int FIXED = OBUF_BYTES + ML_BYTES + 256 + 16 * 64;
+    static constexpr int QP_BYTES = MT > 1 ? RP * QROW : 0;   // CTA copy of the query rows
+    static constexpr int FIXED = OBUF_BYTES + ML_BYTES + QP_BYTES + 256 + 16 * 64;
     static constexpr int STAGES_RAW = (kSmemBudget - FIXED) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
     static_assert(STAGES >= 2, "not enough shared memory for two stages");
@@ -108,7 +109,8 @@ struct Cfg {
     static constexpr int PB_OFF = ZERO_OFF + 128;           // per-warp fp16 weights (FMA path)
     static constexpr int ML_OFF = PB_OFF + 128;
     static constexpr int OBUF_OFF = ML_OFF + ML_BYTES;
-    static constexpr int SMEM_USED = OBUF_OFF + OBUF_BYTES;
+    static constexpr int QP_OFF = OBUF_OFF + OBUF_BYTES;
+    static constexpr int SMEM_USED = QP_OFF + QP_BYTES;
     static constexpr int SMEM_ALLOC = SMEM_USED + 1024;    // room to align the base
 };
 
@@ -928,6 +930,222 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
     }
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core consumer for more than 16 rows per KV head (verify windows):
+// each of the four token warps covers every m16 row tile for its 16 tokens,
+// so K and V fragments are loaded once and reused by all row tiles.  The
+// query fragments are re-read each stage (conflict-free ldmatrix) from a
+// per-CTA copy of the segment's query rows, which keeps registers for the
+// MT output tiles.
+template <class C>
+__device__ void consumer_mma_mt(const Params& p, uint8_t* smem, volatile int* abort_flag)
+{
+    constexpr int MT = C::MT;
+    const int qw = threadIdx.x >> 5;  // token warp 0..3
+    const int lane = threadIdx.x & 31;
+    const int gid = lane >> 2, tig = lane & 3;
+    const uint32_t sbase = smem_u32(smem);
+    const StageMeta* smeta = reinterpret_cast<const StageMeta*>(smem + C::META_OFF);
+    const uint32_t full0 = sbase + C::BAR_OFF;
+    const uint32_t empty0 = full0 + C::STAGES * 8;
+    const uint32_t zero_row = sbase + C::ZERO_OFF;
+    float* mlb = reinterpret_cast<float*>(smem + C::ML_OFF);
+    float* obuf = reinterpret_cast<float*>(smem + C::OBUF_OFF);
+    const float sl2 = p.scale_log2;
+
+    const int k_tok = qw * 16 + (lane >> 4) * 8 + (lane & 7);
+    const int k_sel = (lane >> 3) & 1;
+    const int v_i = ((lane >> 3) & 1) * 8 + (lane & 7);
+    const int v_tok = qw * 16 + v_i;
+    const int v_sel = lane >> 4;
+    // this lane's ldmatrix row address in the CTA copy of the query rows
+    const uint32_t qrow0 = sbase + C::QP_OFF + ((lane & 7) + ((lane >> 3) & 1) * 8) * C::QROW;
+
+    float O[MT][C::D / 8][4];
+    float m[MT][2], l[MT][2];
+    int lim[MT][2];
+
+    int stage = 0;
+    uint32_t phase = 0;
+    for (;;) {
+        if (!mbar_wait_bounded(full0 + stage * 8, phase, kWaitLimitNs)) {
+            *abort_flag = 1;
+            break;
+        }
+        const StageMeta md = smeta[stage];
+        if (md.flags & F_END) break;
+        const uint32_t st = sbase + stage * C::STAGE_BYTES;
+        if (md.flags & F_FIRST) {
+            // copy the segment's query rows out of the stage (it will be reused)
+            const uint4* src = reinterpret_cast<const uint4*>(smem + stage * C::STAGE_BYTES + 2 * C::KV_BYTES);
+            uint4* dst = reinterpret_cast<uint4*>(smem + C::QP_OFF);
+            for (int i = threadIdx.x; i < C::RP * C::QROW / 16; i += C::NCW * 32) dst[i] = src[i];
+            named_bar_sync(2, C::NCW * 32);
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+#pragma unroll
+                for (int n = 0; n < C::D / 8; ++n) O[t][n][0] = O[t][n][1] = O[t][n][2] = O[t][n][3] = 0.f;
+                m[t][0] = m[t][1] = kNegInf;
+                l[t][0] = l[t][1] = 0.f;
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int R = t * 16 + gid + rr * 8;
+                    lim[t][rr] = R < p.rows ? md.L - p.q_len + R / p.G + 1 : md.L;
+                }
+            }
+        }
+        const int nv = md.ntok - qw * 16;
+        if (nv > 0) {
+            float S[MT][2][4];
+#pragma unroll
+            for (int t = 0; t < MT; ++t)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) S[t][nt][0] = S[t][nt][1] = S[t][nt][2] = S[t][nt][3] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < C::D / 16; ++ks) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(st + tile_chunk<C>(k_tok, 2 * ks + k_sel), b0, b1, b2, b3);
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                    uint32_t a[4];
+                    ldsm_x4(qrow0 + t * 16 * C::QROW + ((2 * ks + (lane >> 4)) << 4), a[0], a[1], a[2],
+                            a[3]);
+                    mma_16816(S[t][0], a, b0, b1);
+                    mma_16816(S[t][1], a, b2, b3);
+                }
+            }
+            const int pos0 = md.t0 + qw * 16 + tig * 2;
+            const int st_end = md.t0 + md.ntok;
+            uint32_t pa[MT][4];
+            bool rescale = false;
+            float alpha[MT][2];
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+                const int lim0 = min(lim[t][0], st_end), lim1 = min(lim[t][1], st_end);
+                float mx[2] = {kNegInf, kNegInf};
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int pos = pos0 + nt * 8 + (c & 1);
+                        const float v = pos < ((c >> 1) ? lim1 : lim0) ? S[t][nt][c] * sl2 : kNegInf;
+                        S[t][nt][c] = v;
+                        mx[c >> 1] = fmaxf(mx[c >> 1], v);
+                    }
+                float mu[2];
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
+                    mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
+                    const float mn = fmaxf(m[t][rr], mx[rr]);
+                    mu[rr] = mn == kNegInf ? 0.f : mn;
+                    alpha[t][rr] = ex2(m[t][rr] - mu[rr]);
+                    m[t][rr] = mn;
+                    rescale |= alpha[t][rr] != 1.f;
+                }
+                float ps[2] = {0.f, 0.f};
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const float e = ex2(S[t][nt][c] - mu[c >> 1]);
+                        S[t][nt][c] = e;
+                        ps[c >> 1] += e;
+                    }
+                l[t][0] = l[t][0] * alpha[t][0] + ps[0];
+                l[t][1] = l[t][1] * alpha[t][1] + ps[1];
+                pa[t][0] = pack_half2(S[t][0][0], S[t][0][1]);
+                pa[t][1] = pack_half2(S[t][0][2], S[t][0][3]);
+                pa[t][2] = pack_half2(S[t][1][0], S[t][1][1]);
+                pa[t][3] = pack_half2(S[t][1][2], S[t][1][3]);
+            }
+            if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                for (int t = 0; t < MT; ++t)
+#pragma unroll
+                    for (int n = 0; n < C::D / 8; ++n) {
+                        O[t][n][0] *= alpha[t][0];
+                        O[t][n][1] *= alpha[t][0];
+                        O[t][n][2] *= alpha[t][1];
+                        O[t][n][3] *= alpha[t][1];
+                    }
+            }
+            const bool v_ok = v_i < nv;
+#pragma unroll
+            for (int np = 0; np < C::D / 16; ++np) {
+                const uint32_t addr =
+                    v_ok ? st + C::KV_BYTES + tile_chunk<C>(v_tok, 2 * np + v_sel) : zero_row;
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_trans(addr, b0, b1, b2, b3);
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                    mma_16816(O[t][2 * np], pa[t], b0, b1);
+                    mma_16816(O[t][2 * np + 1], pa[t], b2, b3);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + stage * 8);
+
+        if (md.flags & F_LAST) {
+            const int tid = threadIdx.x;
+#pragma unroll
+            for (int t = 0; t < MT; ++t)
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    float lr = l[t][rr];
+                    lr += __shfl_xor_sync(0xffffffffu, lr, 1);
+                    lr += __shfl_xor_sync(0xffffffffu, lr, 2);
+                    if (tig == 0) {
+                        const int R = t * 16 + gid + rr * 8;
+                        mlb[(qw * C::RP + R) * 2] = m[t][rr];
+                        mlb[(qw * C::RP + R) * 2 + 1] = lr;
+                    }
+                }
+            named_bar_sync(1, C::NCW * 32);
+            float* slice = obuf + (qw & 1) * C::OBUF_SLICE;
+            for (int round = 0; round < 2; ++round) {
+                if ((qw >> 1) == round) {
+#pragma unroll
+                    for (int t = 0; t < MT; ++t) {
+                        const int R0 = t * 16 + gid, R1 = R0 + 8;
+                        const bool row0 = R0 < p.rows, row1 = R1 < p.rows;
+                        const float f0 = row0 ? row_factor<C>(mlb, R0, m[t][0]) : 0.f;
+                        const float f1 = row1 ? row_factor<C>(mlb, R1, m[t][1]) : 0.f;
+#pragma unroll
+                        for (int n = 0; n < C::D / 8; ++n) {
+                            const int col = n * 8 + tig * 2;
+                            float2* o0 = reinterpret_cast<float2*>(slice + R0 * C::OB_STRIDE + col);
+                            float2* o1 = reinterpret_cast<float2*>(slice + R1 * C::OB_STRIDE + col);
+                            float2 a = make_float2(O[t][n][0] * f0, O[t][n][1] * f0);
+                            float2 b = make_float2(O[t][n][2] * f1, O[t][n][3] * f1);
+                            if (round) {
+                                if (row0) {
+                                    const float2 x = *o0;
+                                    a = make_float2(x.x + a.x, x.y + a.y);
+                                }
+                                if (row1) {
+                                    const float2 y = *o1;
+                                    b = make_float2(y.x + b.x, y.y + b.y);
+                                }
+                            }
+                            if (row0) *o0 = a;
+                            if (row1) *o1 = b;
+                        }
+                    }
+                }
+                named_bar_sync(1, C::NCW * 32);
+            }
+            store_segment<C>(p, md, obuf, mlb, tid);
+            named_bar_sync(1, C::NCW * 32);
+        }
+        if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+        }
+    }
+}
+
 template <class C>
 __global__ void __maxnreg__(C::MAXREG)
     paged_attention_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -965,6 +1183,8 @@ __global__ void __maxnreg__(C::MAXREG)
         producer<C>(&tmK, &tmV, p, smem, &abort_flag);
     } else if constexpr (C::FMA) {
         consumer_fma<C>(p, smem, &abort_flag);
+    } else if constexpr (C::MT > 1) {
+        consumer_mma_mt<C>(p, smem, &abort_flag);
     } else {
         consumer_mma<C>(p, smem, &abort_flag);
     }
