@@ -724,28 +724,28 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
             // token-warps 0 and 1 write slices 0 and 1, then 2 and 3 add to them
             const bool row0 = mt * 16 + gid < p.rows, row1 = mt * 16 + gid + 8 < p.rows;
             float* slice = obuf + (qw & 1) * C::OBUF_SLICE;
+            float* r0p = slice + (mt * 16 + gid) * C::OB_STRIDE + tig * 2;
+            float* r1p = r0p + 8 * C::OB_STRIDE;
             for (int round = 0; round < 2; ++round) {
                 if ((qw >> 1) == round) {
+                    // round 1 adds to round 0's values: read them all first so the
+                    // loads pipeline instead of waiting behind each store
+                    float2 x0[C::D / 8], x1[C::D / 8];
 #pragma unroll
                     for (int n = 0; n < C::D / 8; ++n) {
-                        const int col = n * 8 + tig * 2;
-                        float2* o0 = reinterpret_cast<float2*>(slice + (mt * 16 + gid) * C::OB_STRIDE + col);
-                        float2* o1 =
-                            reinterpret_cast<float2*>(slice + (mt * 16 + gid + 8) * C::OB_STRIDE + col);
-                        float2 a = make_float2(O[n][0] * f[0], O[n][1] * f[0]);
-                        float2 b = make_float2(O[n][2] * f[1], O[n][3] * f[1]);
-                        if (round) {
-                            if (row0) {
-                                const float2 x = *o0;
-                                a = make_float2(x.x + a.x, x.y + a.y);
-                            }
-                            if (row1) {
-                                const float2 y = *o1;
-                                b = make_float2(y.x + b.x, y.y + b.y);
-                            }
-                        }
-                        if (row0) *o0 = a;
-                        if (row1) *o1 = b;
+                        x0[n] = make_float2(0.f, 0.f);
+                        x1[n] = make_float2(0.f, 0.f);
+                        if (round && row0) x0[n] = *reinterpret_cast<const float2*>(r0p + n * 8);
+                        if (round && row1) x1[n] = *reinterpret_cast<const float2*>(r1p + n * 8);
+                    }
+#pragma unroll
+                    for (int n = 0; n < C::D / 8; ++n) {
+                        if (row0)
+                            *reinterpret_cast<float2*>(r0p + n * 8) =
+                                make_float2(x0[n].x + O[n][0] * f[0], x0[n].y + O[n][1] * f[0]);
+                        if (row1)
+                            *reinterpret_cast<float2*>(r1p + n * 8) =
+                                make_float2(x1[n].x + O[n][2] * f[1], x1[n].y + O[n][3] * f[1]);
                     }
                 }
                 named_bar_sync(1, C::NCW * 32);
@@ -1112,25 +1112,24 @@ __device__ void consumer_mma_mt(const Params& p, uint8_t* smem, volatile int* ab
                         const bool row0 = R0 < p.rows, row1 = R1 < p.rows;
                         const float f0 = row0 ? row_factor<C>(mlb, R0, m[t][0]) : 0.f;
                         const float f1 = row1 ? row_factor<C>(mlb, R1, m[t][1]) : 0.f;
+                        float* r0p = slice + R0 * C::OB_STRIDE + tig * 2;
+                        float* r1p = slice + R1 * C::OB_STRIDE + tig * 2;
+                        float2 x0[C::D / 8], x1[C::D / 8];  // loads first, then stores
 #pragma unroll
                         for (int n = 0; n < C::D / 8; ++n) {
-                            const int col = n * 8 + tig * 2;
-                            float2* o0 = reinterpret_cast<float2*>(slice + R0 * C::OB_STRIDE + col);
-                            float2* o1 = reinterpret_cast<float2*>(slice + R1 * C::OB_STRIDE + col);
-                            float2 a = make_float2(O[t][n][0] * f0, O[t][n][1] * f0);
-                            float2 b = make_float2(O[t][n][2] * f1, O[t][n][3] * f1);
-                            if (round) {
-                                if (row0) {
-                                    const float2 x = *o0;
-                                    a = make_float2(x.x + a.x, x.y + a.y);
-                                }
-                                if (row1) {
-                                    const float2 y = *o1;
-                                    b = make_float2(y.x + b.x, y.y + b.y);
-                                }
-                            }
-                            if (row0) *o0 = a;
-                            if (row1) *o1 = b;
+                            x0[n] = make_float2(0.f, 0.f);
+                            x1[n] = make_float2(0.f, 0.f);
+                            if (round && row0) x0[n] = *reinterpret_cast<const float2*>(r0p + n * 8);
+                            if (round && row1) x1[n] = *reinterpret_cast<const float2*>(r1p + n * 8);
+                        }
+#pragma unroll
+                        for (int n = 0; n < C::D / 8; ++n) {
+                            if (row0)
+                                *reinterpret_cast<float2*>(r0p + n * 8) =
+                                    make_float2(x0[n].x + O[t][n][0] * f0, x0[n].y + O[t][n][1] * f0);
+                            if (row1)
+                                *reinterpret_cast<float2*>(r1p + n * 8) =
+                                    make_float2(x1[n].x + O[t][n][2] * f1, x1[n].y + O[t][n][3] * f1);
                         }
                     }
                 }
