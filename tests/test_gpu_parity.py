@@ -189,6 +189,29 @@ def test_segment_cost_partition(seg_cost, grid):
     assert_close(out, oracle_subset(wl, list(range(wl.B))), f"seg_cost {seg_cost} grid {grid}")
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,maxlen,grid", [
+    (700, 8, 2, 90, 0),      # > 256 sequences: the device scan loops over chunks
+    (300, 32, 1, 400, 37),   # MQA: 32 query rows per KV head (the largest supported)
+    (1, 16, 4, 131072, 0),   # one 128K-token sequence split across every CTA
+])
+def test_scale_edges(B, Hq, Hkv, maxlen, grid):
+    rng = np.random.Generator(np.random.PCG64(B + Hq))
+    lens = rng.integers(1, maxlen + 1, size=B).astype(np.int32) if B > 1 else np.array([maxlen], np.int32)
+    wl = make_workload("llama70b_gqa", "cuda", lens=lens, seed=23, Hq=Hq, Hkv=Hkv, D=128)
+    out = _run(wl, 1, grid_ctas=grid) if grid else _run(wl)
+    seqs = _sample(wl.lens, min(B, 12))
+    assert_close(out[torch.as_tensor(seqs, device="cuda")], oracle_subset(wl, seqs), f"B{B} Hkv{Hkv}")
+
+
+def test_empty_batch_is_a_no_op():
+    wl = make_workload("tiny", "cuda")
+    bt = torch.zeros((0, 4), dtype=torch.int32, device="cuda")
+    cl = torch.zeros((0,), dtype=torch.int32, device="cuda")
+    q = torch.zeros((0, 1, 4, 64), dtype=torch.float16, device="cuda")
+    out = pkv.paged_decode_attention(q, wl.k_pool, wl.v_pool, bt, cl, wl.scale)
+    assert out.shape == (0, 1, 4, 64) and pkv.device_error() == 0
+
+
 def test_edge_cases():
     """Empty context (zeros), one token (exactly V), exact block multiples,
     a window longer than the context (zeros for rows that see nothing)."""
