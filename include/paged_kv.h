@@ -190,6 +190,19 @@ int paged_verify_attention(const void* q, const void* k_pool, const void* v_pool
                            int32_t block_size, int32_t num_blocks, void* workspace,
                            size_t workspace_bytes, void* stream);
 
+/* Paged (chunked) prefill ([T4] §1: the prompt is processed in parallel;
+ * same formula, paging and GQA grouping as above): q holds a chunk of q_len
+ * new tokens per sequence whose K/V are already in the cache; context_lens
+ * counts them; row j of sequence s attends causally to tokens
+ * 0 .. context_lens[s] - q_len + j.  Tensor cores (tcgen05, fp32 accumulators
+ * in tensor memory); requires head_dim 128, block_size 8 or 16, Hq/Hkv a
+ * divisor of 128.  Needs no workspace.  A row that sees no token gives zeros. */
+int paged_prefill_attention(const void* q, const void* k_pool, const void* v_pool,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq,
+                            const int32_t* context_lens, int32_t q_len, float scale, void* out,
+                            int32_t B, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                            int32_t block_size, int32_t num_blocks, void* stream);
+
 /* Launch knobs for tuning and tests; zero fields mean "default".
  *   grid_ctas        persistent CTAs (default: SMs x CTAs per SM);
  *   min_split_blocks smallest run of work units one CTA takes (default 16),

@@ -22,7 +22,7 @@ from ._abi import KVError, check
 
 __all__ = ["KVPool", "KVError", "pool_bytes", "paged_kv_append", "paged_kv_copy_blocks",
            "workspace_size", "paged_decode_attention", "paged_verify_attention",
-           "paged_attention", "device_error", "lib"]
+           "paged_attention", "paged_prefill_attention", "device_error", "lib"]
 
 _L = _abi.load()
 
@@ -242,6 +242,33 @@ def paged_attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len=
     per-segment cost used to balance CTAs)."""
     return _attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len, out, workspace,
                       grid_ctas, min_split_blocks, use_pdl, "ex", seg_cost_blocks)
+
+
+def paged_prefill_attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len,
+                            out=None):
+    """Causal chunked prefill over the paged cache (tensor cores): row j of
+    sequence s sees tokens 0 .. context_lens[s] - q_len + j."""
+    dev = k_pool.device
+    for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool")):
+        _need(t, n, torch.float16, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(context_lens, "context_lens", torch.int32, dev)
+    nb, Hkv, bs, D = k_pool.shape
+    B = context_lens.numel()
+    Hq = q.shape[-2]
+    if q.shape[-1] != D or q.numel() != B * q_len * Hq * D:
+        raise ValueError("q must be [B][q_len][Hq][D]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B:
+        raise ValueError("block_tables must be [B][max_blocks]")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.float16, dev)
+    check(_L.paged_prefill_attention(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+                                     block_tables.data_ptr(), block_tables.shape[1],
+                                     context_lens.data_ptr(), q_len, float(scale), out.data_ptr(),
+                                     B, Hq, Hkv, D, bs, nb, _stream(dev)),
+          "paged_prefill_attention")
+    return out
 
 
 def device_error(reset: bool = True, device=None) -> int:

@@ -62,6 +62,8 @@ SIGNATURES = {
                             _i32, _i32, _i32, _P, _sz, ctypes.POINTER(PagedAttentionOpts), _P],
                            ctypes.c_int),
     "kv_device_error": ([_PI32, _i32, _P], ctypes.c_int),
+    "paged_prefill_attention": ([_P, _P, _P, _P, _i32, _P, _i32, ctypes.c_float, _P, _i32, _i32,
+                                 _i32, _i32, _i32, _i32, _P], ctypes.c_int),
     "paged_decode_attention_static_ws": ([_P, _P, _P, _P, _i32, _P, ctypes.c_float, _P, _i32,
                                           _i32, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
 }

@@ -1,0 +1,628 @@
+// Paged prefill / chunked-prefill attention on 5th-generation tensor cores
+// (tcgen05, accumulators in tensor memory).
+//
+// What is computed: the prefill phase ("大模型推理加速与显存黑科技 (Inference
+// Acceleration & KV Cache)" §1: the whole prompt is processed in parallel)
+// over the paged cache ("LLM 推理优化：KV Cache、PagedAttention 与量化" §2.2):
+// a chunk of q_len new tokens per sequence, already appended to the cache, each
+// attending causally to every earlier token and to itself:
+//   out[s][j][h] = softmax(scale * q[s][j][h] . K_t) V_t,  t = 0 .. L_s - q_len + j,
+// with the Attention(Q,K,V) formula of the same page's §2 and the tiled
+// online softmax of its §4.2.  Query head h reads KV head h / (Hq/Hkv).
+//
+// Design (sm_100a): one CTA per (sequence, kv head, tile of 128 query rows);
+// the rows of a tile are (position, head-in-group) pairs, so all of them share
+// the K/V tiles staged for their KV head.  Per 64-token stage:
+//   S = Q K^T   tcgen05.mma kind::f16, M128 N64 K128, fp32 in tensor memory
+//   softmax     4 warps, thread i owns row i (= TMEM lane i): no shuffles
+//   O += P V    tcgen05.mma, M128 N128 K64, P fp16 from shared memory
+// Warp roles: warps 0-3 softmax / epilogue, warp 4 TMA producer, warp 5 TMEM
+// allocation + MMA issue.  S is double-buffered so the next S = Q K^T runs
+// while the softmax of the previous stage is computed.  O is rescaled lazily:
+// only when a row's running maximum grows by more than 2^8 (weights stay below
+// 2^8 otherwise, well within fp16 and fp32).  Every wait is bounded; tensor
+// memory is released on every path out of the kernel.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/paged_kv.h"
+#include "kv_device.h"
+#include "kv_ptx.cuh"
+#include "kv_status.h"
+
+namespace pkv_prefill {
+
+using namespace pkv;
+
+constexpr int D = 128;          // head dim served by this kernel
+constexpr int M = 128;          // query rows per CTA (TMEM lanes)
+constexpr int TS = 64;          // tokens per stage (S columns)
+constexpr int STAGES = 3;
+constexpr int NTHREADS = 192;   // 4 softmax warps, producer, MMA warp
+constexpr int TMEM_COLS = 256;  // S0 [0,64) S1 [64,128) O [128,256)
+constexpr uint64_t kWait = 2000000000ull;
+constexpr float kNegInf = -__builtin_huge_valf();
+constexpr float kRescaleThreshold = 8.f;  // log2 units
+
+// shared memory layout (bytes, from a 1024-aligned base)
+constexpr int Q_OFF = 0;                        // [2 halves][128 rows][128 B]
+constexpr int Q_BYTES = 2 * M * 128;            // 32 KB
+constexpr int ST_OFF = Q_OFF + Q_BYTES;         // stages: K [2][64][128 B], V same
+constexpr int KV_HALF = TS * 128;               // 8 KB: one 64-column half of 64 tokens
+constexpr int ST_BYTES = 4 * KV_HALF;           // 32 KB
+constexpr int P_OFF = ST_OFF + STAGES * ST_BYTES;   // [128 rows][128 B] fp16 P
+constexpr int P_BYTES = M * 128;
+constexpr int BAR_OFF = P_OFF + P_BYTES;
+// barriers: q_full, full[ST], empty[ST], s_full[2], s_free[2], p_full, o_done, drain
+constexpr int NBARS = 1 + 2 * STAGES + 2 + 2 + 3;
+constexpr int META_OFF = BAR_OFF + NBARS * 8;   // stage metadata: int4 per stage
+constexpr int TMEM_SLOT_OFF = META_OFF + STAGES * 16;
+constexpr int SMEM_USED = TMEM_SLOT_OFF + 16;
+constexpr int SMEM_ALLOC = SMEM_USED + 1024;
+
+struct Params {
+    const __half* q;
+    __half* out;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    int* err;
+    int32_t max_blocks, B, q_len, Hq, Hkv, G, bs, num_blocks, tiles_per_head;
+    float scale_log2;
+};
+
+// ---- tcgen05 wrappers --------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t slot_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_smem),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16, issued by one thread.
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0)
+        : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05 op this thread issued so far is done.
+__device__ __forceinline__ void umma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+        "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+          "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+          "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+          "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+          "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+          "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+          "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+          "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+          "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+          "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+          "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format: version 1).
+// sbo: bytes between 8-row groups; lbo: bytes between 64-element groups along
+// the leading dimension (MN-major operands only).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFF);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;   // version
+    d |= (uint64_t)2 << 61;   // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor, kind::f16: fp16 A/B, fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_f16(int m, int n, bool b_mn_major)
+{
+    return (1u << 4)                           // D format: f32
+           | (b_mn_major ? (1u << 16) : 0u)    // B major-ness (A is K-major)
+           | ((uint32_t)(n >> 3) << 17)        // N / 8
+           | ((uint32_t)(m >> 4) << 24);       // M / 16
+}
+
+struct StageInfo {
+    int32_t t0, ntok, nblk, flags;
+};
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                   const __grid_constant__ CUtensorMap tmQ, const Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ int abort_flag;
+    const uint32_t sb = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t bar0 = sb + BAR_OFF;
+    const uint32_t q_full = bar0;
+    auto full = [&](int i) { return bar0 + 8 * (1 + i); };
+    auto empty = [&](int i) { return bar0 + 8 * (1 + STAGES + i); };
+    auto s_full = [&](int b) { return bar0 + 8 * (1 + 2 * STAGES + b); };
+    auto s_free = [&](int b) { return bar0 + 8 * (3 + 2 * STAGES + b); };
+    const uint32_t p_full = bar0 + 8 * (5 + 2 * STAGES);
+    const uint32_t o_done = bar0 + 8 * (6 + 2 * STAGES);
+    const uint32_t drain = bar0 + 8 * (7 + 2 * STAGES);
+    StageInfo* sinfo = reinterpret_cast<StageInfo*>(smem + META_OFF);
+
+    // work item
+    const int tile = blockIdx.x % p.tiles_per_head;
+    const int kvh = (blockIdx.x / p.tiles_per_head) % p.Hkv;
+    const int s = blockIdx.x / (p.tiles_per_head * p.Hkv);
+    const int pos_per_tile = M / p.G;
+    const int j0 = tile * pos_per_tile;                    // first window position
+    int jn = p.q_len - j0;
+    if (jn > pos_per_tile) jn = pos_per_tile;              // positions in this tile
+    int32_t L = __ldg(p.context_lens + s);
+    if (L > p.max_blocks * p.bs) {
+        if (threadIdx.x == 0) atomicOr(p.err, KV_DEV_BAD_BLOCK);
+        L = p.max_blocks * p.bs;
+    }
+    // last token any row of this tile may see (exclusive end)
+    int kv_end = L - p.q_len + j0 + jn;
+    if (kv_end > L) kv_end = L;
+    if (kv_end < 0) kv_end = 0;
+    const int nst = (kv_end + TS - 1) / TS;
+
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(q_full, 1);
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(full(i), 1);
+            mbar_init(empty(i), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(s_full(b), 1);
+            mbar_init(s_free(b), 4);
+        }
+        mbar_init(p_full, 4);
+        mbar_init(o_done, 1);
+        mbar_init(drain, 1);
+        fence_barrier_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(sb + TMEM_SLOT_OFF, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + TMEM_SLOT_OFF);
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        const uint64_t pol = l2_policy_evict_first();
+        if (lane == 0) {
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            prefetch_tmap(&tmQ);
+            // Q tile: rows r = (j - j0) * G + g; one box per 64-column half,
+            // G heads x pos_per_tile positions (positions past q_len read zeros)
+            mbar_arrive_expect_tx(q_full, Q_BYTES);
+            const int z = s * p.q_len + j0;
+            for (int h = 0; h < 2; ++h)
+                asm volatile(
+                    "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                    " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(sb + Q_OFF + h * M * 128),
+                    "l"(reinterpret_cast<uint64_t>(&tmQ)), "r"(h * 64), "r"(kvh * p.G), "r"(z),
+                    "r"(q_full)
+                    : "memory");
+        }
+        bool ok = true;
+        for (int j = 0; j < nst && ok; ++j) {
+            const int slot = j % STAGES;
+            if (j >= STAGES) {
+                if (!mbar_wait_bounded(empty(slot), ((j / STAGES) - 1) & 1, kWait) ||
+                    *reinterpret_cast<volatile int*>(&abort_flag)) {
+                    ok = false;
+                    break;
+                }
+            }
+            const int t0 = j * TS;
+            int ntok = kv_end - t0;
+            if (ntok > TS) ntok = TS;
+            const int nblk = (ntok + p.bs - 1) / p.bs;
+            int32_t id = -1;
+            if (lane < nblk) id = __ldg(p.block_tables + (int64_t)s * p.max_blocks + t0 / p.bs + lane);
+            const bool bad = lane < nblk && (id < 0 || id >= p.num_blocks);
+            const bool load = lane < nblk && !bad;
+            const unsigned lmask = __ballot_sync(0xffffffffu, load);
+            if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, KV_DEV_BAD_BLOCK);
+            if (lane == 0) {
+                sinfo[slot].t0 = t0;
+                sinfo[slot].ntok = ntok;
+                sinfo[slot].nblk = nblk;
+                sinfo[slot].flags = 0;
+                mbar_arrive_expect_tx(full(slot), (uint32_t)__popc(lmask) * (uint32_t)(p.bs * D * 2 * 2));
+            }
+            __syncwarp();
+            if (load) {
+                const uint32_t st = sb + ST_OFF + slot * ST_BYTES;
+                const int32_t y = (id * p.Hkv + kvh) * p.bs;
+                // K half h of block `lane` -> rows [lane*bs, lane*bs+bs) of region h
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t rowoff = (uint32_t)(lane * p.bs * 128);
+                    tma_load_2d(st + h * KV_HALF + rowoff, &tmK, h * 64, y, full(slot), pol);
+                    tma_load_2d(st + 2 * KV_HALF + h * KV_HALF + rowoff, &tmV, h * 64, y, full(slot), pol);
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            atomicOr(p.err, KV_DEV_TIMEOUT);
+            abort_flag = 1;
+        }
+        // drain: the last issue into each slot must have landed
+        const int issued = ok ? nst : 0;
+        for (int i = lane; i < STAGES && i < issued; i += 32) {
+            const int n_i = (issued - i + STAGES - 1) / STAGES;
+            if (!mbar_wait_bounded(full(i), (n_i - 1) & 1, kWait)) atomicOr(p.err, KV_DEV_TIMEOUT);
+        }
+        if (lane == 0 && !mbar_wait_bounded(q_full, 0, kWait)) atomicOr(p.err, KV_DEV_TIMEOUT);
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issue
+        if (lane == 0) {
+            const uint32_t idS = idesc_f16(M, TS, false);
+            const uint32_t idO = idesc_f16(M, D, true);
+            bool ok = mbar_wait_bounded(q_full, 0, kWait);
+            tc_fence_after();
+            const uint32_t qa = sb + Q_OFF;
+            const uint32_t pa = sb + P_OFF;
+            for (int j = 0; j <= nst && ok; ++j) {
+                if (j < nst) {
+                    const int slot = j % STAGES, b = j & 1;
+                    ok = mbar_wait_bounded(full(slot), (j / STAGES) & 1, kWait);
+                    if (ok && j >= 2) ok = mbar_wait_bounded(s_free(b), ((j >> 1) - 1) & 1, kWait);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t kb = sb + ST_OFF + slot * ST_BYTES;
+                    // S_b = Q K^T over 8 k-steps of 16 dims (4 per 64-column half)
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t off = (k >> 2) * 0 + (k & 3) * 32;
+                        const uint64_t a = smem_desc(qa + (k >> 2) * M * 128 + off, 16, 1024);
+                        const uint64_t bd = smem_desc(kb + (k >> 2) * KV_HALF + off, 16, 1024);
+                        umma_f16(tmem + b * TS, a, bd, idS, k > 0 ? 1u : 0u);
+                    }
+                    umma_commit(s_full(b));
+                }
+                if (j >= 1) {
+                    const int jj = j - 1, slot = jj % STAGES;
+                    ok = mbar_wait_bounded(p_full, jj & 1, kWait);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t vb = sb + ST_OFF + slot * ST_BYTES + 2 * KV_HALF;
+                    // O += P V over 4 k-steps of 16 tokens; V is MN-major (dims
+                    // contiguous): 64-dim groups 8 KB apart, 8-token groups 1 KB apart
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t a = smem_desc(pa + k * 32, 16, 1024);
+                        const uint64_t bd = smem_desc(vb + k * 16 * 128, KV_HALF, 1024);
+                        umma_f16(tmem + 2 * TS, a, bd, idO, (jj > 0 || k > 0) ? 1u : 0u);
+                    }
+                    umma_commit(o_done);
+                    umma_commit(empty(slot));
+                }
+            }
+            if (!ok) {
+                atomicOr(p.err, KV_DEV_TIMEOUT);
+                abort_flag = 1;
+            }
+            // everything issued must have finished before tensor memory is freed
+            umma_commit(drain);
+            if (!mbar_wait_bounded(drain, 0, kWait)) atomicOr(p.err, KV_DEV_TIMEOUT);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int r = threadIdx.x;  // row = TMEM lane
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const int jr = r / p.G;                       // position within the tile
+        const bool row_ok = jr < jn;
+        const int lim = L - p.q_len + j0 + jr;        // last visible token (inclusive)
+        float m = kNegInf, l = 0.f;
+        bool ok = true;
+        uint8_t* prow = smem + P_OFF + r * 128;
+        for (int j = 0; j < nst && ok; ++j) {
+            const int b = j & 1, slot = j % STAGES;
+            ok = mbar_wait_bounded(s_full(b), (j >> 1) & 1, kWait);
+            if (!ok) break;
+            tc_fence_after();
+            float sv[TS];
+            {
+                float t32[32];
+                tmem_ld32(lane_base + b * TS, t32);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sv[i] = t32[i];
+                tmem_ld32(lane_base + b * TS + 32, t32);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sv[32 + i] = t32[i];
+            }
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_free(b));
+            // acquire the producer's stage metadata directly (its phase is
+            // complete and cannot move on before this stage's P V)
+            ok = mbar_wait_bounded(full(slot), (j / STAGES) & 1, kWait);
+            if (!ok) break;
+            StageInfo si;
+            si.t0 = reinterpret_cast<volatile int32_t*>(&sinfo[slot])[0];
+            si.ntok = reinterpret_cast<volatile int32_t*>(&sinfo[slot])[1];
+            int vis = lim - si.t0 + 1;                // columns this row may see
+            if (vis > si.ntok) vis = si.ntok;
+            if (!row_ok) vis = 0;
+            float mx = kNegInf;
+#pragma unroll
+            for (int c = 0; c < TS; ++c) {
+                sv[c] = c < vis ? sv[c] * p.scale_log2 : kNegInf;
+                mx = fmaxf(mx, sv[c]);
+            }
+            // the previous P V must be done before P is overwritten (and before
+            // O may be rescaled)
+            if (j >= 1) {
+                ok = mbar_wait_bounded(o_done, (j - 1) & 1, kWait);
+                if (!ok) break;
+                tc_fence_after();
+            }
+            const bool grow = mx > m + kRescaleThreshold;
+            if (__any_sync(0xffffffffu, grow)) {
+                const float mn = grow ? mx : m;
+                const float alpha = mn == kNegInf ? 1.f : ex2(m - mn);
+                if (j >= 1) {
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        float o32[32];
+                        tmem_ld32(lane_base + 2 * TS + c0, o32);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o32[i] *= alpha;
+                        tmem_st32(lane_base + 2 * TS + c0, o32);
+                    }
+                    tmem_wait_st();
+                }
+                l *= alpha;
+                m = mn;
+            }
+            const float mu = m == kNegInf ? 0.f : m;
+            // P row: fp16 weights, 128-byte row written with the 128-byte swizzle
+            float ps = 0.f;
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float a = ex2(sv[c8 * 8 + 2 * e] - mu);
+                    const float bq = ex2(sv[c8 * 8 + 2 * e + 1] - mu);
+                    ps += a + bq;
+                    w[e] = pack_half2(a, bq);
+                }
+                *reinterpret_cast<uint4*>(prow + ((c8 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            l += ps;
+            // V rows past the staged tokens must be finite zeros for the MMA
+            if (si.ntok < TS) {
+                uint8_t* vb = smem + ST_OFF + slot * ST_BYTES + 2 * KV_HALF;
+                for (int i = r; i < (TS - si.ntok) * 16; i += 128) {
+                    const int row = si.ntok + i / 16, ch = i % 16;  // 16 chunks: 2 halves x 8
+                    *reinterpret_cast<uint4*>(vb + (ch >> 3) * KV_HALF + row * 128 + ((ch & 7) << 4)) =
+                        make_uint4(0, 0, 0, 0);
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            // all 128 softmax threads wrote their part: one arrive per warp
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+        }
+        // epilogue: O / l, fp16, one 256-byte row per thread
+        if (ok && nst > 0) ok = mbar_wait_bounded(o_done, (nst - 1) & 1, kWait);
+        if (!ok) {
+            if (lane == 0) {
+                atomicOr(p.err, KV_DEV_TIMEOUT);
+                abort_flag = 1;
+            }
+        } else {
+            tc_fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            __half* dst = p.out + (((int64_t)s * p.q_len + j0 + jr) * p.Hq + (int64_t)kvh * p.G +
+                                   (r % p.G)) * D;
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                float o32[32];
+                tmem_ld32(lane_base + 2 * TS + c0, o32);
+                tmem_wait_ld();
+                if (nst == 0) {  // nothing visible (context shorter than the window)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o32[i] = 0.f;
+                }
+                if (row_ok) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        uint4 v;
+                        v.x = pack_half2(o32[i] * inv, o32[i + 1] * inv);
+                        v.y = pack_half2(o32[i + 2] * inv, o32[i + 3] * inv);
+                        v.z = pack_half2(o32[i + 4] * inv, o32[i + 5] * inv);
+                        v.w = pack_half2(o32[i + 6] * inv, o32[i + 7] * inv);
+                        *reinterpret_cast<uint4*>(dst + c0 + i) = v;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+}  // namespace pkv_prefill
+
+// ===========================================================================
+// Host side
+namespace {
+
+using namespace pkv_prefill;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_enc = nullptr;
+std::mutex g_mu;
+
+int encoder()
+{
+    if (g_enc) return KV_OK;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+        return kv_fail(KV_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    g_enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return KV_OK;
+}
+
+int encode(CUtensorMap* m, const void* base, cuuint32_t rank, const cuuint64_t* dims,
+           const cuuint64_t* strides, const cuuint32_t* box)
+{
+    const cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = g_enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, rank, const_cast<void*>(base), dims, strides,
+                       box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? KV_OK : kv_fail(KV_ERR_CUDA, "cuTensorMapEncodeTiled failed (prefill)");
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" int paged_prefill_attention(const void* q, const void* k_pool, const void* v_pool,
+                                       const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                       const int32_t* context_lens, int32_t q_len, float scale,
+                                       void* out, int32_t B, int32_t Hq, int32_t Hkv,
+                                       int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                                       void* stream)
+{
+    if (B < 0 || q_len < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || num_blocks < 1 || max_blocks_per_seq < 1)
+        return kv_fail(KV_ERR_INVALID, "paged_prefill_attention: bad sizes");
+    if (head_dim != 128) return kv_fail(KV_ERR_INVALID, "paged_prefill_attention: head_dim must be 128");
+    if (block_size != 8 && block_size != 16)
+        return kv_fail(KV_ERR_INVALID, "paged_prefill_attention: block_size must be 8 or 16");
+    const int G = Hq / Hkv;
+    if (G > M || M % G)
+        return kv_fail(KV_ERR_INVALID, "paged_prefill_attention: Hq/Hkv must divide 128");
+    if ((uint64_t)num_blocks * Hkv * block_size >= (1ull << 31) || (uint64_t)B * q_len >= (1ull << 31))
+        return kv_fail(KV_ERR_INVALID, "paged_prefill_attention: sizes exceed 32-bit coordinates");
+    if (B == 0) return KV_OK;
+    if (!q || !k_pool || !v_pool || !block_tables || !context_lens || !out)
+        return kv_fail(KV_ERR_INVALID, "paged_prefill_attention: null pointer");
+    if (!aligned16(q) || !aligned16(out) || !aligned16(k_pool) || !aligned16(v_pool))
+        return kv_fail(KV_ERR_INVALID, "paged_prefill_attention: buffers must be 16-byte aligned");
+    int* err = kv_error_word_ptr();
+    if (!err) return kv_fail(KV_ERR_CUDA, "paged_prefill_attention: no device error word");
+    int rc;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        rc = encoder();
+    }
+    if (rc != KV_OK) return rc;
+    const int ppt = M / G;
+    const int tiles = (q_len + ppt - 1) / ppt;
+    const uint64_t grid = (uint64_t)B * Hkv * tiles;
+    if (grid >= (1ull << 31)) return kv_fail(KV_ERR_INVALID, "paged_prefill_attention: grid too large");
+    // K / V pools as [rows][128] fp16, box = [bs rows][64 columns]
+    CUtensorMap tk, tv, tq;
+    const uint64_t rows = (uint64_t)num_blocks * Hkv * block_size;
+    const cuuint64_t pd[2] = {(cuuint64_t)D, rows};
+    const cuuint64_t ps[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t pb[2] = {64, (cuuint32_t)block_size};
+    if ((rc = encode(&tk, k_pool, 2, pd, ps, pb)) != KV_OK) return rc;
+    if ((rc = encode(&tv, v_pool, 2, pd, ps, pb)) != KV_OK) return rc;
+    // q as [B*q_len positions][Hq heads][128], box = [ppt positions][G heads][64]
+    const cuuint64_t qd[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)B * q_len};
+    const cuuint64_t qs[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+    const cuuint32_t qb[3] = {64, (cuuint32_t)G, (cuuint32_t)ppt};
+    if ((rc = encode(&tq, q, 3, qd, qs, qb)) != KV_OK) return rc;
+
+    Params prm;
+    prm.q = static_cast<const __half*>(q);
+    prm.out = static_cast<__half*>(out);
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    prm.err = err;
+    prm.max_blocks = max_blocks_per_seq;
+    prm.B = B;
+    prm.q_len = q_len;
+    prm.Hq = Hq;
+    prm.Hkv = Hkv;
+    prm.G = G;
+    prm.bs = block_size;
+    prm.num_blocks = num_blocks;
+    prm.tiles_per_head = tiles;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    static std::mutex amu;
+    static unsigned long long configured = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    {
+        std::lock_guard<std::mutex> lock(amu);
+        if (dev < 64 && !(configured & (1ull << dev))) {
+            rc = kv_cuda_check(cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                    SMEM_ALLOC),
+                               "cudaFuncSetAttribute (prefill)");
+            if (rc != KV_OK) return rc;
+            configured |= 1ull << dev;
+        }
+    }
+    prefill_kernel<<<(unsigned)grid, NTHREADS, SMEM_ALLOC, static_cast<cudaStream_t>(stream)>>>(tk, tv, tq,
+                                                                                                prm);
+    return kv_cuda_check(cudaGetLastError(), "paged_prefill_attention launch");
+}
