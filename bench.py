@@ -76,6 +76,26 @@ def algorithmic_bytes(lens, Hq, Hkv, D, bs, q_len):
     return kv, kv + qo + tab
 
 
+def prefill_flops(lens, Hq, D, q_len):
+    """Flops of causal chunked prefill: every row j of a sequence of length L
+    sees L - q_len + j + 1 tokens; q.K and P.V cost 2*D flops per token each."""
+    tot = 0
+    for L in lens:
+        L = int(L)
+        seen = q_len * (L - q_len) + q_len * (q_len + 1) // 2
+        tot += seen * Hq * D * 4
+    return tot
+
+
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (cuBLAS bf16 burst; fp16 runs at the same dense rate)"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 def measured_hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -249,6 +269,81 @@ def build_steps(pkv, wl, n_steps, device, seed):
         }
         steps.append(st)
     return steps
+
+
+def run_prefill(args):
+    """Chunked prefill: append the chunk's K/V, then causal attention of the
+    chunk over the paged cache; reported in TFLOP/s against the tensor peak."""
+    import numpy as np
+    import torch
+    import paged_kv_cache_371_b200 as pkv
+    from workloads import make_workload, normal_fp16
+    from workloads.synth import CONFIGS
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    spec = CONFIGS[args.workload]
+    wl = make_workload(args.workload, device, seed=rank_seed(spec.seed, rank), B=args.batch or None)
+    q_len, Hq, Hkv, D, bs = spec.q_len, spec.Hq, spec.Hkv, spec.D, spec.bs
+    bt, cl = torch.as_tensor(wl.block_tables, device=device), torch.as_tensor(wl.lens, device=device)
+    # slots of the chunk's tokens (positions L - q_len .. L - 1 of each sequence)
+    slots = []
+    for s_, L in enumerate(wl.lens):
+        for t in range(int(L) - q_len, int(L)):
+            slots.append(int(wl.block_tables[s_, t // bs]) * bs + t % bs)
+    slots = torch.as_tensor(np.array(slots, np.int64), device=device)
+    kn = normal_fp16((len(slots), Hkv, D), 901, device)
+    vn = normal_fp16((len(slots), Hkv, D), 902, device)
+    out = torch.empty_like(wl.q)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev=None):
+        pkv.paged_kv_append(kn, vn, slots, wl.k_pool, wl.v_pool)
+        if ev is not None:
+            ev.record(stream)
+        pkv.paged_prefill_attention(wl.q, wl.k_pool, wl.v_pool, bt, cl, wl.scale, q_len, out=out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert pkv.device_error() == 0
+    es = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ea = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ee = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        for k in range(args.steps):
+            flush.zero_()
+            es[k].record(stream)
+            step(ea[k])
+            ee[k].record(stream)
+        torch.cuda.synchronize()
+    assert pkv.device_error() == 0
+    step_ms = [es[k].elapsed_time(ee[k]) for k in range(args.steps)]
+    attn_ms = [ea[k].elapsed_time(ee[k]) for k in range(args.steps)]
+    fl = prefill_flops(wl.lens, Hq, D, q_len)
+    peak, kind = measured_tensor_peak()
+    tot_fl, _, t_all = aggregate(fl * args.steps, 0, sum(step_ms), world, device)
+    value = tot_fl / (t_all * 1e-3) / 1e12
+    achieved = fl / (statistics.mean(attn_ms) * 1e-3) / 1e12
+    if rank != 0:
+        return None
+    return {
+        "metric": "paged prefill attention TFLOP/s", "value": round(value, 2), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(t_all / args.steps, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": args.workload, "description": spec.description, "B": wl.B,
+                   "Hq": Hq, "Hkv": Hkv, "head_dim": D, "block_size": bs, "q_len": q_len,
+                   "mean_context": float(np.mean(wl.lens)),
+                   "step": "append the chunk's K/V + causal paged prefill attention",
+                   "l2": "flushed before every timed step (256 MB memset)"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "kernel": "paged_prefill_kernel (tcgen05)", "peak_kind": kind},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
 
 
 def run_ours(args):
@@ -529,7 +624,13 @@ def run_reference(args):
 
 def main(argv=None):
     args = parse_args(argv)
-    res = run_reference(args) if args.impl == "reference" else run_ours(args)
+    from workloads.synth import CONFIGS
+    if args.impl == "reference":
+        res = run_reference(args)
+    elif CONFIGS[args.workload].q_len > 32:
+        res = run_prefill(args)
+    else:
+        res = run_ours(args)
     if res is not None:
         print(json.dumps(res), flush=True)
 

@@ -93,6 +93,12 @@ CONFIGS = {
         "long_verify", 5, B=8, Hq=32, Hkv=8, D=128, bs=16, q_len=5, lens=_const(32768),
         description="as long_decode with a causal 5-token verify window per sequence "
                     "(the 5 draft tokens are the last 5 of the 32768)"),
+    "prefill_chunk": ConfigSpec(
+        "prefill_chunk", 6, B=8, Hq=64, Hkv=8, D=128, bs=16, q_len=512,
+        lens=_uniform(1024 + 512, 4096 + 512),
+        description="chunked prefill, Llama-2-70B-shaped GQA 64/8, head_dim 128, block 16: "
+                    "8 sequences, a 512-token chunk on prefixes U[1024,4096] (the chunk's "
+                    "K/V already in the cache)"),
 }
 
 PREFIX_TOKENS = 2048  # shared system-prompt prefix of the prefix_beam config
