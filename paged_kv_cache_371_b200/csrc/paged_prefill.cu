@@ -15,10 +15,13 @@
 // the K/V tiles staged for their KV head.  Per 64-token stage:
 //   S = Q K^T   tcgen05.mma kind::f16, M128 N64 K128, fp32 in tensor memory
 //   softmax     4 warps, thread i owns row i (= TMEM lane i): no shuffles
-//   O += P V    tcgen05.mma, M128 N128 K64, P fp16 from shared memory
+//   O += P V    tcgen05.mma, M128 N128 K64, P fp16 in tensor memory (it
+//               replaces the stage's S columns), V from shared memory
 // Warp roles: warps 0-3 softmax / epilogue, warp 4 TMA producer, warp 5 TMEM
 // allocation + MMA issue.  S is double-buffered so the next S = Q K^T runs
-// while the softmax of the previous stage is computed.  O is rescaled lazily:
+// while the softmax of the previous stage is computed, and two CTAs share an
+// SM (96 KB shared memory, 256 TMEM columns each) so one CTA's MMAs run while
+// the other's softmax does.  O is rescaled lazily:
 // only when a row's running maximum grows by more than 2^8 (weights stay below
 // 2^8 otherwise, well within fp16 and fp32).  Every wait is bounded; tensor
 // memory is released on every path out of the kernel.
@@ -41,7 +44,7 @@ using namespace pkv;
 constexpr int D = 128;          // head dim served by this kernel
 constexpr int M = 128;          // query rows per CTA (TMEM lanes)
 constexpr int TS = 64;          // tokens per stage (S columns)
-constexpr int STAGES = 3;
+constexpr int STAGES = 2;
 constexpr int NTHREADS = 192;   // 4 softmax warps, producer, MMA warp
 constexpr int TMEM_COLS = 256;  // S0 [0,64) S1 [64,128) O [128,256)
 constexpr uint64_t kWait = 2000000000ull;
@@ -54,9 +57,7 @@ constexpr int Q_BYTES = 2 * M * 128;            // 32 KB
 constexpr int ST_OFF = Q_OFF + Q_BYTES;         // stages: K [2][64][128 B], V same
 constexpr int KV_HALF = TS * 128;               // 8 KB: one 64-column half of 64 tokens
 constexpr int ST_BYTES = 4 * KV_HALF;           // 32 KB
-constexpr int P_OFF = ST_OFF + STAGES * ST_BYTES;   // [128 rows][128 B] fp16 P
-constexpr int P_BYTES = M * 128;
-constexpr int BAR_OFF = P_OFF + P_BYTES;
+constexpr int BAR_OFF = ST_OFF + STAGES * ST_BYTES;
 // barriers: q_full, full[ST], empty[ST], s_full[2], s_free[2], p_full, o_done, drain
 constexpr int NBARS = 1 + 2 * STAGES + 2 + 2 + 3;
 constexpr int META_OFF = BAR_OFF + NBARS * 8;   // stage metadata: int4 per stage
@@ -102,6 +103,19 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint6
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}"
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0)
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]: A (K-major, fp16 pairs per 32-bit
+// column, row i in lane i) from tensor memory.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0)
         : "memory");
 }
 
@@ -178,7 +192,7 @@ struct StageInfo {
     int32_t t0, ntok, nblk, flags;
 };
 
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __launch_bounds__(NTHREADS, 2)
     prefill_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ CUtensorMap tmQ, const Params p)
 {
@@ -320,7 +334,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             bool ok = mbar_wait_bounded(q_full, 0, kWait);
             tc_fence_after();
             const uint32_t qa = sb + Q_OFF;
-            const uint32_t pa = sb + P_OFF;
             for (int j = 0; j <= nst && ok; ++j) {
                 if (j < nst) {
                     const int slot = j % STAGES, b = j & 1;
@@ -344,12 +357,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t vb = sb + ST_OFF + slot * ST_BYTES + 2 * KV_HALF;
-                    // O += P V over 4 k-steps of 16 tokens; V is MN-major (dims
+                    // O += P V over 4 k-steps of 16 tokens.  P: fp16 pairs in the
+                    // first 32 columns of S buffer (jj & 1).  V is MN-major (dims
                     // contiguous): 64-dim groups 8 KB apart, 8-token groups 1 KB apart
                     for (int k = 0; k < 4; ++k) {
-                        const uint64_t a = smem_desc(pa + k * 32, 16, 1024);
                         const uint64_t bd = smem_desc(vb + k * 16 * 128, KV_HALF, 1024);
-                        umma_f16(tmem + 2 * TS, a, bd, idO, (jj > 0 || k > 0) ? 1u : 0u);
+                        umma_f16_ts(tmem + 2 * TS, tmem + (jj & 1) * TS + k * 8, bd, idO,
+                                    (jj > 0 || k > 0) ? 1u : 0u);
                     }
                     umma_commit(o_done);
                     umma_commit(empty(slot));
@@ -373,7 +387,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int lim = L - p.q_len + j0 + jr;        // last visible token (inclusive)
         float m = kNegInf, l = 0.f;
         bool ok = true;
-        uint8_t* prow = smem + P_OFF + r * 128;
         for (int j = 0; j < nst && ok; ++j) {
             const int b = j & 1, slot = j % STAGES;
             ok = mbar_wait_bounded(s_full(b), (j >> 1) & 1, kWait);
@@ -390,9 +403,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 for (int i = 0; i < 32; ++i) sv[32 + i] = t32[i];
             }
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s_free(b));
             // acquire the producer's stage metadata directly (its phase is
             // complete and cannot move on before this stage's P V)
             ok = mbar_wait_bounded(full(slot), (j / STAGES) & 1, kWait);
@@ -415,6 +425,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 ok = mbar_wait_bounded(o_done, (j - 1) & 1, kWait);
                 if (!ok) break;
                 tc_fence_after();
+                // P V of the previous stage is done: its S buffer (holding that
+                // stage's P) may take the next S
+                __syncwarp();
+                if (lane == 0) mbar_arrive(s_free((j - 1) & 1));
             }
             const bool grow = mx > m + kRescaleThreshold;
             if (__any_sync(0xffffffffu, grow)) {
@@ -435,19 +449,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 m = mn;
             }
             const float mu = m == kNegInf ? 0.f : m;
-            // P row: fp16 weights, 128-byte row written with the 128-byte swizzle
+            // P row: fp16 weights packed in pairs into the first 32 columns of
+            // this stage's S buffer (the tensor-memory A operand of P V)
             float ps = 0.f;
+            {
+                float pw[32];
 #pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) {
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float a = ex2(sv[c8 * 8 + 2 * e] - mu);
-                    const float bq = ex2(sv[c8 * 8 + 2 * e + 1] - mu);
+                for (int e = 0; e < 32; ++e) {
+                    const float a = ex2(sv[2 * e] - mu);
+                    const float bq = ex2(sv[2 * e + 1] - mu);
                     ps += a + bq;
-                    w[e] = pack_half2(a, bq);
+                    pw[e] = __uint_as_float(pack_half2(a, bq));
                 }
-                *reinterpret_cast<uint4*>(prow + ((c8 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                tmem_st32(lane_base + b * TS, pw);
             }
             l += ps;
             // V rows past the staged tokens must be finite zeros for the MMA
@@ -459,7 +473,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         make_uint4(0, 0, 0, 0);
                 }
             }
-            fence_proxy_async();
+            fence_proxy_async();  // the V zeros above are read by the tensor core
+            tmem_wait_st();
             tc_fence_before();
             // all 128 softmax threads wrote their part: one arrive per warp
             __syncwarp();
