@@ -413,12 +413,20 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             int vis = lim - si.t0 + 1;                // columns this row may see
             if (vis > si.ntok) vis = si.ntok;
             if (!row_ok) vis = 0;
-            float mx = kNegInf;
+            // raw scores stay unscaled; scale > 0 commutes with the maximum
+            if (!__all_sync(0xffffffffu, vis >= TS)) {  // boundary stage: mask
 #pragma unroll
-            for (int c = 0; c < TS; ++c) {
-                sv[c] = c < vis ? sv[c] * p.scale_log2 : kNegInf;
-                mx = fmaxf(mx, sv[c]);
+                for (int c = 0; c < TS; ++c) sv[c] = c < vis ? sv[c] : kNegInf;
             }
+            float mx4[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
+#pragma unroll
+            for (int c = 0; c < TS; c += 4) {
+                mx4[0] = fmaxf(mx4[0], sv[c]);
+                mx4[1] = fmaxf(mx4[1], sv[c + 1]);
+                mx4[2] = fmaxf(mx4[2], sv[c + 2]);
+                mx4[3] = fmaxf(mx4[3], sv[c + 3]);
+            }
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * p.scale_log2;
             // the previous P V must be done before P is overwritten (and before
             // O may be rescaled)
             if (j >= 1) {
@@ -451,19 +459,20 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             const float mu = m == kNegInf ? 0.f : m;
             // P row: fp16 weights packed in pairs into the first 32 columns of
             // this stage's S buffer (the tensor-memory A operand of P V)
-            float ps = 0.f;
+            float ps4[4] = {0.f, 0.f, 0.f, 0.f};
             {
                 float pw[32];
+                const float sl2 = p.scale_log2;
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const float a = ex2(sv[2 * e] - mu);
-                    const float bq = ex2(sv[2 * e + 1] - mu);
-                    ps += a + bq;
+                    const float a = ex2(fmaf(sv[2 * e], sl2, -mu));
+                    const float bq = ex2(fmaf(sv[2 * e + 1], sl2, -mu));
+                    ps4[e & 3] += a + bq;
                     pw[e] = __uint_as_float(pack_half2(a, bq));
                 }
                 tmem_st32(lane_base + b * TS, pw);
             }
-            l += ps;
+            l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
             // V rows past the staged tokens must be finite zeros for the MMA
             if (si.ntok < TS) {
                 uint8_t* vb = smem + ST_OFF + slot * ST_BYTES + 2 * KV_HALF;
