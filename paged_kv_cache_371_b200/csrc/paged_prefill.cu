@@ -19,7 +19,9 @@
 //               replaces the stage's S columns), V from shared memory
 // Warp roles: warps 0-3 softmax / epilogue, warp 4 TMA producer, warp 5 TMEM
 // allocation + MMA issue.  S is double-buffered so the next S = Q K^T runs
-// while the softmax of the previous stage is computed, and two CTAs share an
+// while the softmax of the previous stage is computed; K and V arrive through
+// separate two-slot rings, so a K slot refills as soon as its S is done (the
+// next K tile lands while this stage's softmax and P V run); two CTAs share an
 // SM (96 KB shared memory, 256 TMEM columns each) so one CTA's MMAs run while
 // the other's softmax does.  O is rescaled lazily:
 // only when a row's running maximum grows by more than 2^8 (weights stay below
@@ -44,7 +46,7 @@ using namespace pkv;
 constexpr int D = 128;          // head dim served by this kernel
 constexpr int M = 128;          // query rows per CTA (TMEM lanes)
 constexpr int TS = 64;          // tokens per stage (S columns)
-constexpr int STAGES = 2;
+constexpr int KV_SLOTS = 2;     // slots in each of the K and V rings
 constexpr int NTHREADS = 192;   // 4 softmax warps, producer, MMA warp
 constexpr int TMEM_COLS = 256;  // S0 [0,64) S1 [64,128) O [128,256)
 constexpr uint64_t kWait = 2000000000ull;
@@ -54,16 +56,18 @@ constexpr float kRescaleThreshold = 8.f;  // log2 units
 // shared memory layout (bytes, from a 1024-aligned base)
 constexpr int Q_OFF = 0;                        // [2 halves][128 rows][128 B]
 constexpr int Q_BYTES = 2 * M * 128;            // 32 KB
-constexpr int ST_OFF = Q_OFF + Q_BYTES;         // stages: K [2][64][128 B], V same
 constexpr int KV_HALF = TS * 128;               // 8 KB: one 64-column half of 64 tokens
-constexpr int ST_BYTES = 4 * KV_HALF;           // 32 KB
-constexpr int BAR_OFF = ST_OFF + STAGES * ST_BYTES;
-// barriers: q_full, full[ST], empty[ST], s_full[2], s_free[2], p_full, o_done, drain
-constexpr int NBARS = 1 + 2 * STAGES + 2 + 2 + 3;
-constexpr int META_OFF = BAR_OFF + NBARS * 8;   // stage metadata: int4 per stage
-constexpr int TMEM_SLOT_OFF = META_OFF + STAGES * 16;
+constexpr int SLOT_BYTES = 2 * KV_HALF;         // 16 KB: K (or V) of one stage
+constexpr int K_OFF = Q_OFF + Q_BYTES;          // K ring
+constexpr int V_OFF = K_OFF + KV_SLOTS * SLOT_BYTES;  // V ring
+constexpr int BAR_OFF = V_OFF + KV_SLOTS * SLOT_BYTES;
+// barriers: q_full, kfull[KS], kempty[KS], vfull[KS], vempty[KS], s_full[2],
+// s_free[2], p_full[2], drain
+constexpr int NBARS = 1 + 4 * KV_SLOTS + 2 + 2 + 2 + 1;
+constexpr int TMEM_SLOT_OFF = BAR_OFF + NBARS * 8;
 constexpr int SMEM_USED = TMEM_SLOT_OFF + 16;
 constexpr int SMEM_ALLOC = SMEM_USED + 1024;
+static_assert(2 * (SMEM_ALLOC + 1024) <= 233472, "two CTAs per SM must fit");
 
 struct Params {
     const __half* q;
@@ -188,10 +192,6 @@ __host__ __device__ constexpr uint32_t idesc_f16(int m, int n, bool b_mn_major)
            | ((uint32_t)(m >> 4) << 24);       // M / 16
 }
 
-struct StageInfo {
-    int32_t t0, ntok, nblk, flags;
-};
-
 __global__ void __launch_bounds__(NTHREADS, 2)
     prefill_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ CUtensorMap tmQ, const Params p)
@@ -204,14 +204,20 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t bar0 = sb + BAR_OFF;
     const uint32_t q_full = bar0;
-    auto full = [&](int i) { return bar0 + 8 * (1 + i); };
-    auto empty = [&](int i) { return bar0 + 8 * (1 + STAGES + i); };
-    auto s_full = [&](int b) { return bar0 + 8 * (1 + 2 * STAGES + b); };
-    auto s_free = [&](int b) { return bar0 + 8 * (3 + 2 * STAGES + b); };
-    const uint32_t p_full = bar0 + 8 * (5 + 2 * STAGES);
-    const uint32_t o_done = bar0 + 8 * (6 + 2 * STAGES);
-    const uint32_t drain = bar0 + 8 * (7 + 2 * STAGES);
-    StageInfo* sinfo = reinterpret_cast<StageInfo*>(smem + META_OFF);
+    // K and V rings are separate: a K slot is free once S = Q K^T of its
+    // stage is done, well before that stage's P V, so the K tile of a later
+    // stage is in flight while the softmax and P V of this one run.
+    auto kfull = [&](int i) { return bar0 + 8 * (1 + i); };
+    auto kempty = [&](int i) { return bar0 + 8 * (1 + KV_SLOTS + i); };
+    auto vfull = [&](int i) { return bar0 + 8 * (1 + 2 * KV_SLOTS + i); };
+    auto vempty = [&](int i) { return bar0 + 8 * (1 + 3 * KV_SLOTS + i); };
+    auto s_full = [&](int b) { return bar0 + 8 * (1 + 4 * KV_SLOTS + b); };
+    auto s_free = [&](int b) { return bar0 + 8 * (3 + 4 * KV_SLOTS + b); };
+    // one P barrier per S buffer: a softmax warp can run a stage ahead of the
+    // others, but not two (stage j+2 needs P V of stage j, hence every warp's
+    // arrive for stage j), so arrivals for different stages never share a phase
+    auto p_full = [&](int b) { return bar0 + 8 * (5 + 4 * KV_SLOTS + b); };
+    const uint32_t drain = bar0 + 8 * (7 + 4 * KV_SLOTS);
 
     // work item
     const int tile = blockIdx.x % p.tiles_per_head;
@@ -235,16 +241,17 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     if (threadIdx.x == 0) {
         abort_flag = 0;
         mbar_init(q_full, 1);
-        for (int i = 0; i < STAGES; ++i) {
-            mbar_init(full(i), 1);
-            mbar_init(empty(i), 1);
+        for (int i = 0; i < KV_SLOTS; ++i) {
+            mbar_init(kfull(i), 1);
+            mbar_init(kempty(i), 1);
+            mbar_init(vfull(i), 1);
+            mbar_init(vempty(i), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(s_full(b), 1);
-            mbar_init(s_free(b), 4);
+            mbar_init(s_free(b), 1);
+            mbar_init(p_full(b), 4);
         }
-        mbar_init(p_full, 4);
-        mbar_init(o_done, 1);
         mbar_init(drain, 1);
         fence_barrier_init();
     }
@@ -276,15 +283,17 @@ __global__ void __launch_bounds__(NTHREADS, 2)
                     "r"(q_full)
                     : "memory");
         }
-        bool ok = true;
-        for (int j = 0; j < nst && ok; ++j) {
-            const int slot = j % STAGES;
-            if (j >= STAGES) {
-                if (!mbar_wait_bounded(empty(slot), ((j / STAGES) - 1) & 1, kWait) ||
-                    *reinterpret_cast<volatile int*>(&abort_flag)) {
-                    ok = false;
-                    break;
-                }
+        // K (or V) of stage j into its ring slot: block `lane` of the stage
+        // -> rows [lane*bs, lane*bs+bs) of each 64-column half of the slot.
+        // Returns false if the slot never came free (timeout or abort).
+        auto issue = [&](int j, bool is_v) -> bool {
+            const int slot = j % KV_SLOTS;
+            const uint32_t fullb = is_v ? vfull(slot) : kfull(slot);
+            if (j >= KV_SLOTS) {
+                const uint32_t emptyb = is_v ? vempty(slot) : kempty(slot);
+                if (!mbar_wait_bounded(emptyb, ((j / KV_SLOTS) - 1) & 1, kWait) ||
+                    *reinterpret_cast<volatile int*>(&abort_flag))
+                    return false;
             }
             const int t0 = j * TS;
             int ntok = kv_end - t0;
@@ -295,35 +304,49 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             const bool bad = lane < nblk && (id < 0 || id >= p.num_blocks);
             const bool load = lane < nblk && !bad;
             const unsigned lmask = __ballot_sync(0xffffffffu, load);
-            if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, KV_DEV_BAD_BLOCK);
-            if (lane == 0) {
-                sinfo[slot].t0 = t0;
-                sinfo[slot].ntok = ntok;
-                sinfo[slot].nblk = nblk;
-                sinfo[slot].flags = 0;
-                mbar_arrive_expect_tx(full(slot), (uint32_t)__popc(lmask) * (uint32_t)(p.bs * D * 2 * 2));
-            }
+            if (!is_v && __any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, KV_DEV_BAD_BLOCK);
+            if (lane == 0)
+                mbar_arrive_expect_tx(fullb, (uint32_t)__popc(lmask) * (uint32_t)(p.bs * D * 2));
             __syncwarp();
             if (load) {
-                const uint32_t st = sb + ST_OFF + slot * ST_BYTES;
+                const uint32_t dst = sb + (is_v ? V_OFF : K_OFF) + slot * SLOT_BYTES +
+                                     (uint32_t)(lane * p.bs * 128);
                 const int32_t y = (id * p.Hkv + kvh) * p.bs;
-                // K half h of block `lane` -> rows [lane*bs, lane*bs+bs) of region h
-                for (int h = 0; h < 2; ++h) {
-                    const uint32_t rowoff = (uint32_t)(lane * p.bs * 128);
-                    tma_load_2d(st + h * KV_HALF + rowoff, &tmK, h * 64, y, full(slot), pol);
-                    tma_load_2d(st + 2 * KV_HALF + h * KV_HALF + rowoff, &tmV, h * 64, y, full(slot), pol);
-                }
+                const CUtensorMap* tm = is_v ? &tmV : &tmK;
+                tma_load_2d(dst, tm, 0, y, fullb, pol);
+                tma_load_2d(dst + KV_HALF, tm, 64, y, fullb, pol);
             }
+            return true;
+        };
+        // issue order K(0), K(1), V(0), K(2), V(1), ...: K runs one stage ahead
+        bool ok = true;
+        int k_issued = 0, v_issued = 0;
+        if (nst > 0) {
+            ok = issue(0, false);
+            if (ok) k_issued = 1;
+        }
+        for (int j = 0; j < nst && ok; ++j) {
+            if (j + 1 < nst) {
+                if (!(ok = issue(j + 1, false))) break;
+                ++k_issued;
+            }
+            if (!(ok = issue(j, true))) break;
+            ++v_issued;
         }
         if (!ok && lane == 0) {
             atomicOr(p.err, KV_DEV_TIMEOUT);
             abort_flag = 1;
         }
-        // drain: the last issue into each slot must have landed
-        const int issued = ok ? nst : 0;
-        for (int i = lane; i < STAGES && i < issued; i += 32) {
-            const int n_i = (issued - i + STAGES - 1) / STAGES;
-            if (!mbar_wait_bounded(full(i), (n_i - 1) & 1, kWait)) atomicOr(p.err, KV_DEV_TIMEOUT);
+        // drain: the last copy into each slot of each ring must have landed
+        for (int i = lane; i < KV_SLOTS; i += 32) {
+            if (i < k_issued) {
+                const int n_i = (k_issued - i + KV_SLOTS - 1) / KV_SLOTS;
+                if (!mbar_wait_bounded(kfull(i), (n_i - 1) & 1, kWait)) atomicOr(p.err, KV_DEV_TIMEOUT);
+            }
+            if (i < v_issued) {
+                const int n_i = (v_issued - i + KV_SLOTS - 1) / KV_SLOTS;
+                if (!mbar_wait_bounded(vfull(i), (n_i - 1) & 1, kWait)) atomicOr(p.err, KV_DEV_TIMEOUT);
+            }
         }
         if (lane == 0 && !mbar_wait_bounded(q_full, 0, kWait)) atomicOr(p.err, KV_DEV_TIMEOUT);
     } else if (warp == 5) {
@@ -336,27 +359,29 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             const uint32_t qa = sb + Q_OFF;
             for (int j = 0; j <= nst && ok; ++j) {
                 if (j < nst) {
-                    const int slot = j % STAGES, b = j & 1;
-                    ok = mbar_wait_bounded(full(slot), (j / STAGES) & 1, kWait);
+                    const int slot = j % KV_SLOTS, b = j & 1;
+                    ok = mbar_wait_bounded(kfull(slot), (j / KV_SLOTS) & 1, kWait);
                     if (ok && j >= 2) ok = mbar_wait_bounded(s_free(b), ((j >> 1) - 1) & 1, kWait);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t kb = sb + ST_OFF + slot * ST_BYTES;
+                    const uint32_t kb = sb + K_OFF + slot * SLOT_BYTES;
                     // S_b = Q K^T over 8 k-steps of 16 dims (4 per 64-column half)
                     for (int k = 0; k < 8; ++k) {
-                        const uint32_t off = (k >> 2) * 0 + (k & 3) * 32;
+                        const uint32_t off = (k & 3) * 32;
                         const uint64_t a = smem_desc(qa + (k >> 2) * M * 128 + off, 16, 1024);
                         const uint64_t bd = smem_desc(kb + (k >> 2) * KV_HALF + off, 16, 1024);
                         umma_f16(tmem + b * TS, a, bd, idS, k > 0 ? 1u : 0u);
                     }
                     umma_commit(s_full(b));
+                    umma_commit(kempty(slot));  // K of stage j consumed
                 }
                 if (j >= 1) {
-                    const int jj = j - 1, slot = jj % STAGES;
-                    ok = mbar_wait_bounded(p_full, jj & 1, kWait);
+                    const int jj = j - 1, slot = jj % KV_SLOTS;
+                    ok = mbar_wait_bounded(p_full(jj & 1), (jj >> 1) & 1, kWait);
+                    if (ok) ok = mbar_wait_bounded(vfull(slot), (jj / KV_SLOTS) & 1, kWait);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t vb = sb + ST_OFF + slot * ST_BYTES + 2 * KV_HALF;
+                    const uint32_t vb = sb + V_OFF + slot * SLOT_BYTES;
                     // O += P V over 4 k-steps of 16 tokens.  P: fp16 pairs in the
                     // first 32 columns of S buffer (jj & 1).  V is MN-major (dims
                     // contiguous): 64-dim groups 8 KB apart, 8-token groups 1 KB apart
@@ -365,8 +390,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
                         umma_f16_ts(tmem + 2 * TS, tmem + (jj & 1) * TS + k * 8, bd, idO,
                                     (jj > 0 || k > 0) ? 1u : 0u);
                     }
-                    umma_commit(o_done);
-                    umma_commit(empty(slot));
+                    umma_commit(s_free(jj & 1));  // P V of stage jj done: S buffer free
+                    umma_commit(vempty(slot));    // V of stage jj consumed
                 }
             }
             if (!ok) {
@@ -388,7 +413,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         float m = kNegInf, l = 0.f;
         bool ok = true;
         for (int j = 0; j < nst && ok; ++j) {
-            const int b = j & 1, slot = j % STAGES;
+            const int b = j & 1, slot = j % KV_SLOTS;
             ok = mbar_wait_bounded(s_full(b), (j >> 1) & 1, kWait);
             if (!ok) break;
             tc_fence_after();
@@ -403,15 +428,11 @@ __global__ void __launch_bounds__(NTHREADS, 2)
                 for (int i = 0; i < 32; ++i) sv[32 + i] = t32[i];
             }
             tmem_wait_ld();
-            // acquire the producer's stage metadata directly (its phase is
-            // complete and cannot move on before this stage's P V)
-            ok = mbar_wait_bounded(full(slot), (j / STAGES) & 1, kWait);
-            if (!ok) break;
-            StageInfo si;
-            si.t0 = reinterpret_cast<volatile int32_t*>(&sinfo[slot])[0];
-            si.ntok = reinterpret_cast<volatile int32_t*>(&sinfo[slot])[1];
-            int vis = lim - si.t0 + 1;                // columns this row may see
-            if (vis > si.ntok) vis = si.ntok;
+            const int t0 = j * TS;
+            int ntok = kv_end - t0;                   // staged tokens (< TS: last stage)
+            if (ntok > TS) ntok = TS;
+            int vis = lim - t0 + 1;                   // columns this row may see
+            if (vis > ntok) vis = ntok;
             if (!row_ok) vis = 0;
             // raw scores stay unscaled; scale > 0 commutes with the maximum
             if (!__all_sync(0xffffffffu, vis >= TS)) {  // boundary stage: mask
@@ -427,22 +448,21 @@ __global__ void __launch_bounds__(NTHREADS, 2)
                 mx4[3] = fmaxf(mx4[3], sv[c + 3]);
             }
             const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * p.scale_log2;
-            // the previous P V must be done before P is overwritten (and before
-            // O may be rescaled)
-            if (j >= 1) {
-                ok = mbar_wait_bounded(o_done, (j - 1) & 1, kWait);
-                if (!ok) break;
-                tc_fence_after();
-                // P V of the previous stage is done: its S buffer (holding that
-                // stage's P) may take the next S
-                __syncwarp();
-                if (lane == 0) mbar_arrive(s_free((j - 1) & 1));
-            }
+            // P of this stage goes to its own S buffer, which no pending P V
+            // reads, so the exponentials need not wait for the previous P V;
+            // only a rescale of O does.
             const bool grow = mx > m + kRescaleThreshold;
             if (__any_sync(0xffffffffu, grow)) {
                 const float mn = grow ? mx : m;
                 const float alpha = mn == kNegInf ? 1.f : ex2(m - mn);
                 if (j >= 1) {
+                    // P V of stage j-1 (the last one issued) must be done: the
+                    // ((j-1)/2)-th phase of its S buffer's barrier.  The phase
+                    // before it (stage j-3) completed before S(j-1) was issued,
+                    // and the one after needs this warp's arrive below.
+                    ok = mbar_wait_bounded(s_free((j - 1) & 1), ((j - 1) >> 1) & 1, kWait);
+                    if (!ok) break;
+                    tc_fence_after();
                     for (int c0 = 0; c0 < D; c0 += 32) {
                         float o32[32];
                         tmem_ld32(lane_base + 2 * TS + c0, o32);
@@ -474,10 +494,14 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             }
             l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
             // V rows past the staged tokens must be finite zeros for the MMA
-            if (si.ntok < TS) {
-                uint8_t* vb = smem + ST_OFF + slot * ST_BYTES + 2 * KV_HALF;
-                for (int i = r; i < (TS - si.ntok) * 16; i += 128) {
-                    const int row = si.ntok + i / 16, ch = i % 16;  // 16 chunks: 2 halves x 8
+            // (the copy of this stage's V must have landed first; V of stage
+            // j+2 cannot start before this stage's P V, so the phase is this one)
+            if (ntok < TS) {
+                ok = mbar_wait_bounded(vfull(slot), (j / KV_SLOTS) & 1, kWait);
+                if (!ok) break;
+                uint8_t* vb = smem + V_OFF + slot * SLOT_BYTES;
+                for (int i = r; i < (TS - ntok) * 16; i += 128) {
+                    const int row = ntok + i / 16, ch = i % 16;  // 16 chunks: 2 halves x 8
                     *reinterpret_cast<uint4*>(vb + (ch >> 3) * KV_HALF + row * 128 + ((ch & 7) << 4)) =
                         make_uint4(0, 0, 0, 0);
                 }
@@ -487,10 +511,11 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             tc_fence_before();
             // all 128 softmax threads wrote their part: one arrive per warp
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(p_full(b));
         }
         // epilogue: O / l, fp16, one 256-byte row per thread
-        if (ok && nst > 0) ok = mbar_wait_bounded(o_done, (nst - 1) & 1, kWait);
+        // (the MMA warp commits `drain` once, after the last P V)
+        if (ok && nst > 0) ok = mbar_wait_bounded(drain, 0, kWait);
         if (!ok) {
             if (lane == 0) {
                 atomicOr(p.err, KV_DEV_TIMEOUT);
