@@ -69,6 +69,24 @@ constexpr int SMEM_USED = TMEM_SLOT_OFF + 16;
 constexpr int SMEM_ALLOC = SMEM_USED + 1024;
 static_assert(2 * (SMEM_ALLOC + 1024) <= 233472, "two CTAs per SM must fit");
 
+// Progress watchdog for the polling loops: true once kWait of wall time has
+// passed without progress (the clock is read every 1024 idle polls).
+struct Idle {
+    uint32_t n = 0;
+    uint64_t t0 = 0;
+    __device__ __forceinline__ void reset() { n = 0; }
+    __device__ __forceinline__ bool expired()
+    {
+        if ((++n & 1023u) != 0) return false;
+        const uint64_t now = globaltimer_ns();
+        if (n == 1024u) {
+            t0 = now;
+            return false;
+        }
+        return now - t0 > kWait;
+    }
+};
+
 struct Params {
     const __half* q;
     __half* out;
@@ -283,18 +301,11 @@ __global__ void __launch_bounds__(NTHREADS, 2)
                     "r"(q_full)
                     : "memory");
         }
-        // K (or V) of stage j into its ring slot: block `lane` of the stage
-        // -> rows [lane*bs, lane*bs+bs) of each 64-column half of the slot.
-        // Returns false if the slot never came free (timeout or abort).
-        auto issue = [&](int j, bool is_v) -> bool {
+        // K (or V) of stage j into its (free) ring slot: block `lane` of the
+        // stage -> rows [lane*bs, lane*bs+bs) of each 64-column half of the slot.
+        auto issue = [&](int j, bool is_v) {
             const int slot = j % KV_SLOTS;
             const uint32_t fullb = is_v ? vfull(slot) : kfull(slot);
-            if (j >= KV_SLOTS) {
-                const uint32_t emptyb = is_v ? vempty(slot) : kempty(slot);
-                if (!mbar_wait_bounded(emptyb, ((j / KV_SLOTS) - 1) & 1, kWait) ||
-                    *reinterpret_cast<volatile int*>(&abort_flag))
-                    return false;
-            }
             const int t0 = j * TS;
             int ntok = kv_end - t0;
             if (ntok > TS) ntok = TS;
@@ -316,22 +327,40 @@ __global__ void __launch_bounds__(NTHREADS, 2)
                 tma_load_2d(dst, tm, 0, y, fullb, pol);
                 tma_load_2d(dst + KV_HALF, tm, 64, y, fullb, pol);
             }
-            return true;
         };
-        // issue order K(0), K(1), V(0), K(2), V(1), ...: K runs one stage ahead
+        // slot of stage j free?  (its previous use, stage j - KV_SLOTS, consumed;
+        // lane 0 decides for the warp)
+        auto slot_free = [&](int j, bool is_v) {
+            bool f = true;
+            if (j >= KV_SLOTS)
+                f = mbar_test(is_v ? vempty(j % KV_SLOTS) : kempty(j % KV_SLOTS), ((j / KV_SLOTS) - 1) & 1);
+            return __shfl_sync(0xffffffffu, f ? 1 : 0, 0) != 0;
+        };
+        // Poll both rings and issue whichever slot frees first: a K slot frees
+        // when S of its stage is done, a V slot when P V is; neither waits
+        // behind the other.
         bool ok = true;
         int k_issued = 0, v_issued = 0;
-        if (nst > 0) {
-            ok = issue(0, false);
-            if (ok) k_issued = 1;
-        }
-        for (int j = 0; j < nst && ok; ++j) {
-            if (j + 1 < nst) {
-                if (!(ok = issue(j + 1, false))) break;
-                ++k_issued;
+        Idle idle;
+        while (k_issued < nst || v_issued < nst) {
+            bool prog = false;
+            if (k_issued < nst && slot_free(k_issued, false)) {
+                issue(k_issued++, false);
+                prog = true;
             }
-            if (!(ok = issue(j, true))) break;
-            ++v_issued;
+            if (v_issued < k_issued && slot_free(v_issued, true)) {
+                issue(v_issued++, true);
+                prog = true;
+            }
+            if (prog) {
+                idle.reset();
+                continue;
+            }
+            if (__shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&abort_flag), 0) ||
+                __shfl_sync(0xffffffffu, idle.expired() ? 1 : 0, 0)) {
+                ok = false;
+                break;
+            }
         }
         if (!ok && lane == 0) {
             atomicOr(p.err, KV_DEV_TIMEOUT);
@@ -357,13 +386,17 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             bool ok = mbar_wait_bounded(q_full, 0, kWait);
             tc_fence_after();
             const uint32_t qa = sb + Q_OFF;
-            for (int j = 0; j <= nst && ok; ++j) {
-                if (j < nst) {
-                    const int slot = j % KV_SLOTS, b = j & 1;
-                    ok = mbar_wait_bounded(kfull(slot), (j / KV_SLOTS) & 1, kWait);
-                    if (ok && j >= 2) ok = mbar_wait_bounded(s_free(b), ((j >> 1) - 1) & 1, kWait);
-                    if (!ok) break;
+            // Poll and issue whichever is ready: S of the next stage (its K
+            // tile landed and the P V that last read its S buffer is done) or
+            // P V of the oldest stage with P written and V landed.
+            int ns = 0, np = 0;  // S issued, P V issued
+            Idle idle;
+            while (ok && np < nst) {
+                bool prog = false;
+                if (ns < nst && mbar_test(kfull(ns % KV_SLOTS), (ns / KV_SLOTS) & 1) &&
+                    (ns < 2 || mbar_test(s_free(ns & 1), ((ns >> 1) - 1) & 1))) {
                     tc_fence_after();
+                    const int slot = ns % KV_SLOTS, b = ns & 1;
                     const uint32_t kb = sb + K_OFF + slot * SLOT_BYTES;
                     // S_b = Q K^T over 8 k-steps of 16 dims (4 per 64-column half)
                     for (int k = 0; k < 8; ++k) {
@@ -373,26 +406,32 @@ __global__ void __launch_bounds__(NTHREADS, 2)
                         umma_f16(tmem + b * TS, a, bd, idS, k > 0 ? 1u : 0u);
                     }
                     umma_commit(s_full(b));
-                    umma_commit(kempty(slot));  // K of stage j consumed
+                    umma_commit(kempty(slot));  // K of stage ns consumed
+                    ++ns;
+                    prog = true;
                 }
-                if (j >= 1) {
-                    const int jj = j - 1, slot = jj % KV_SLOTS;
-                    ok = mbar_wait_bounded(p_full(jj & 1), (jj >> 1) & 1, kWait);
-                    if (ok) ok = mbar_wait_bounded(vfull(slot), (jj / KV_SLOTS) & 1, kWait);
-                    if (!ok) break;
+                if (np < ns && mbar_test(p_full(np & 1), (np >> 1) & 1) &&
+                    mbar_test(vfull(np % KV_SLOTS), (np / KV_SLOTS) & 1)) {
                     tc_fence_after();
+                    const int slot = np % KV_SLOTS;
                     const uint32_t vb = sb + V_OFF + slot * SLOT_BYTES;
                     // O += P V over 4 k-steps of 16 tokens.  P: fp16 pairs in the
-                    // first 32 columns of S buffer (jj & 1).  V is MN-major (dims
+                    // first 32 columns of S buffer (np & 1).  V is MN-major (dims
                     // contiguous): 64-dim groups 8 KB apart, 8-token groups 1 KB apart
                     for (int k = 0; k < 4; ++k) {
                         const uint64_t bd = smem_desc(vb + k * 16 * 128, KV_HALF, 1024);
-                        umma_f16_ts(tmem + 2 * TS, tmem + (jj & 1) * TS + k * 8, bd, idO,
-                                    (jj > 0 || k > 0) ? 1u : 0u);
+                        umma_f16_ts(tmem + 2 * TS, tmem + (np & 1) * TS + k * 8, bd, idO,
+                                    (np > 0 || k > 0) ? 1u : 0u);
                     }
-                    umma_commit(s_free(jj & 1));  // P V of stage jj done: S buffer free
-                    umma_commit(vempty(slot));    // V of stage jj consumed
+                    umma_commit(s_free(np & 1));  // P V of stage np done: S buffer free
+                    umma_commit(vempty(slot));    // V of stage np consumed
+                    ++np;
+                    prog = true;
                 }
+                if (prog)
+                    idle.reset();
+                else if (*reinterpret_cast<volatile int*>(&abort_flag) || idle.expired())
+                    ok = false;
             }
             if (!ok) {
                 atomicOr(p.err, KV_DEV_TIMEOUT);
