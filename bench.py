@@ -105,18 +105,18 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_sha():
+def kernel_source_sha(kernel="paged_attention.cu"):
     h = hashlib.sha256()
-    for name in ("paged_attention.cu", "kv_ptx.cuh"):
+    for name in (kernel, "kv_ptx.cuh"):
         with open(os.path.join(ROOT, "paged_kv_cache_371_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload):
+def ncu_traffic(workload, kernel="paged_attention.cu"):
     """DRAM bytes per launch of the attention kernel from a committed ncu
     summary, if it was taken on the current kernel source (else None)."""
-    sha = kernel_source_sha()
+    sha = kernel_source_sha(kernel)
     for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         kv = {}
         with open(path, encoding="utf-8") as f:
@@ -339,7 +339,8 @@ def run_prefill(args):
                    "step": "append the chunk's K/V + causal paged prefill attention",
                    "l2": "flushed before every timed step (256 MB memset)"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
-                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": ncu_traffic(args.workload, "paged_prefill.cu"),
                      "kernel": "paged_prefill_kernel (tcgen05)", "peak_kind": kind},
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
