@@ -132,6 +132,38 @@ int kv_batch_reserve_slots(kv_pool* pool, int32_t B, int32_t* tables, int32_t ta
                            int64_t* slots_out /* [B] */, int32_t* cow_pairs_out /* [2B] */,
                            int32_t* n_cow_out, int32_t* n_done_out);
 
+/* Prefix cache ([T3] §2.3 (3): requests sharing a prompt prefix are found by
+ * hashing block contents and point their tables at the same physical blocks;
+ * §2.3 (1): blocks nothing references are kept in LRU order).  A cached block
+ * is keyed by (parent, tokens): the cached block holding the previous
+ * block_size tokens (-1 for a first block) and its own block_size token ids,
+ * compared exactly; a match of block i therefore implies blocks 0..i-1.  Only
+ * full blocks are cached.  The cache holds one reference on each cached
+ * block (callers must not free that reference); host-only, not thread-safe.
+ *
+ * kv_prefix_match: walks the full blocks of tokens[0..n_tokens) from the
+ * start and stops at the first miss or after table_capacity blocks; each hit
+ * gets one more reference (for the new request) and is written to
+ * table_out[i]; *n_matched_out = hits.  The request then holds
+ * n_matched * block_size tokens of K/V and allocates the rest as usual. */
+int kv_prefix_match(kv_pool* pool, const int32_t* tokens, int32_t n_tokens, int32_t* table_out,
+                    int32_t table_capacity, int32_t* n_matched_out);
+/* kv_prefix_register: caches the full blocks of a request whose K/V are in
+ * the pool (table[i] holds tokens[i*bs .. i*bs+bs)), in order.  A block
+ * already cached under the same key is only marked used; the walk stops at a
+ * key cached in another block or at a block cached under another key.
+ * *n_cached_out (nullable) = leading blocks of table now cached under this
+ * prefix.  KV_ERR_INVALID if a table entry is not a live block (nothing
+ * changes). */
+int kv_prefix_register(kv_pool* pool, const int32_t* tokens, int32_t n_tokens, const int32_t* table,
+                       int32_t n_blocks, int32_t* n_cached_out);
+/* kv_prefix_evict: frees up to n cached blocks that only the cache still
+ * references and that have no cached child, least recently used first
+ * (matched or registered counts as a use); their ids go to ids_out[k]
+ * (nullable), in eviction order, and to the top of the free list. */
+int kv_prefix_evict(kv_pool* pool, int32_t n, int32_t* ids_out, int32_t* n_evicted_out);
+int kv_prefix_num_cached(const kv_pool* pool, int32_t* n_out);
+
 /* ---------------------------------------------------------------------------
  * Device calls.
  */
@@ -152,6 +184,30 @@ int paged_kv_append(const void* k_new, const void* v_new, const int64_t* slot_ma
 int paged_kv_copy_blocks(void* k_pool, void* v_pool, const int32_t* pairs, int32_t n,
                          int32_t Hkv, int32_t head_dim, int32_t block_size, int32_t num_blocks,
                          void* stream);
+
+/* Block swap between the pools and host memory ([T3] §2.3 (1): when the pool
+ * is full, a preempted request's blocks are moved to CPU memory and brought
+ * back when it resumes).  staging (device) and host hold
+ * [2 (K, V)][n][Hkv][block_size][head_dim] fp16: 2*n*Hkv*bs*D*2 bytes,
+ * staging 16-byte aligned; host should be pinned (cudaHostAlloc) for the
+ * copy to be asynchronous; both are owned by the caller.  block_ids is a
+ * DEVICE int32 array [n], n <= 65535.
+ *   swap_out: a gather kernel copies K and V of block_ids[i] to staging row
+ *     i, then one cudaMemcpyAsync copies staging to host (host may be NULL:
+ *     the blocks then stay in staging).
+ *   swap_in: one cudaMemcpyAsync copies host to staging (skipped if host is
+ *     NULL), then a scatter kernel writes row i to block_ids[i].
+ * Both are stream-ordered and bit-exact; the host buffer must stay valid
+ * until the stream reaches the copy.  Out-of-range ids are skipped and flag
+ * KV_DEV_BAD_BLOCK.  The host block manager is not touched: free the
+ * swapped-out ids, and allocate fresh ids for the swap-in, with block_free /
+ * block_alloc. */
+int paged_kv_swap_out(const void* k_pool, const void* v_pool, const int32_t* block_ids, int32_t n,
+                      void* staging, void* host, int32_t Hkv, int32_t head_dim, int32_t block_size,
+                      int32_t num_blocks, void* stream);
+int paged_kv_swap_in(void* k_pool, void* v_pool, const int32_t* block_ids, int32_t n, void* staging,
+                     const void* host, int32_t Hkv, int32_t head_dim, int32_t block_size,
+                     int32_t num_blocks, void* stream);
 
 /* Bytes of device workspace paged_decode_attention / paged_verify_attention
  * need for these head counts on the current device (partial results of

@@ -121,3 +121,111 @@ class BlockPoolSpec:
             table[-1] = new
             return OK, new * bs + off, last, new
         return OK, last * bs + off, -1, -1
+
+
+class PrefixCacheSpec:
+    """Content-addressed cache of full blocks over a BlockPoolSpec.
+
+    What the pages fix ([T3] §2.3 (3) and (1)): requests whose prompts share
+    a prefix are detected by hashing block contents and point their tables at
+    the same physical blocks; the pool keeps blocks that nothing references
+    in LRU order.
+
+    Readings (the pages give no more detail):
+      * a block's identity is its parent block (the cached block holding the
+        previous 16 tokens, -1 for the first) together with its own tokens:
+        the key chains, so a match of block i implies a match of blocks
+        0..i-1 (the K/V of a block depend on every earlier token).  Keys are
+        compared exactly; the hash only places them (here: a dict);
+      * only full blocks are cached and matched;
+      * the cache holds one reference on every cached block, so a block
+        outlives the requests that wrote it;
+      * match(tokens) walks the prompt's full blocks from the start and stops
+        at the first miss; every hit adds one reference (a fork) for the new
+        request and counts as a use;
+      * register(tokens, table) caches the table's full blocks in order; a
+        block already cached under the same key is only marked used; the walk
+        stops at a key cached under another block, or at a block cached under
+        another key;
+      * evict(n) releases up to n cached blocks that only the cache still
+        references and that have no cached child (so a parent is never
+        reused while a child's key names it), least recently used first;
+        each is freed in the pool.
+    """
+
+    def __init__(self, pool: BlockPoolSpec):
+        self.pool = pool
+        self.entries = {}    # (parent, tokens) -> block
+        self.key_of = {}     # block -> (parent, tokens)
+        self.children = {}   # block -> cached children
+        self.last_use = {}   # block -> use counter value
+        self.clock = 0
+
+    def _use(self, b):
+        self.clock += 1
+        self.last_use[b] = self.clock
+
+    def num_cached(self) -> int:
+        return len(self.key_of)
+
+    def match(self, tokens):
+        bs = self.pool.block_size
+        table, parent = [], -1
+        for i in range(len(tokens) // bs):
+            b = self.entries.get((parent, tuple(tokens[i * bs:(i + 1) * bs])))
+            if b is None:
+                break
+            self.pool.refcount[b] += 1
+            self._use(b)
+            table.append(b)
+            parent = b
+        return OK, table
+
+    def register(self, tokens, table):
+        bs = self.pool.block_size
+        n = min(len(tokens) // bs, len(table))
+        for b in table[:n]:
+            if not 0 <= b < self.pool.num_blocks or self.pool.refcount[b] == 0:
+                return ERR_INVALID, 0
+        parent, done = -1, 0
+        for i in range(n):
+            b = table[i]
+            key = (parent, tuple(tokens[i * bs:(i + 1) * bs]))
+            have = self.entries.get(key)
+            if have is None:
+                if b in self.key_of:
+                    break
+                self.entries[key] = b
+                self.key_of[b] = key
+                self.children[b] = 0
+                if parent >= 0:
+                    self.children[parent] += 1
+                self.pool.refcount[b] += 1
+                self._use(b)
+            elif have == b:
+                self._use(b)
+            else:
+                break
+            parent = b
+            done += 1
+        return OK, done
+
+    def evict(self, n: int):
+        if n < 0:
+            return ERR_INVALID, []
+        out = []
+        while len(out) < n:
+            cand = [b for b in self.key_of
+                    if self.children[b] == 0 and self.pool.refcount[b] == 1]
+            if not cand:
+                break
+            b = min(cand, key=lambda x: self.last_use[x])
+            key = self.key_of.pop(b)
+            del self.entries[key]
+            del self.children[b]
+            del self.last_use[b]
+            if key[0] >= 0:
+                self.children[key[0]] -= 1
+            self.pool.free([b])
+            out.append(b)
+        return OK, out

@@ -22,7 +22,8 @@ from ._abi import KVError, check
 
 __all__ = ["KVPool", "KVError", "pool_bytes", "paged_kv_append", "paged_kv_copy_blocks",
            "workspace_size", "paged_decode_attention", "paged_verify_attention",
-           "paged_attention", "paged_prefill_attention", "device_error", "lib"]
+           "paged_attention", "paged_prefill_attention", "paged_kv_swap_out", "paged_kv_swap_in",
+           "swap_staging_bytes", "device_error", "lib"]
 
 _L = _abi.load()
 
@@ -146,6 +147,39 @@ class KVPool:
               "kv_batch_reserve_slots")
         return slots, pairs[:ncow.value].copy()
 
+    # -- prefix cache --------------------------------------------------------
+    def prefix_match(self, tokens) -> list:
+        """Cached blocks holding the longest cached prefix of ``tokens`` (one
+        reference added to each, for the caller)."""
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        cap = t.size // self.block_size
+        out = np.zeros(max(cap, 1), np.int32)
+        n = ctypes.c_int32()
+        check(_L.kv_prefix_match(self._h, _i32p(t), t.size, _i32p(out), cap, ctypes.byref(n)),
+              "kv_prefix_match")
+        return out[:n.value].tolist()
+
+    def prefix_register(self, tokens, table) -> int:
+        """Cache the full blocks of a request; returns how many leading blocks
+        of ``table`` are now cached under this prefix."""
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        b = np.ascontiguousarray(table, dtype=np.int32)
+        n = ctypes.c_int32()
+        check(_L.kv_prefix_register(self._h, _i32p(t), t.size, _i32p(b), b.size, ctypes.byref(n)),
+              "kv_prefix_register")
+        return n.value
+
+    def prefix_evict(self, n: int) -> list:
+        ids = np.zeros(max(n, 1), np.int32)
+        k = ctypes.c_int32()
+        check(_L.kv_prefix_evict(self._h, n, _i32p(ids), ctypes.byref(k)), "kv_prefix_evict")
+        return ids[:k.value].tolist()
+
+    def num_cached(self) -> int:
+        n = ctypes.c_int32()
+        check(_L.kv_prefix_num_cached(self._h, ctypes.byref(n)), "kv_prefix_num_cached")
+        return n.value
+
 
 # ---------------------------------------------------------------------------
 # device calls
@@ -174,6 +208,55 @@ def paged_kv_copy_blocks(k_pool: torch.Tensor, v_pool: torch.Tensor, pairs: torc
     n = pairs.numel() // 2
     check(_L.paged_kv_copy_blocks(k_pool.data_ptr(), v_pool.data_ptr(), pairs.data_ptr(), n, Hkv, D,
                                   bs, nb, _stream(dev)), "paged_kv_copy_blocks")
+
+
+def swap_staging_bytes(k_pool: torch.Tensor, n: int) -> int:
+    """Bytes of the staging (and host) buffer of a swap of n blocks."""
+    _, Hkv, bs, D = k_pool.shape
+    return 2 * n * Hkv * bs * D * 2
+
+
+def paged_kv_swap_out(k_pool: torch.Tensor, v_pool: torch.Tensor, block_ids: torch.Tensor,
+                      staging: torch.Tensor, host: Optional[torch.Tensor] = None) -> None:
+    """K and V of ``block_ids`` (device int32) -> ``staging`` (device, uint8 or
+    fp16) -> ``host`` (pinned CPU tensor of the same byte size, optional)."""
+    dev = k_pool.device
+    _need(k_pool, "k_pool", torch.float16, dev)
+    _need(v_pool, "v_pool", torch.float16, dev)
+    _need(block_ids, "block_ids", torch.int32, dev)
+    nb, Hkv, bs, D = k_pool.shape
+    n = block_ids.numel()
+    _swap_buffers(staging, host, dev, swap_staging_bytes(k_pool, n))
+    check(_L.paged_kv_swap_out(k_pool.data_ptr(), v_pool.data_ptr(), block_ids.data_ptr(), n,
+                               staging.data_ptr(), host.data_ptr() if host is not None else None, Hkv,
+                               D, bs, nb, _stream(dev)), "paged_kv_swap_out")
+
+
+def paged_kv_swap_in(k_pool: torch.Tensor, v_pool: torch.Tensor, block_ids: torch.Tensor,
+                     staging: torch.Tensor, host: Optional[torch.Tensor] = None) -> None:
+    """``host`` (optional) -> ``staging`` -> K and V of ``block_ids``."""
+    dev = k_pool.device
+    _need(k_pool, "k_pool", torch.float16, dev)
+    _need(v_pool, "v_pool", torch.float16, dev)
+    _need(block_ids, "block_ids", torch.int32, dev)
+    nb, Hkv, bs, D = k_pool.shape
+    n = block_ids.numel()
+    _swap_buffers(staging, host, dev, swap_staging_bytes(k_pool, n))
+    check(_L.paged_kv_swap_in(k_pool.data_ptr(), v_pool.data_ptr(), block_ids.data_ptr(), n,
+                              staging.data_ptr(), host.data_ptr() if host is not None else None, Hkv,
+                              D, bs, nb, _stream(dev)), "paged_kv_swap_in")
+
+
+def _swap_buffers(staging, host, dev, nbytes):
+    if staging.device != dev or not staging.is_contiguous():
+        raise ValueError("staging must be a contiguous tensor on the pools' device")
+    if staging.numel() * staging.element_size() < nbytes:
+        raise ValueError(f"staging holds fewer than {nbytes} bytes")
+    if host is not None:
+        if host.device.type != "cpu" or not host.is_contiguous():
+            raise ValueError("host must be a contiguous CPU tensor")
+        if host.numel() * host.element_size() < nbytes:
+            raise ValueError(f"host holds fewer than {nbytes} bytes")
 
 
 def workspace_size(Hq: int, Hkv: int, q_len: int, head_dim: int, grid_ctas: int = 0) -> int:

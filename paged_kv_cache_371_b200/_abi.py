@@ -66,6 +66,12 @@ SIGNATURES = {
                                  _i32, _i32, _i32, _i32, _P], ctypes.c_int),
     "paged_decode_attention_static_ws": ([_P, _P, _P, _P, _i32, _P, ctypes.c_float, _P, _i32,
                                           _i32, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
+    "kv_prefix_match": ([_P, _PI32, _i32, _PI32, _i32, _PI32], ctypes.c_int),
+    "kv_prefix_register": ([_P, _PI32, _i32, _PI32, _i32, _PI32], ctypes.c_int),
+    "kv_prefix_evict": ([_P, _i32, _PI32, _PI32], ctypes.c_int),
+    "kv_prefix_num_cached": ([_P, _PI32], ctypes.c_int),
+    "paged_kv_swap_out": ([_P, _P, _P, _i32, _P, _P, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
+    "paged_kv_swap_in": ([_P, _P, _P, _i32, _P, _P, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
 }
 
 

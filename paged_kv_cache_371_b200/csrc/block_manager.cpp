@@ -20,13 +20,8 @@
 #include <vector>
 
 #include "../../include/paged_kv.h"
+#include "kv_pool_impl.h"
 #include "kv_status.h"
-
-struct kv_pool {
-    kv_pool_config cfg;
-    std::vector<int32_t> refcount;   // 0 = free
-    std::vector<int32_t> free_stack; // top = back()
-};
 
 namespace {
 

@@ -73,7 +73,68 @@ __global__ void copy_blocks_kernel(uint4* __restrict__ k_pool, uint4* __restrict
     }
 }
 
+// Swap staging: [2 (K, V)][n][block chunks].  to_pool = 0: pool blocks ids[i]
+// -> staging row i; 1: the reverse.  Out-of-range ids are skipped and flagged.
+__global__ void swap_blocks_kernel(uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
+                                   const int32_t* __restrict__ ids, int32_t n,
+                                   uint4* __restrict__ staging, int64_t chunks_per_block,
+                                   int32_t num_blocks, int to_pool, int* err)
+{
+    const int32_t i = blockIdx.y;
+    const int32_t b = __ldg(ids + i);
+    if (b < 0 || b >= num_blocks) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(err, KV_DEV_BAD_BLOCK);
+        return;
+    }
+    uint4* kp = k_pool + (int64_t)b * chunks_per_block;
+    uint4* vp = v_pool + (int64_t)b * chunks_per_block;
+    uint4* ks = staging + (int64_t)i * chunks_per_block;
+    uint4* vs = staging + ((int64_t)n + i) * chunks_per_block;
+    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < chunks_per_block;
+         c += (int64_t)gridDim.x * blockDim.x) {
+        if (to_pool) {
+            kp[c] = ks[c];
+            vp[c] = vs[c];
+        } else {
+            ks[c] = kp[c];
+            vs[c] = vp[c];
+        }
+    }
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int swap_impl(void* k_pool, void* v_pool, const int32_t* ids, int32_t n, void* staging, void* host,
+              int32_t Hkv, int32_t head_dim, int32_t block_size, int32_t num_blocks, int to_pool,
+              void* stream, const char* name)
+{
+    if (n < 0 || n > 65535 || Hkv <= 0 || head_dim <= 0 || head_dim % 8 != 0 || block_size <= 0 ||
+        num_blocks <= 0)
+        return kv_fail(KV_ERR_INVALID, name);
+    if (n == 0) return KV_OK;
+    if (!k_pool || !v_pool || !ids || !staging) return kv_fail(KV_ERR_INVALID, name);
+    if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned16(staging))
+        return kv_fail(KV_ERR_INVALID, name);
+    int* err = kv_error_word_ptr();
+    if (!err) return kv_fail(KV_ERR_CUDA, name);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t cpb = (int64_t)Hkv * block_size * head_dim / 8;
+    const size_t bytes = (size_t)2 * n * cpb * 16;
+    int rc;
+    if (to_pool && host &&
+        (rc = kv_cuda_check(cudaMemcpyAsync(staging, host, bytes, cudaMemcpyHostToDevice, st), name)) != KV_OK)
+        return rc;
+    const int threads = 256;
+    int64_t bx = (cpb + threads - 1) / threads;
+    if (bx > 64) bx = 64;
+    swap_blocks_kernel<<<dim3((unsigned)bx, (unsigned)n), threads, 0, st>>>(
+        static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), ids, n, static_cast<uint4*>(staging),
+        cpb, num_blocks, to_pool, err);
+    if ((rc = kv_cuda_check(cudaGetLastError(), name)) != KV_OK) return rc;
+    if (!to_pool && host)
+        return kv_cuda_check(cudaMemcpyAsync(host, staging, bytes, cudaMemcpyDeviceToHost, st), name);
+    return KV_OK;
+}
 
 }  // namespace
 
@@ -146,6 +207,22 @@ int paged_kv_copy_blocks(void* k_pool, void* v_pool, const int32_t* pairs, int32
     copy_blocks_kernel<<<grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), pairs, n, cpb, num_blocks, err);
     return kv_cuda_check(cudaGetLastError(), "paged_kv_copy_blocks");
+}
+
+int paged_kv_swap_out(const void* k_pool, const void* v_pool, const int32_t* block_ids, int32_t n,
+                      void* staging, void* host, int32_t Hkv, int32_t head_dim, int32_t block_size,
+                      int32_t num_blocks, void* stream)
+{
+    return swap_impl(const_cast<void*>(k_pool), const_cast<void*>(v_pool), block_ids, n, staging, host,
+                     Hkv, head_dim, block_size, num_blocks, 0, stream, "paged_kv_swap_out: bad argument");
+}
+
+int paged_kv_swap_in(void* k_pool, void* v_pool, const int32_t* block_ids, int32_t n, void* staging,
+                     const void* host, int32_t Hkv, int32_t head_dim, int32_t block_size,
+                     int32_t num_blocks, void* stream)
+{
+    return swap_impl(k_pool, v_pool, block_ids, n, staging, const_cast<void*>(host), Hkv, head_dim,
+                     block_size, num_blocks, 1, stream, "paged_kv_swap_in: bad argument");
 }
 
 int kv_device_error(int32_t* word_out, int32_t reset, void* stream)
