@@ -49,6 +49,13 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oracle_append.restype = ctypes.c_int
     L.oracle_copy_blocks.argtypes = [P, i32, i32, i32, i32, i32, P, P]
     L.oracle_copy_blocks.restype = ctypes.c_int
+    L.oracle_k_scales.argtypes = [P, ctypes.c_int64, i32, i32, P]
+    L.oracle_k_scales.restype = ctypes.c_int
+    L.oracle_append_q8k.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, P, P]
+    L.oracle_append_q8k.restype = ctypes.c_int
+    L.oracle_paged_attention_q8k.argtypes = [P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, i32,
+                                             i32, ctypes.c_double, P]
+    L.oracle_paged_attention_q8k.restype = ctypes.c_int
     return L
 
 
@@ -146,3 +153,60 @@ def copy_blocks(k_pool, v_pool, pairs, L: ctypes.CDLL | None = None):
     if rc != 0:
         raise ValueError(f"oracle_copy_blocks rejected its inputs (code {rc})")
     return k16.view(np.float16), v16.view(np.float16)
+
+
+# -- quantised K pool (int8 codes, one fp32 scale per KV head and channel) --
+def k_scales(k, L: ctypes.CDLL | None = None) -> np.ndarray:
+    """Per-(KV head, channel) scales max|k| / 127 of calibration keys
+    k: fp16 [T][Hkv][D] -> fp32 [Hkv][D]."""
+    L = L or lib()
+    k16 = _as_u16(k)
+    T, Hkv, D = k16.shape
+    out = np.zeros((Hkv, D), np.float32)
+    rc = L.oracle_k_scales(_ptr(k16), T, Hkv, D, _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_k_scales rejected its inputs (code {rc})")
+    return out
+
+
+def append_q8k(kq_pool, v_pool, k_new, v_new, slot_mapping, scales, L: ctypes.CDLL | None = None):
+    """Return copies of the code pool (int8) and V pool with the new tokens
+    written: K quantised with ``scales``, V as is."""
+    L = L or lib()
+    k8 = np.ascontiguousarray(kq_pool, dtype=np.int8).copy()
+    v16 = _as_u16(v_pool).copy()
+    nb, Hkv, bs, D = k8.shape
+    kn, vn = _as_u16(k_new), _as_u16(v_new)
+    sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    sc = np.ascontiguousarray(scales, dtype=np.float32)
+    T = int(sm.shape[0])
+    assert kn.size == T * Hkv * D and vn.size == T * Hkv * D and sc.shape == (Hkv, D)
+    rc = L.oracle_append_q8k(_ptr(kn), _ptr(vn), _ptr(sm), T, Hkv, D, bs, nb, _ptr(sc), _ptr(k8),
+                             _ptr(v16))
+    if rc != 0:
+        raise ValueError(f"oracle_append_q8k rejected its inputs (code {rc})")
+    return k8, v16.view(np.float16)
+
+
+def paged_attention_q8k(q, kq_pool, scales, v_pool, block_tables, context_lens, *, scale, q_len=1,
+                        L: ctypes.CDLL | None = None) -> np.ndarray:
+    """Exact attention with K = code * scale (fp64), V fp16; as paged_attention."""
+    L = L or lib()
+    q16 = _as_u16(q)
+    k8 = np.ascontiguousarray(kq_pool, dtype=np.int8)
+    v16 = _as_u16(v_pool)
+    nb, Hkv, bs, D = k8.shape
+    sc = np.ascontiguousarray(scales, dtype=np.float32)
+    B = int(context_lens.shape[0])
+    Hq = q16.shape[-2]
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    if bt.ndim == 1:
+        bt = bt.reshape(B, -1)
+    out = np.zeros(q16.shape, dtype=np.float64)
+    rc = L.oracle_paged_attention_q8k(_ptr(q16), _ptr(k8), _ptr(sc), _ptr(v16), _ptr(bt), bt.shape[1],
+                                      _ptr(cl), B, q_len, Hq, Hkv, D, bs, nb, float(scale), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_paged_attention_q8k rejected its inputs (code {rc})")
+    return out
+

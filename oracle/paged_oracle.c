@@ -136,14 +136,17 @@ static size_t pool_row(int64_t p, int32_t kvh, int32_t o, int32_t Hkv, int32_t b
  *   M = max_t s_t,  w_t = exp(s_t - M),  Z = sum_t w_t
  *   out[s][j][h][:] = sum_t w_t V_t / Z
  * A row that sees no key (last < 0) is all zeros.
+ * K is read from an fp16 pool (k16), or from an 8-bit code pool (k8) as
+ * code * k_scales[kvh][d] (see the quantised pool below).
  * Returns ORACLE_ERR_TABLE if a table entry that is read lies outside
  * [0, num_blocks), ORACLE_ERR_ARG on bad sizes.
  */
-int oracle_paged_attention(const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
-                           const int32_t* block_tables, int32_t max_blocks_per_seq,
-                           const int32_t* context_lens, int32_t B, int32_t q_len, int32_t Hq,
-                           int32_t Hkv, int32_t D, int32_t bs, int32_t num_blocks, double scale,
-                           double* out)
+static int attention_rows(const uint16_t* q, const uint16_t* k16, const int8_t* k8,
+                          const float* k_scales, const uint16_t* v_pool,
+                          const int32_t* block_tables, int32_t max_blocks_per_seq,
+                          const int32_t* context_lens, int32_t B, int32_t q_len, int32_t Hq,
+                          int32_t Hkv, int32_t D, int32_t bs, int32_t num_blocks, double scale,
+                          double* out)
 {
     if (B < 0 || q_len < 1 || Hq < 1 || Hkv < 1 || D < 1 || bs < 1 || Hq % Hkv != 0)
         return ORACLE_ERR_ARG;
@@ -180,9 +183,13 @@ int oracle_paged_attention(const uint16_t* q, const uint16_t* k_pool, const uint
         double M = -INFINITY;
         for (int32_t t = 0; t < n; ++t) {
             int32_t p = block_tables[(size_t)s * max_blocks_per_seq + t / bs];
-            const uint16_t* krow = k_pool + pool_row(p, kvh, t % bs, Hkv, bs, D);
+            const size_t row = pool_row(p, kvh, t % bs, Hkv, bs, D);
             double dot = 0.0;
-            for (int32_t d = 0; d < D; ++d) dot += qd[d] * oracle_half_to_double(krow[d]);
+            for (int32_t d = 0; d < D; ++d) {
+                const double kd = k8 ? (double)k8[row + d] * (double)k_scales[(size_t)kvh * D + d]
+                                     : oracle_half_to_double(k16[row + d]);
+                dot += qd[d] * kd;
+            }
             sc[t] = scale * dot;
             if (sc[t] > M) M = sc[t];
         }
@@ -203,6 +210,83 @@ int oracle_paged_attention(const uint16_t* q, const uint16_t* k_pool, const uint
         free(sc);
     }
     return ORACLE_OK;
+}
+
+int oracle_paged_attention(const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
+                           const int32_t* block_tables, int32_t max_blocks_per_seq,
+                           const int32_t* context_lens, int32_t B, int32_t q_len, int32_t Hq,
+                           int32_t Hkv, int32_t D, int32_t bs, int32_t num_blocks, double scale,
+                           double* out)
+{
+    return attention_rows(q, k_pool, NULL, NULL, v_pool, block_tables, max_blocks_per_seq,
+                          context_lens, B, q_len, Hq, Hkv, D, bs, num_blocks, scale, out);
+}
+
+/*
+ * Quantised K pool.  [T2] §"KV Cache量化": INT8 KV caches; keys are quantised
+ * per channel (KVQuant), because their distribution is uneven across
+ * channels.  [T3] §4.2: keys per channel at low bit width, values stay FP16.
+ * Reading (the printed pseudo-code divides the maximum by 2^bits - 1 but
+ * clamps to the signed range, and takes a signed maximum): symmetric 8-bit
+ * codes, one scale per (KV head, channel) fixed from calibration tokens,
+ *   scale[h][d] = max_t |K[t][h][d]| / 127   (1 for an all-zero channel),
+ *   code = clamp(rint(k / scale), -128, 127),   K~ = code * scale.
+ * Codes are integers decided by floating point, so they are computed in the
+ * kernel's precision: fp32, correctly rounded division, round half to even.
+ * Code pool: int8 [num_blocks][Hkv][bs][D]; scales: fp32 [Hkv][D].
+ */
+int oracle_k_scales(const uint16_t* k, int64_t T, int32_t Hkv, int32_t D, float* scales)
+{
+    if (T < 0 || Hkv < 1 || D < 1) return ORACLE_ERR_ARG;
+    for (int32_t h = 0; h < Hkv; ++h)
+        for (int32_t d = 0; d < D; ++d) {
+            double amax = 0.0;
+            for (int64_t t = 0; t < T; ++t) {
+                const double v = fabs(oracle_half_to_double(k[((size_t)t * Hkv + h) * D + d]));
+                if (v > amax) amax = v;
+            }
+            /* |fp16| is exact in fp32; one correctly rounded fp32 division */
+            scales[(size_t)h * D + d] = amax > 0.0 ? (float)amax / 127.0f : 1.0f;
+        }
+    return ORACLE_OK;
+}
+
+static int8_t k_code(uint16_t k, float scale)
+{
+    const float r = rintf((float)oracle_half_to_double(k) / scale);
+    return (int8_t)(r < -128.0f ? -128.0f : (r > 127.0f ? 127.0f : r));
+}
+
+int oracle_append_q8k(const uint16_t* new_k, const uint16_t* new_v, const int64_t* slot_mapping,
+                      int32_t T, int32_t Hkv, int32_t D, int32_t bs, int32_t num_blocks,
+                      const float* k_scales, int8_t* kq_pool, uint16_t* v_pool)
+{
+    for (int32_t t = 0; t < T; ++t)
+        if (slot_mapping[t] >= (int64_t)num_blocks * bs) return ORACLE_ERR_ARG;
+    for (int32_t t = 0; t < T; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        int64_t p = slot / bs;
+        int32_t o = (int32_t)(slot % bs);
+        for (int32_t h = 0; h < Hkv; ++h) {
+            for (int32_t d = 0; d < D; ++d) {
+                const size_t src = ((size_t)t * Hkv + h) * D + d;
+                kq_pool[pool_row(p, h, o, Hkv, bs, D) + d] = k_code(new_k[src], k_scales[(size_t)h * D + d]);
+                v_pool[pool_row(p, h, o, Hkv, bs, D) + d] = new_v[src];
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+int oracle_paged_attention_q8k(const uint16_t* q, const int8_t* kq_pool, const float* k_scales,
+                               const uint16_t* v_pool, const int32_t* block_tables,
+                               int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t B,
+                               int32_t q_len, int32_t Hq, int32_t Hkv, int32_t D, int32_t bs,
+                               int32_t num_blocks, double scale, double* out)
+{
+    return attention_rows(q, NULL, kq_pool, k_scales, v_pool, block_tables, max_blocks_per_seq,
+                          context_lens, B, q_len, Hq, Hkv, D, bs, num_blocks, scale, out);
 }
 
 /*

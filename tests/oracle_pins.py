@@ -285,6 +285,79 @@ def pin_copy_blocks(L):
     assert np.array_equal(V2.view(np.uint16), refV.view(np.uint16))
 
 
+def pin_q8k_attention_exact_scales(L):
+    """Power-of-two scales make every dequantised key an fp16 value: attention
+    over the codes must equal the fp16 attention on those values bit for bit
+    (scale factor, its (head, channel) index, code pool layout)."""
+    rng = _rng(61)
+    nb, Hkv, bs, D, Hq = 12, 2, 4, 16, 4
+    codes = rng.integers(-128, 128, size=(nb, Hkv, bs, D)).astype(np.int8)
+    scales = np.ldexp(1.0, -rng.integers(3, 9, size=(Hkv, D))).astype(np.float32)
+    exact = codes.astype(np.float64) * scales[None, :, None, :].astype(np.float64)
+    kdq = exact.astype(np.float16)
+    assert np.array_equal(kdq.astype(np.float64), exact)
+    V = _f16(rng, (nb, Hkv, bs, D))
+    lens = np.array([13, 20, 1], np.int32)
+    perm = rng.permutation(nb).astype(np.int32)
+    tables = np.full((3, 5), -1, np.int32)
+    tables[0, :4], tables[1, :5], tables[2, :1] = perm[:4], perm[4:9], perm[9:10]
+    q = _f16(rng, (3, 1, Hq, D))
+    got = oracle.paged_attention_q8k(q, codes, scales, V, tables, lens, scale=0.25, L=L)
+    ref = oracle.paged_attention(q, kdq, V, tables, lens, scale=0.25, L=L)
+    assert np.array_equal(got, ref)
+
+
+def pin_q8k_codes(L):
+    """Scales and codes: the channel maximum maps to +-127, the round trip
+    stays within half a step, codes are odd in k, exact half steps round to
+    even and clamp at the ends, and codes land where the fp16 append puts K."""
+    rng = _rng(71)
+    T, Hkv, D = 40, 3, 8
+    k = _f16(rng, (T, Hkv, D), 2.0)
+    k[:, 2, 5] = 0                                   # an all-zero channel
+    sc = oracle.k_scales(k, L=L)
+    assert sc.shape == (Hkv, D) and sc[2, 5] == 1.0
+    kf = k.astype(np.float64)
+    amax = np.abs(kf).max(axis=0)
+    live = amax > 0
+    # ~ max|k| / 127 (the step that spans the symmetric 8-bit range)
+    np.testing.assert_allclose(sc[live], amax[live] / 127.0, rtol=1e-6)
+    slots = np.arange(T, dtype=np.int64)
+    zk = np.zeros((T, Hkv, 1, D), np.int8)
+    zv = np.zeros((T, Hkv, 1, D), np.float16)
+    K8, V2 = oracle.append_q8k(zk, zv, k, -k, slots, sc, L=L)
+    c = K8[:, :, 0, :].astype(np.int64)
+    assert np.array_equal(V2[:, :, 0, :].view(np.uint16), (-k).view(np.uint16))
+    arg = np.abs(kf).argmax(axis=0)
+    top = np.take_along_axis(c, arg[None], axis=0)[0]
+    assert np.array_equal(top[live], np.sign(np.take_along_axis(kf, arg[None], axis=0)[0])[live] * 127)
+    assert np.all(np.abs(c * sc.astype(np.float64)[None] - kf) <= sc.astype(np.float64)[None] * (0.5 + 1e-6))
+    Kn, _ = oracle.append_q8k(zk, zv, -k, k, slots, sc, L=L)
+    assert np.array_equal(Kn.astype(np.int64), -K8.astype(np.int64))
+    # half steps with an exact scale of 1/4
+    half = np.array([0.125, 0.375, -0.125, -0.375, 0.625, 31.875, -32.125, 33.0, -33.0], np.float16)
+    want = np.array([0, 2, 0, -2, 2, 127, -128, 127, -128], np.int64)
+    n = half.size
+    hk = np.zeros((n, 1, D), np.float16)
+    hk[:, 0, 3] = half
+    s4 = np.full((1, D), 0.25, np.float32)
+    H8, _ = oracle.append_q8k(np.zeros((n, 1, 1, D), np.int8), np.zeros((n, 1, 1, D), np.float16),
+                              hk, hk, np.arange(n, dtype=np.int64), s4, L=L)
+    assert np.array_equal(H8[:, 0, 0, 3].astype(np.int64), want)
+    # placement: exact multiples of power-of-two scales go where the fp16
+    # append puts them
+    nb, bs = 5, 4
+    p2 = np.ldexp(1.0, -rng.integers(2, 6, size=(Hkv, D))).astype(np.float32)
+    cc = rng.integers(-127, 128, size=(7, Hkv, D))
+    kk = (cc * p2[None].astype(np.float64)).astype(np.float16)
+    sl = np.array([3, 17, -1, 0, 9, 12, 19], np.int64)
+    Q8, _ = oracle.append_q8k(np.zeros((nb, Hkv, bs, D), np.int8), np.zeros((nb, Hkv, bs, D), np.float16),
+                              kk, kk, sl, p2, L=L)
+    F16, _ = oracle.append(np.zeros((nb, Hkv, bs, D), np.float16), np.zeros((nb, Hkv, bs, D), np.float16),
+                           kk, kk, sl, L=L)
+    assert np.array_equal(Q8.astype(np.float64) * p2[None, :, None, :], F16.astype(np.float64))
+
+
 PINS = [pin_half_decoding, pin_memory_formula, pin_attention_vs_sdpa, pin_permutation_invariance,
         pin_brute_force, pin_verify_causal, pin_closed_forms, pin_shared_prefix_equals_private,
-        pin_append, pin_copy_blocks]
+        pin_append, pin_copy_blocks, pin_q8k_attention_exact_scales, pin_q8k_codes]

@@ -25,7 +25,14 @@ MUTANTS = {
     "softmax_sign": ("double w = exp(sc[t] - M);", "double w = exp(M - sc[t]);"),
     "table_index_offset": ("int32_t p = block_tables[(size_t)s * max_blocks_per_seq + t / bs];\n            const uint16_t* vrow",
                            "int32_t p = block_tables[(size_t)s * max_blocks_per_seq + (t + 1) / bs];\n            const uint16_t* vrow"),
-    "append_slot_split": ("int32_t o = (int32_t)(slot % bs);", "int32_t o = (int32_t)(slot / num_blocks);"),
+    "append_slot_split": ("int32_t o = (int32_t)(slot % bs);\n        for (int32_t h = 0; h < Hkv; ++h) {\n            for (int32_t d = 0; d < D; ++d) {\n                k_pool",
+                          "int32_t o = (int32_t)(slot / num_blocks);\n        for (int32_t h = 0; h < Hkv; ++h) {\n            for (int32_t d = 0; d < D; ++d) {\n                k_pool"),
+    "q8k_scale_dropped": ("(double)k8[row + d] * (double)k_scales[(size_t)kvh * D + d]", "(double)k8[row + d]"),
+    "q8k_scale_ignores_head": ("(double)k_scales[(size_t)kvh * D + d]", "(double)k_scales[(size_t)d]"),
+    "q8k_truncating_round": ("rintf(", "truncf("),
+    "q8k_scale_over_255": ("(float)amax / 127.0f", "(float)amax / 255.0f"),
+    "q8k_append_scale_ignores_head": ("k_code(new_k[src], k_scales[(size_t)h * D + d])", "k_code(new_k[src], k_scales[(size_t)d])"),
+    "q8k_no_clamp": ("(r > 127.0f ? 127.0f : r)", "r"),
     "append_k_only": ("v_pool[pool_row(p, h, o, Hkv, bs, D) + d] = new_v[((size_t)t * Hkv + h) * D + d];",
                       "v_pool[pool_row(p, h, o, Hkv, bs, D) + d] = new_k[((size_t)t * Hkv + h) * D + d];"),
     "copy_direction": ("k_pool[dst + e] = k_pool[src + e];", "k_pool[src + e] = k_pool[dst + e];"),
