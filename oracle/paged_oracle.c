@@ -233,6 +233,8 @@ int oracle_paged_attention(const uint16_t* q, const uint16_t* k_pool, const uint
  *   code = clamp(rint(k / scale), -128, 127),   K~ = code * scale.
  * Codes are integers decided by floating point, so they are computed in the
  * kernel's precision: fp32, correctly rounded division, round half to even.
+ * The pages say nothing of non-finite keys: +-inf clamp like any large value,
+ * and a NaN (e.g. an unwritten slot, never attended) stores code 0.
  * Code pool: int8 [num_blocks][Hkv][bs][D]; scales: fp32 [Hkv][D].
  */
 int oracle_k_scales(const uint16_t* k, int64_t T, int32_t Hkv, int32_t D, float* scales)
@@ -254,6 +256,7 @@ int oracle_k_scales(const uint16_t* k, int64_t T, int32_t Hkv, int32_t D, float*
 static int8_t k_code(uint16_t k, float scale)
 {
     const float r = rintf((float)oracle_half_to_double(k) / scale);
+    if (isnan(r)) return 0; /* a NaN key (an unwritten slot) stores code 0 */
     return (int8_t)(r < -128.0f ? -128.0f : (r > 127.0f ? 127.0f : r));
 }
 

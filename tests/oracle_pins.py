@@ -335,8 +335,9 @@ def pin_q8k_codes(L):
     Kn, _ = oracle.append_q8k(zk, zv, -k, k, slots, sc, L=L)
     assert np.array_equal(Kn.astype(np.int64), -K8.astype(np.int64))
     # half steps with an exact scale of 1/4
-    half = np.array([0.125, 0.375, -0.125, -0.375, 0.625, 31.875, -32.125, 33.0, -33.0], np.float16)
-    want = np.array([0, 2, 0, -2, 2, 127, -128, 127, -128], np.int64)
+    half = np.array([0.125, 0.375, -0.125, -0.375, 0.625, 31.875, -32.125, 33.0, -33.0,
+                     np.inf, -np.inf, np.nan], np.float16)
+    want = np.array([0, 2, 0, -2, 2, 127, -128, 127, -128, 127, -128, 0], np.int64)
     n = half.size
     hk = np.zeros((n, 1, D), np.float16)
     hk[:, 0, 3] = half
