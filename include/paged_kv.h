@@ -56,6 +56,7 @@ extern "C" {
 #define KV_DEV_BAD_BLOCK 1   /* a block-table entry outside [0, num_blocks) */
 #define KV_DEV_BAD_SLOT 2    /* an append slot beyond the pool */
 #define KV_DEV_TIMEOUT 4     /* a pipeline wait ran past its limit */
+#define KV_DEV_BAD_SCALE 8   /* a K scale that is not positive and finite */
 
 /* Text of the last error raised on the calling thread ("" if none). */
 const char* kv_last_error_string(void);
@@ -184,6 +185,38 @@ int paged_kv_append(const void* k_new, const void* v_new, const int64_t* slot_ma
 int paged_kv_copy_blocks(void* k_pool, void* v_pool, const int32_t* pairs, int32_t n,
                          int32_t Hkv, int32_t head_dim, int32_t block_size, int32_t num_blocks,
                          void* stream);
+
+/* Quantised K pool ([T2] §"KV Cache量化": INT8 KV caches, keys quantised per
+ * channel as in KVQuant; [T3] §4.2: keys per channel at low bit width, values
+ * kept in FP16).  The K pool holds int8 codes [num_blocks][Hkv][bs][D] (half
+ * the bytes of fp16), the V pool stays fp16; one fp32 scale per (KV head,
+ * channel), k_scales [Hkv][D], fixed by the caller (e.g. from calibration
+ * tokens with paged_kv_k_scales).  Key t of head h is code * k_scales[h][d].
+ *
+ * paged_kv_k_scales: k_scales[h][d] = max_t |k[t][h][d]| / 127 over the
+ * DEVICE fp16 tokens k [T][Hkv][D] (1 for an all-zero channel); fp32,
+ * correctly rounded division. */
+int paged_kv_k_scales(const void* k, int64_t T, int32_t Hkv, int32_t head_dim, float* k_scales,
+                      void* stream);
+/* paged_kv_append_q8k: paged_kv_append with K written as codes
+ *   code = clamp(rint(k / k_scales[h][d]), -128, 127)
+ * (fp32, correctly rounded division, round half to even: bit-exact and
+ * reproducible on the host) and V copied; a NaN key stores code 0.  A scale
+ * that is not positive and finite writes code 0 and flags KV_DEV_BAD_SCALE. */
+int paged_kv_append_q8k(const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                        const float* k_scales, void* kq_pool, void* v_pool, int32_t T, int32_t Hkv,
+                        int32_t head_dim, int32_t block_size, int32_t num_blocks, void* stream);
+/* paged_attention_q8k: paged_verify_attention (q_len = 1: decode) over an int8
+ * K pool: scores use key t = code * k_scales[kvh][:].  The scales are folded
+ * into q once per (sequence, kv head) segment (q_d * k_scales[d], rounded to
+ * fp16); codes are exact fp16 integers, so the products stay exact in fp32.
+ * Requires head_dim 128; k_scales device, 8-byte aligned; workspace as for
+ * paged_attention_workspace_size.  Otherwise as paged_verify_attention. */
+int paged_attention_q8k(const void* q, const void* kq_pool, const float* k_scales,
+                        const void* v_pool, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                        const int32_t* context_lens, int32_t q_len, float scale, void* out,
+                        int32_t B, int32_t Hq, int32_t Hkv, int32_t head_dim, int32_t block_size,
+                        int32_t num_blocks, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Block swap between the pools and host memory ([T3] §2.3 (1): when the pool
  * is full, a preempted request's blocks are moved to CPU memory and brought

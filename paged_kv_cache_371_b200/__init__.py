@@ -23,7 +23,8 @@ from ._abi import KVError, check
 __all__ = ["KVPool", "KVError", "pool_bytes", "paged_kv_append", "paged_kv_copy_blocks",
            "workspace_size", "paged_decode_attention", "paged_verify_attention",
            "paged_attention", "paged_prefill_attention", "paged_kv_swap_out", "paged_kv_swap_in",
-           "swap_staging_bytes", "device_error", "lib"]
+           "swap_staging_bytes", "paged_kv_k_scales", "paged_kv_append_q8k", "paged_attention_q8k",
+           "device_error", "lib"]
 
 _L = _abi.load()
 
@@ -267,10 +268,15 @@ def workspace_size(Hq: int, Hkv: int, q_len: int, head_dim: int, grid_ctas: int 
 
 
 def _attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len, out, workspace,
-               grid_ctas, min_split_blocks, use_pdl, entry, seg_cost_blocks=0):
+               grid_ctas, min_split_blocks, use_pdl, entry, seg_cost_blocks=0, k_scales=None):
     dev = k_pool.device
-    for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool")):
+    _need(k_pool, "k_pool", torch.int8 if entry == "q8k" else torch.float16, dev)
+    for t, n in ((q, "q"), (v_pool, "v_pool")):
         _need(t, n, torch.float16, dev)
+    if entry == "q8k":
+        _need(k_scales, "k_scales", torch.float32, dev)
+        if tuple(k_scales.shape) != (k_pool.shape[1], k_pool.shape[3]):
+            raise ValueError("k_scales must be [Hkv][D]")
     _need(block_tables, "block_tables", torch.int32, dev)
     _need(context_lens, "context_lens", torch.int32, dev)
     nb, Hkv, bs, D = k_pool.shape
@@ -298,11 +304,52 @@ def _attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len, out,
         rc = _L.paged_decode_attention(*args, *tail, _stream(dev))
     elif entry == "verify":
         rc = _L.paged_verify_attention(*args, q_len, *tail, _stream(dev))
+    elif entry == "q8k":
+        rc = _L.paged_attention_q8k(q.data_ptr(), k_pool.data_ptr(), k_scales.data_ptr(),
+                                    v_pool.data_ptr(), block_tables.data_ptr(), mb,
+                                    context_lens.data_ptr(), q_len, *tail, _stream(dev))
     else:
         o = _abi.PagedAttentionOpts(grid_ctas, min_split_blocks, use_pdl, seg_cost_blocks)
         rc = _L.paged_attention_ex(*args, q_len, *tail, ctypes.byref(o), _stream(dev))
     check(rc, f"paged attention ({entry})")
     return out
+
+
+def paged_kv_k_scales(k: torch.Tensor) -> torch.Tensor:
+    """Per-(KV head, channel) scales max|k| / 127 of calibration keys
+    k [T][Hkv][D] fp16 (device) -> fp32 [Hkv][D]."""
+    dev = k.device
+    _need(k, "k", torch.float16, dev)
+    T, Hkv, D = k.shape
+    out = torch.empty((Hkv, D), dtype=torch.float32, device=dev)
+    check(_L.paged_kv_k_scales(k.data_ptr(), T, Hkv, D, out.data_ptr(), _stream(dev)),
+          "paged_kv_k_scales")
+    return out
+
+
+def paged_kv_append_q8k(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor,
+                        k_scales: torch.Tensor, kq_pool: torch.Tensor, v_pool: torch.Tensor) -> None:
+    """Append with K quantised to int8 codes (per-channel scales), V as fp16."""
+    dev = v_pool.device
+    _need(kq_pool, "kq_pool", torch.int8, dev)
+    for t, n in ((v_pool, "v_pool"), (k_new, "k_new"), (v_new, "v_new")):
+        _need(t, n, torch.float16, dev)
+    _need(k_scales, "k_scales", torch.float32, dev)
+    _need(slot_mapping, "slot_mapping", torch.int64, dev)
+    nb, Hkv, bs, D = kq_pool.shape
+    if tuple(v_pool.shape) != (nb, Hkv, bs, D) or tuple(k_scales.shape) != (Hkv, D):
+        raise ValueError("pool / scale shapes disagree")
+    T = slot_mapping.numel()
+    check(_L.paged_kv_append_q8k(k_new.data_ptr(), v_new.data_ptr(), slot_mapping.data_ptr(),
+                                 k_scales.data_ptr(), kq_pool.data_ptr(), v_pool.data_ptr(), T, Hkv,
+                                 D, bs, nb, _stream(dev)), "paged_kv_append_q8k")
+
+
+def paged_attention_q8k(q, kq_pool, k_scales, v_pool, block_tables, context_lens, scale, q_len=1,
+                        out=None, workspace=None):
+    """Decode (q_len = 1) or causal verify attention over an int8 K pool."""
+    return _attention(q, kq_pool, v_pool, block_tables, context_lens, scale, q_len, out, workspace,
+                      0, 0, 0, "q8k", k_scales=k_scales)
 
 
 def paged_decode_attention(q, k_pool, v_pool, block_tables, context_lens, scale, out=None,

@@ -15,6 +15,7 @@ KV_ERR_CUDA = 4
 KV_DEV_BAD_BLOCK = 1
 KV_DEV_BAD_SLOT = 2
 KV_DEV_TIMEOUT = 4
+KV_DEV_BAD_SCALE = 8
 
 
 class KvPoolConfig(ctypes.Structure):
@@ -72,6 +73,10 @@ SIGNATURES = {
     "kv_prefix_num_cached": ([_P, _PI32], ctypes.c_int),
     "paged_kv_swap_out": ([_P, _P, _P, _i32, _P, _P, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
     "paged_kv_swap_in": ([_P, _P, _P, _i32, _P, _P, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
+    "paged_kv_k_scales": ([_P, ctypes.c_int64, _i32, _i32, _P, _P], ctypes.c_int),
+    "paged_kv_append_q8k": ([_P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
+    "paged_attention_q8k": ([_P, _P, _P, _P, _P, _i32, _P, _i32, ctypes.c_float, _P, _i32, _i32, _i32,
+                             _i32, _i32, _i32, _P, _sz, _P], ctypes.c_int),
 }
 
 

@@ -7,6 +7,7 @@
 // §2.3 (2) of the same page (the block a beam writes into is copied first).
 // Both are plain byte moves: 16-byte vector loads/stores, fully coalesced
 // within each (token, head) row and each block.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -71,6 +72,70 @@ __global__ void copy_blocks_kernel(uint4* __restrict__ k_pool, uint4* __restrict
         kd[c] = ks[c];
         vd[c] = vs[c];
     }
+}
+
+// Quantised K ("大模型推理加速：从 KV Cache 到投机采样的工程实践" §"KV Cache量化":
+// keys per channel; "LLM 推理优化：KV Cache、PagedAttention 与量化" §4.2: keys
+// at low bit width per channel, values FP16): code = clamp(rint(k / s), -128,
+// 127) with one fp32 scale s per (KV head, channel); correctly rounded fp32
+// division, round half to even.  One thread per 8 channels of one (token,
+// head) row: 8 codes (8 bytes) of K, 16 bytes of V.
+__global__ void append_q8k_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                                  const int64_t* __restrict__ slot_mapping,
+                                  const float* __restrict__ k_scales, uint2* __restrict__ kq_pool,
+                                  uint4* __restrict__ v_pool, int32_t T, int32_t Hkv,
+                                  int32_t chunks_per_row, int32_t bs, int64_t num_slots, int* err)
+{
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t per_tok = (int64_t)Hkv * chunks_per_row;
+    if (i >= (int64_t)T * per_tok) return;
+    const int32_t t = (int32_t)(i / per_tok);
+    const int32_t rem = (int32_t)(i % per_tok);
+    const int32_t h = rem / chunks_per_row;
+    const int32_t c = rem % chunks_per_row;
+    const int64_t slot = __ldg(slot_mapping + t);
+    if (slot < 0) return;
+    if (slot >= num_slots) {
+        if (rem == 0) atomicOr(err, KV_DEV_BAD_SLOT);
+        return;
+    }
+    const int64_t blk = slot / bs;
+    const int32_t off = (int32_t)(slot % bs);
+    const int64_t dst = ((blk * Hkv + h) * bs + off) * chunks_per_row + c;
+    const uint4 kv = __ldg(k_new + i);
+    const float* sc = k_scales + ((int64_t)h * chunks_per_row + c) * 8;
+    const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+    uint32_t packed[2] = {0u, 0u};
+    bool bad = false;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const uint32_t w = kw[e >> 1];
+        const float k = __half2float(__ushort_as_half((unsigned short)(e & 1 ? w >> 16 : w & 0xffff)));
+        const float s = __ldg(sc + e);
+        int code = 0;
+        if (s > 0.f && s <= 3.402823466e38f) {
+            const float r = rintf(__fdiv_rn(k, s));
+            code = r != r ? 0 : (int)fminf(fmaxf(r, -128.f), 127.f);  // NaN key: code 0
+        } else {
+            bad = true;
+        }
+        packed[e >> 2] |= (uint32_t)(code & 0xff) << (8 * (e & 3));
+    }
+    if (bad) atomicOr(err, KV_DEV_BAD_SCALE);
+    kq_pool[dst] = make_uint2(packed[0], packed[1]);
+    v_pool[dst] = __ldg(v_new + i);
+}
+
+// Calibration scales: s[h][d] = max_t |k[t][h][d]| / 127 (1 for an all-zero
+// channel); one thread per (head, channel), over all T tokens.
+__global__ void k_scales_kernel(const __half* __restrict__ k, int64_t T, int32_t Hkv, int32_t D,
+                                float* __restrict__ scales)
+{
+    const int32_t i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= Hkv * D) return;
+    float amax = 0.f;
+    for (int64_t t = 0; t < T; ++t) amax = fmaxf(amax, fabsf(__half2float(k[t * Hkv * D + i])));
+    scales[i] = amax > 0.f ? __fdiv_rn(amax, 127.f) : 1.f;
 }
 
 // Swap staging: [2 (K, V)][n][block chunks].  to_pool = 0: pool blocks ids[i]
@@ -207,6 +272,43 @@ int paged_kv_copy_blocks(void* k_pool, void* v_pool, const int32_t* pairs, int32
     copy_blocks_kernel<<<grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), pairs, n, cpb, num_blocks, err);
     return kv_cuda_check(cudaGetLastError(), "paged_kv_copy_blocks");
+}
+
+int paged_kv_append_q8k(const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                        const float* k_scales, void* kq_pool, void* v_pool, int32_t T, int32_t Hkv,
+                        int32_t head_dim, int32_t block_size, int32_t num_blocks, void* stream)
+{
+    if (T < 0 || Hkv <= 0 || head_dim <= 0 || head_dim % 8 != 0 || block_size <= 0 ||
+        num_blocks <= 0)
+        return kv_fail(KV_ERR_INVALID, "paged_kv_append_q8k: bad sizes");
+    if (T == 0) return KV_OK;
+    if (!k_new || !v_new || !slot_mapping || !k_scales || !kq_pool || !v_pool)
+        return kv_fail(KV_ERR_INVALID, "paged_kv_append_q8k: null pointer");
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(kq_pool) || !aligned16(v_pool) ||
+        (reinterpret_cast<uintptr_t>(k_scales) & 3u))
+        return kv_fail(KV_ERR_INVALID, "paged_kv_append_q8k: misaligned buffer");
+    int* err = kv_error_word_ptr();
+    if (!err) return kv_fail(KV_ERR_CUDA, "paged_kv_append_q8k: no device error word");
+    const int32_t cpr = head_dim / 8;
+    const int64_t total = (int64_t)T * Hkv * cpr;
+    const int threads = 256;
+    const int64_t blocks = (total + threads - 1) / threads;
+    append_q8k_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), slot_mapping, k_scales,
+        static_cast<uint2*>(kq_pool), static_cast<uint4*>(v_pool), T, Hkv, cpr, block_size,
+        (int64_t)num_blocks * block_size, err);
+    return kv_cuda_check(cudaGetLastError(), "paged_kv_append_q8k");
+}
+
+int paged_kv_k_scales(const void* k, int64_t T, int32_t Hkv, int32_t head_dim, float* scales,
+                      void* stream)
+{
+    if (T < 0 || Hkv <= 0 || head_dim <= 0 || !scales || (T > 0 && !k))
+        return kv_fail(KV_ERR_INVALID, "paged_kv_k_scales: bad argument");
+    const int n = Hkv * head_dim;
+    k_scales_kernel<<<(n + 127) / 128, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __half*>(k), T, Hkv, head_dim, scales);
+    return kv_cuda_check(cudaGetLastError(), "paged_kv_k_scales");
 }
 
 int paged_kv_swap_out(const void* k_pool, const void* v_pool, const int32_t* block_ids, int32_t n,

@@ -69,15 +69,18 @@ struct Params {
     float* part_lse;  // [grid][2][RP]
     int4* meta;       // [grid]: {s, kvh, first cta, slot in first cta} or s = -1
     int* err;
+    const float* k_scale;  // [Hkv][D] channel scales of an int8 K pool (else null)
     int32_t max_blocks, B, q_len, Hq, Hkv, G, rows, num_blocks, min_share;
     int32_t seg_cost;  // virtual blocks charged per (sequence, kv-head) segment
     float scale_log2;
 };
 
-template <int D_, int BS_, int MT_, bool FMA_>
+template <int D_, int BS_, int MT_, bool FMA_, bool KQ_ = false>
 struct Cfg {
     static constexpr int D = D_, BS = BS_, MT = MT_;
     static constexpr bool FMA = FMA_;
+    static constexpr bool KQ = KQ_;  // K pool of int8 codes with per-channel scales
+    static_assert(!KQ || D == 128, "int8 K pools are served at head_dim 128");
     static constexpr int NH = D / 64;                       // 64-column halves per row
     static constexpr int NBS = kTS / BS;                    // blocks per stage
     static constexpr int RP = FMA ? 1 : 16 * MT;            // padded rows
@@ -88,12 +91,16 @@ struct Cfg {
     static constexpr int WARPS_PER_SUBPART = (THREADS / 32 + 3) / 4;
     static constexpr int MAXREG_RAW = (16384 / (32 * WARPS_PER_SUBPART)) / 8 * 8;
     static constexpr int MAXREG = MAXREG_RAW > 255 ? 255 : MAXREG_RAW;
-    static constexpr int TILE_BYTES = BS * D * 2;           // one (block, kv-head) tile
-    static constexpr int KV_BYTES = kTS * D * 2;            // K (or V) bytes per stage
+    static constexpr int TILE_BYTES = BS * D * 2;           // one (block, kv-head) fp16 tile
+    static constexpr int KV_BYTES = kTS * D * 2;            // fp16 K (or V) bytes per stage
+    static constexpr int K_TILE_BYTES = KQ ? BS * D : TILE_BYTES;
+    static constexpr int K_BYTES = KQ ? kTS * D : KV_BYTES;
+    static constexpr int V_OFF = K_BYTES;                   // stage: K, V, query rows
     // query rows of a segment, one per 16-byte-padded row (conflict-free ldmatrix)
     static constexpr int QROW = D * 2 + 16;
     static constexpr int Q_BYTES = (RP * QROW + 1023) / 1024 * 1024;
-    static constexpr int STAGE_BYTES = 2 * KV_BYTES + Q_BYTES;
+    static constexpr int Q_OFF = K_BYTES + KV_BYTES;
+    static constexpr int STAGE_BYTES = Q_OFF + Q_BYTES;
     static constexpr int OB_STRIDE = D + 8;                 // floats per obuf row
     static constexpr int OBUF_SLICE = RP * OB_STRIDE;               // floats
     static constexpr int OBUF_BYTES = 2 * OBUF_SLICE * 4;           // two merge slices
@@ -155,6 +162,70 @@ __device__ __forceinline__ uint32_t tile_chunk(int tok, int cg)
     const int r = tok % C::BS;
     const int u = r * C::NH + (cg >> 3);
     return (uint32_t)((tok / C::BS) * C::TILE_BYTES + u * 128 + (((cg & 7) ^ (u & 7)) << 4));
+}
+
+// The same for an int8 K tile: one 128-byte unit (D = 128 codes) per token.
+template <class C>
+__device__ __forceinline__ uint32_t tile_chunk_k8(int tok, int cg)
+{
+    const int r = tok % C::BS;
+    return (uint32_t)((tok / C::BS) * C::K_TILE_BYTES + r * 128 + ((cg ^ (r & 7)) << 4));
+}
+
+// int8 codes -> exact fp16 integers: the byte x + 128 (x ^ 0x80) becomes the
+// low mantissa byte of an fp16 with exponent byte 0x64, i.e. 1024 + x + 128;
+// one half2 subtraction of 1152 leaves x.  Two codes (low 16 bits of w)
+// give one half2.
+__device__ __forceinline__ uint32_t i8x2_to_h2(uint32_t w)
+{
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, 0x5140;" : "=r"(r) : "r"(w ^ 0x8080u), "r"(0x64646464u));
+    const __half2 v = __hsub2(*reinterpret_cast<const __half2*>(&r),
+                              __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480)));
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Four codes -> two half2 (bytes 0-1, bytes 2-3).
+__device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t& lo, uint32_t& hi)
+{
+    const uint32_t u = w ^ 0x80808080u;
+    uint32_t a, b;
+    asm("prmt.b32 %0, %1, %2, 0x5140;" : "=r"(a) : "r"(u), "r"(0x64646464u));
+    asm("prmt.b32 %0, %1, %2, 0x7362;" : "=r"(b) : "r"(u), "r"(0x64646464u));
+    const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+    const __half2 va = __hsub2(*reinterpret_cast<const __half2*>(&a), bias);
+    const __half2 vb = __hsub2(*reinterpret_cast<const __half2*>(&b), bias);
+    lo = *reinterpret_cast<const uint32_t*>(&va);
+    hi = *reinterpret_cast<const uint32_t*>(&vb);
+}
+
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr)
+{
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return v;
+}
+
+// B fragments of k-step ks for the two n8 tiles (tokens t0 and t0 + 8) from an
+// int8 K stage: token t's codes of dims 16ks + 2tig, +1 (b0 / b2) and
+// 16ks + 8 + 2tig, +1 (b1 / b3), the m16n8k16 B layout.
+template <class C>
+__device__ __forceinline__ void k8_frag(uint32_t st, int t0, int ks, int tig, uint32_t& b0,
+                                        uint32_t& b1, uint32_t& b2, uint32_t& b3)
+{
+    const uint32_t a0 = st + tile_chunk_k8<C>(t0, ks) + 2 * tig;
+    const uint32_t a1 = st + tile_chunk_k8<C>(t0 + 8, ks) + 2 * tig;
+    b0 = i8x2_to_h2(lds_u16(a0));
+    b1 = i8x2_to_h2(lds_u16(a0 + 8));
+    b2 = i8x2_to_h2(lds_u16(a1));
+    b3 = i8x2_to_h2(lds_u16(a1 + 8));
+}
+
+// q times the channel scales of an int8 K pool (fp16 pair, round to nearest).
+__device__ __forceinline__ uint32_t scale_h2(uint32_t h2, float2 sc)
+{
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+    return pack_half2(f.x * sc.x, f.y * sc.y);
 }
 
 // One TMA copy of the tile whose first row is `y` in the pool's row space.
@@ -412,7 +483,7 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
                 if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, KV_DEV_BAD_BLOCK);
                 const bool firstst = (d.flags & F_FIRST) != 0;
                 const uint32_t qbytes = (uint32_t)(p.G * C::D * 2);  // query bytes per window row
-                uint32_t bytes = (uint32_t)__popc(lmask) * (uint32_t)(2 * C::BS * C::D * 2);
+                uint32_t bytes = (uint32_t)__popc(lmask) * (uint32_t)(C::K_TILE_BYTES + C::TILE_BYTES);
                 if (firstst) bytes += qbytes * (uint32_t)p.q_len;
                 const uint32_t full = full0 + stage * 8;
                 if (lane == 0) {
@@ -430,15 +501,18 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
                 const uint32_t st = sbase + stage * C::STAGE_BYTES;
                 if (load) {
                     const int32_t y = (id * p.Hkv + d.kvh) * C::BS;
-                    const uint32_t off = (uint32_t)(lane * C::TILE_BYTES);
-                    tma_load_tile<C::NH>(st + off, tmK, y, full, pol);
-                    tma_load_tile<C::NH>(st + C::KV_BYTES + off, tmV, y, full, pol);
+                    if constexpr (C::KQ)
+                        tma_load_2d(st + (uint32_t)(lane * C::K_TILE_BYTES), tmK, 0, y, full, pol);
+                    else
+                        tma_load_tile<C::NH>(st + (uint32_t)(lane * C::TILE_BYTES), tmK, y, full, pol);
+                    tma_load_tile<C::NH>(st + C::V_OFF + (uint32_t)(lane * C::TILE_BYTES), tmV, y, full,
+                                         pol);
                 }
                 if (firstst && lane < p.rows) {  // row R = j*G + g of the segment's queries
                     const int j = lane / p.G, g = lane % p.G;
                     const __half* src =
                         p.q + (((int64_t)d.s * p.q_len + j) * p.Hq + (int64_t)d.kvh * p.G + g) * C::D;
-                    bulk_load(st + 2 * C::KV_BYTES + lane * C::QROW, src, C::D * 2, full);
+                    bulk_load(st + C::Q_OFF + lane * C::QROW, src, C::D * 2, full);
                 }
                 ++k_issued;
             }
@@ -599,13 +673,27 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
         if (md.flags & F_FIRST) {
             // A fragments of this warp's 16 query rows: matrices (rows 0-7 | 8-15)
             // x (columns 16ks.. | 16ks+8..), one padded row address per lane
-            const uint32_t qrow = st + 2 * C::KV_BYTES +
+            const uint32_t qrow = st + C::Q_OFF +
                                   (mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * C::QROW;
             const int r0 = mt * 16 + gid;
 #pragma unroll
             for (int ks = 0; ks < C::D / 16; ++ks)
                 ldsm_x4(qrow + ((2 * ks + (lane >> 4)) << 4), qa[ks][0], qa[ks][1], qa[ks][2],
                         qa[ks][3]);
+            if constexpr (C::KQ) {
+                // fold the channel scales of the int8 keys into q: (a0, a1) hold
+                // dims 16ks + 2tig, +1; (a2, a3) dims 16ks + 8 + 2tig, +1
+                const float* sc = p.k_scale + (int64_t)md.kvh * C::D + 2 * tig;
+#pragma unroll
+                for (int ks = 0; ks < C::D / 16; ++ks) {
+                    const float2 s_lo = *reinterpret_cast<const float2*>(sc + 16 * ks);
+                    const float2 s_hi = *reinterpret_cast<const float2*>(sc + 16 * ks + 8);
+                    qa[ks][0] = scale_h2(qa[ks][0], s_lo);
+                    qa[ks][1] = scale_h2(qa[ks][1], s_lo);
+                    qa[ks][2] = scale_h2(qa[ks][2], s_hi);
+                    qa[ks][3] = scale_h2(qa[ks][3], s_hi);
+                }
+            }
 #pragma unroll
             for (int n = 0; n < C::D / 8; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.f;
             m[0] = m[1] = kNegInf;
@@ -625,7 +713,10 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
 #pragma unroll
             for (int ks = 0; ks < C::D / 16; ++ks) {
                 uint32_t b0, b1, b2, b3;
-                ldsm_x4(st + tile_chunk<C>(k_tok, 2 * ks + k_sel), b0, b1, b2, b3);
+                if constexpr (C::KQ)
+                    k8_frag<C>(st, qw * 16 + gid, ks, tig, b0, b1, b2, b3);
+                else
+                    ldsm_x4(st + tile_chunk<C>(k_tok, 2 * ks + k_sel), b0, b1, b2, b3);
                 if (ks & 1) {
                     mma_16816(T[0], qa[ks], b0, b1);
                     mma_16816(T[1], qa[ks], b2, b3);
@@ -693,7 +784,7 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
 #pragma unroll
             for (int np = 0; np < C::D / 16; ++np) {
                 const uint32_t addr =
-                    v_ok ? st + C::KV_BYTES + tile_chunk<C>(v_tok, 2 * np + v_sel) : zero_row;
+                    v_ok ? st + C::V_OFF + tile_chunk<C>(v_tok, 2 * np + v_sel) : zero_row;
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4_trans(addr, b0, b1, b2, b3);
                 mma_16816(O[2 * np], pa, b0, b1);
@@ -786,16 +877,20 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
     const float sl2 = p.scale_log2;
 
     const int c = lane & 7, grp = lane >> 3;
-    uint32_t koff[4][NH];  // chunk c of each unit of tokens grp + 4i
+    // chunk c of each unit of tokens grp + 4i; int8 keys: one 128-byte unit
+    // per token, chunk c = dims 16c .. 16c+15
+    uint32_t koff[4][NH];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int h = 0; h < NH; ++h) koff[i][h] = tile_chunk<C>(qw * 16 + grp + 4 * i, h * 8 + c);
+        for (int h = 0; h < NH; ++h)
+            koff[i][h] = C::KQ ? tile_chunk_k8<C>(qw * 16 + grp + 4 * i, c)
+                               : tile_chunk<C>(qw * 16 + grp + 4 * i, h * 8 + c);
     const int v_col = lane * DPT;
     const int v_cg = v_col / 8;          // chunk holding my output columns
     const int v_byte = (v_col % 8) * 2;  // byte offset inside that chunk
 
-    uint32_t qh[NH][4];  // q columns h*64 + c*8 .. +8 as fp16 pairs
+    uint32_t qh[NH][4];  // q columns h*64 + c*8 .. +8 (int8 keys: 16c + 8h ..) as fp16 pairs
     float o[DPT];
     float m = kNegInf, l = 0.f;
 
@@ -812,11 +907,18 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
         if (md.flags & F_FIRST) {
 #pragma unroll
             for (int h = 0; h < NH; ++h) {
-                const uint4 v = *reinterpret_cast<const uint4*>(st + 2 * C::KV_BYTES + (h * 64 + c * 8) * 2);
+                const int d0 = C::KQ ? 16 * c + 8 * h : h * 64 + c * 8;
+                const uint4 v = *reinterpret_cast<const uint4*>(st + C::Q_OFF + d0 * 2);
                 qh[h][0] = v.x;
                 qh[h][1] = v.y;
                 qh[h][2] = v.z;
                 qh[h][3] = v.w;
+                if constexpr (C::KQ) {  // fold the channel scales of the int8 keys into q
+                    const float* sc = p.k_scale + (int64_t)md.kvh * C::D + d0;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        qh[h][e] = scale_h2(qh[h][e], *reinterpret_cast<const float2*>(sc + 2 * e));
+                }
             }
 #pragma unroll
             for (int i = 0; i < DPT; ++i) o[i] = 0.f;
@@ -830,14 +932,30 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 float a0 = 0.f, a1 = 0.f;
+                if constexpr (C::KQ) {
+                    // 16 codes: dims 16c .. 16c+15 <-> qh[0] (first 8), qh[1]
+                    const uint4 kv = *reinterpret_cast<const uint4*>(st + koff[i][0]);
+                    const uint32_t kw8[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-                for (int h = 0; h < NH; ++h) {
-                    const uint4 kv = *reinterpret_cast<const uint4*>(st + koff[i][h]);
-                    const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+                    for (int w = 0; w < 4; ++w) {
+                        uint32_t lo, hi;
+                        i8x4_to_h2x2(kw8[w], lo, hi);
+                        const uint32_t qa_ = qh[w >> 1][(w & 1) * 2], qb_ = qh[w >> 1][(w & 1) * 2 + 1];
+                        a0 = fma_h((uint16_t)(qa_ & 0xffff), (uint16_t)(lo & 0xffff), a0);
+                        a1 = fma_h((uint16_t)(qa_ >> 16), (uint16_t)(lo >> 16), a1);
+                        a0 = fma_h((uint16_t)(qb_ & 0xffff), (uint16_t)(hi & 0xffff), a0);
+                        a1 = fma_h((uint16_t)(qb_ >> 16), (uint16_t)(hi >> 16), a1);
+                    }
+                } else {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        a0 = fma_h((uint16_t)(qh[h][e] & 0xffff), (uint16_t)(kw[e] & 0xffff), a0);
-                        a1 = fma_h((uint16_t)(qh[h][e] >> 16), (uint16_t)(kw[e] >> 16), a1);
+                    for (int h = 0; h < NH; ++h) {
+                        const uint4 kv = *reinterpret_cast<const uint4*>(st + koff[i][h]);
+                        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            a0 = fma_h((uint16_t)(qh[h][e] & 0xffff), (uint16_t)(kw[e] & 0xffff), a0);
+                            a1 = fma_h((uint16_t)(qh[h][e] >> 16), (uint16_t)(kw[e] >> 16), a1);
+                        }
                     }
                 }
                 acc[i] = a0 + a1;
@@ -877,7 +995,7 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
             const uint4 pw0 = reinterpret_cast<const uint4*>(pbuf)[0];
             const uint4 pw1 = reinterpret_cast<const uint4*>(pbuf)[1];
             const uint32_t pw[8] = {pw0.x, pw0.y, pw0.z, pw0.w, pw1.x, pw1.y, pw1.z, pw1.w};
-            const uint8_t* vb = st + C::KV_BYTES + v_byte;
+            const uint8_t* vb = st + C::V_OFF + v_byte;
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
                 if (t < nv) {
@@ -977,9 +1095,23 @@ __device__ void consumer_mma_mt(const Params& p, uint8_t* smem, volatile int* ab
         const uint32_t st = sbase + stage * C::STAGE_BYTES;
         if (md.flags & F_FIRST) {
             // copy the segment's query rows out of the stage (it will be reused)
-            const uint4* src = reinterpret_cast<const uint4*>(smem + stage * C::STAGE_BYTES + 2 * C::KV_BYTES);
+            const uint4* src = reinterpret_cast<const uint4*>(smem + stage * C::STAGE_BYTES + C::Q_OFF);
             uint4* dst = reinterpret_cast<uint4*>(smem + C::QP_OFF);
-            for (int i = threadIdx.x; i < C::RP * C::QROW / 16; i += C::NCW * 32) dst[i] = src[i];
+            for (int i = threadIdx.x; i < C::RP * C::QROW / 16; i += C::NCW * 32) {
+                uint4 v = src[i];
+                if constexpr (C::KQ) {
+                    // fold the channel scales of the int8 keys into q
+                    const int col = i % (C::QROW / 16);  // 8 dims per 16-byte chunk
+                    if (col < C::D / 8) {
+                        const float* sc = p.k_scale + (int64_t)md.kvh * C::D + col * 8;
+                        v.x = scale_h2(v.x, *reinterpret_cast<const float2*>(sc));
+                        v.y = scale_h2(v.y, *reinterpret_cast<const float2*>(sc + 2));
+                        v.z = scale_h2(v.z, *reinterpret_cast<const float2*>(sc + 4));
+                        v.w = scale_h2(v.w, *reinterpret_cast<const float2*>(sc + 6));
+                    }
+                }
+                dst[i] = v;
+            }
             named_bar_sync(2, C::NCW * 32);
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
@@ -1004,7 +1136,10 @@ __device__ void consumer_mma_mt(const Params& p, uint8_t* smem, volatile int* ab
 #pragma unroll
             for (int ks = 0; ks < C::D / 16; ++ks) {
                 uint32_t b0, b1, b2, b3;
-                ldsm_x4(st + tile_chunk<C>(k_tok, 2 * ks + k_sel), b0, b1, b2, b3);
+                if constexpr (C::KQ)
+                    k8_frag<C>(st, qw * 16 + gid, ks, tig, b0, b1, b2, b3);
+                else
+                    ldsm_x4(st + tile_chunk<C>(k_tok, 2 * ks + k_sel), b0, b1, b2, b3);
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
                     uint32_t a[4];
@@ -1074,7 +1209,7 @@ __device__ void consumer_mma_mt(const Params& p, uint8_t* smem, volatile int* ab
 #pragma unroll
             for (int np = 0; np < C::D / 16; ++np) {
                 const uint32_t addr =
-                    v_ok ? st + C::KV_BYTES + tile_chunk<C>(v_tok, 2 * np + v_sel) : zero_row;
+                    v_ok ? st + C::V_OFF + tile_chunk<C>(v_tok, 2 * np + v_sel) : zero_row;
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4_trans(addr, b0, b1, b2, b3);
 #pragma unroll
@@ -1167,7 +1302,7 @@ __global__ void __maxnreg__(C::MAXREG)
     if constexpr (!C::FMA) {
         const int used = p.rows * C::QROW;
         for (int st = 0; st < C::STAGES; ++st) {
-            uint8_t* qa = smem + st * C::STAGE_BYTES + 2 * C::KV_BYTES;
+            uint8_t* qa = smem + st * C::STAGE_BYTES + C::Q_OFF;
             for (int i = used + threadIdx.x * 16; i < C::RP * C::QROW; i += C::THREADS * 16)
                 *reinterpret_cast<uint4*>(qa + i) = make_uint4(0, 0, 0, 0);
         }
@@ -1254,7 +1389,7 @@ std::mutex g_mu;
 struct TmapEntry {
     const void* ptr;
     uint64_t rows;
-    int D, BS, dev;
+    int D, BS, dev, int8;
     CUtensorMap map;
 };
 constexpr int kTmapCache = 32;
@@ -1276,18 +1411,38 @@ int get_encoder()
 // Tensor map of a pool viewed as [num_blocks*Hkv*BS rows][D] fp16 whose box
 // is one (block, kv-head) tile, 128-byte swizzle.  Cached by (pointer, shape,
 // device).
-int pool_tmap(const void* pool, uint64_t rows, int D, int BS, CUtensorMap* out)
+int pool_tmap(const void* pool, uint64_t rows, int D, int BS, CUtensorMap* out, int int8 = 0)
 {
     int dev = 0;
     cudaGetDevice(&dev);
     std::lock_guard<std::mutex> lock(g_mu);
     for (auto& e : g_tmaps)
-        if (e.ptr == pool && e.rows == rows && e.D == D && e.BS == BS && e.dev == dev) {
+        if (e.ptr == pool && e.rows == rows && e.D == D && e.BS == BS && e.dev == dev &&
+            e.int8 == int8) {
             *out = e.map;
             return KV_OK;
         }
     int rc = get_encoder();
     if (rc != KV_OK) return rc;
+    if (int8) {
+        // int8 code pool as [rows][128]: a box of BS rows is one (block,
+        // kv-head) tile of 128-byte rows, 128-byte swizzle
+        CUtensorMap m;
+        const cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+        const cuuint64_t gstride[1] = {(cuuint64_t)D};
+        const cuuint32_t box[2] = {(cuuint32_t)D, (cuuint32_t)BS};
+        const cuuint32_t estride[2] = {1, 1};
+        CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(pool), gdim,
+                              gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return kv_fail(KV_ERR_CUDA, "cuTensorMapEncodeTiled failed (int8 K)");
+        TmapEntry& e = g_tmaps[g_tmap_next];
+        g_tmap_next = (g_tmap_next + 1) % kTmapCache;
+        e = {pool, rows, D, BS, dev, int8, m};
+        *out = m;
+        return KV_OK;
+    }
     // The pool as [rows][D/64][64] fp16: a box of BS rows is one whole
     // contiguous (block, kv-head) tile, written with the 128-byte swizzle.
     CUtensorMap m;
@@ -1304,7 +1459,7 @@ int pool_tmap(const void* pool, uint64_t rows, int D, int BS, CUtensorMap* out)
     if (r != CUDA_SUCCESS) return kv_fail(KV_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     TmapEntry& e = g_tmaps[g_tmap_next];
     g_tmap_next = (g_tmap_next + 1) % kTmapCache;
-    e = {pool, rows, D, BS, dev, m};
+    e = {pool, rows, D, BS, dev, 0, m};
     *out = m;
     return KV_OK;
 }
@@ -1365,13 +1520,13 @@ int launch(const CUtensorMap& tk, const CUtensorMap& tv, const Params& prm, int 
                          "lse_merge_kernel launch");
 }
 
-template <int D, int BS>
+template <int D, int BS, bool KQ = false>
 int dispatch_rows(int rows, const CUtensorMap& tk, const CUtensorMap& tv, const Params& prm,
                   int grid, bool pdl, cudaStream_t st)
 {
-    if (rows == 1) return launch<Cfg<D, BS, 1, true>>(tk, tv, prm, grid, pdl, st);
-    if (rows <= 16) return launch<Cfg<D, BS, 1, false>>(tk, tv, prm, grid, pdl, st);
-    return launch<Cfg<D, BS, 2, false>>(tk, tv, prm, grid, pdl, st);
+    if (rows == 1) return launch<Cfg<D, BS, 1, true, KQ>>(tk, tv, prm, grid, pdl, st);
+    if (rows <= 16) return launch<Cfg<D, BS, 1, false, KQ>>(tk, tv, prm, grid, pdl, st);
+    return launch<Cfg<D, BS, 2, false, KQ>>(tk, tv, prm, grid, pdl, st);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -1381,12 +1536,16 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
                    const int32_t* context_lens, int32_t q_len, float scale, void* out, int32_t B,
                    int32_t Hq, int32_t Hkv, int32_t D, int32_t BS, int32_t num_blocks,
                    void* workspace, size_t ws_bytes, const paged_attention_opts* opts,
-                   void* stream)
+                   void* stream, const float* k_scale = nullptr)
 {
     if (B < 0 || q_len < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || num_blocks < 1 ||
         max_blocks_per_seq < 1)
         return kv_fail(KV_ERR_INVALID, "paged attention: bad sizes");
     if (D != 64 && D != 128) return kv_fail(KV_ERR_INVALID, "paged attention: head_dim must be 64 or 128");
+    if (k_scale && D != 128)
+        return kv_fail(KV_ERR_INVALID, "paged attention: int8 K pools need head_dim 128");
+    if (k_scale && (reinterpret_cast<uintptr_t>(k_scale) & 7u))
+        return kv_fail(KV_ERR_INVALID, "paged attention: k_scales must be 8-byte aligned");
     if (BS != 8 && BS != 16) return kv_fail(KV_ERR_INVALID, "paged attention: block_size must be 8 or 16");
     const int G = Hq / Hkv;
     const int rows = G * q_len;
@@ -1411,7 +1570,7 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
 
     CUtensorMap tk, tv;
     const uint64_t prow = (uint64_t)num_blocks * Hkv * BS;
-    int rc = pool_tmap(k_pool, prow, D, BS, &tk);
+    int rc = pool_tmap(k_pool, prow, D, BS, &tk, k_scale ? 1 : 0);
     if (rc != KV_OK) return rc;
     rc = pool_tmap(v_pool, prow, D, BS, &tv);
     if (rc != KV_OK) return rc;
@@ -1428,6 +1587,7 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
     off += ((size_t)grid * 2 * rp * 4 + 15) / 16 * 16;
     prm.part_o = reinterpret_cast<float*>(ws + off);
     prm.err = err;
+    prm.k_scale = k_scale;
     prm.max_blocks = max_blocks_per_seq;
     prm.B = B;
     prm.q_len = q_len;
@@ -1442,6 +1602,9 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
     prm.scale_log2 = scale * 1.4426950408889634f;
     const bool pdl = !(opts && opts->use_pdl < 0);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (k_scale)
+        return BS == 8 ? dispatch_rows<128, 8, true>(rows, tk, tv, prm, grid, pdl, st)
+                       : dispatch_rows<128, 16, true>(rows, tk, tv, prm, grid, pdl, st);
     if (D == 64) {
         return BS == 8 ? dispatch_rows<64, 8>(rows, tk, tv, prm, grid, pdl, st)
                        : dispatch_rows<64, 16>(rows, tk, tv, prm, grid, pdl, st);
@@ -1490,6 +1653,18 @@ int paged_verify_attention(const void* q, const void* k_pool, const void* v_pool
     return attention_impl(q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens, q_len,
                           scale, out, B, Hq, Hkv, head_dim, block_size, num_blocks, workspace,
                           workspace_bytes, nullptr, stream);
+}
+
+int paged_attention_q8k(const void* q, const void* kq_pool, const float* k_scales,
+                        const void* v_pool, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                        const int32_t* context_lens, int32_t q_len, float scale, void* out,
+                        int32_t B, int32_t Hq, int32_t Hkv, int32_t head_dim, int32_t block_size,
+                        int32_t num_blocks, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (!k_scales) return kv_fail(KV_ERR_INVALID, "paged_attention_q8k: null k_scales");
+    return attention_impl(q, kq_pool, v_pool, block_tables, max_blocks_per_seq, context_lens, q_len,
+                          scale, out, B, Hq, Hkv, head_dim, block_size, num_blocks, workspace,
+                          workspace_bytes, nullptr, stream, k_scales);
 }
 
 int paged_attention_ex(const void* q, const void* k_pool, const void* v_pool,
