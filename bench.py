@@ -66,14 +66,53 @@ def rank_seed(base_seed: int, rank: int) -> int:
     return base_seed + 7919 * rank
 
 
-def algorithmic_bytes(lens, Hq, Hkv, D, bs, q_len):
+def algorithmic_bytes(lens, Hq, Hkv, D, bs, q_len, k_bytes=2):
     """(K/V bytes read, all bytes) of one attention launch: K and V rows of
-    every visible token, q and out, the used table entries and the lengths."""
+    every visible token, q and out, the used table entries and the lengths
+    (k_bytes = 1: int8 K codes, plus the fp32 channel scales)."""
     L = [int(x) for x in lens]
-    kv = sum(L) * Hkv * D * 2 * 2
+    kv = sum(L) * Hkv * D * (k_bytes + 2)
     qo = len(L) * q_len * Hq * D * 2 * 2
     tab = sum(-(-x // bs) for x in L) * 4 + len(L) * 4
-    return kv, kv + qo + tab
+    scales = Hkv * D * 4 if k_bytes == 1 else 0
+    return kv, kv + qo + tab + scales
+
+
+def split_workload(name):
+    """'<config>' or '<config>_q8k' (the same config with an int8 K pool)."""
+    return (name[:-4], True) if name.endswith("_q8k") else (name, False)
+
+
+def pool_tokens(pool):
+    """[num_blocks][Hkv][bs][D] -> [num_blocks*bs][Hkv][D] in slot order (a copy)."""
+    nb, Hkv, bs, D = pool.shape
+    return pool.permute(0, 2, 1, 3).reshape(nb * bs, Hkv, D).contiguous()
+
+
+def quantise_pool_device(pkv, wl):
+    """int8 K pool of the workload through the library: channel scales from
+    every pool token, then the quantising append of every slot."""
+    import torch
+    nb, Hkv, bs, D = wl.k_pool.shape
+    kt, vt = pool_tokens(wl.k_pool), pool_tokens(wl.v_pool)
+    sc = pkv.paged_kv_k_scales(kt)
+    kq = torch.empty((nb, Hkv, bs, D), dtype=torch.int8, device=wl.k_pool.device)
+    slots = torch.arange(nb * bs, dtype=torch.int64, device=wl.k_pool.device)
+    pkv.paged_kv_append_q8k(kt, vt, slots, sc, kq, wl.v_pool)
+    del kt, vt
+    return kq, sc
+
+
+def quantise_pool_host(K):
+    """The same with the oracle on host arrays: (codes, scales)."""
+    import numpy as np
+    import oracle
+    n, Hkv, bs, D = K.shape
+    toks = K.transpose(0, 2, 1, 3).reshape(n * bs, Hkv, D).copy()
+    sc = oracle.k_scales(toks)
+    K8, _ = oracle.append_q8k(np.zeros(K.shape, np.int8), np.zeros_like(K), toks, toks,
+                              np.arange(n * bs, dtype=np.int64), sc)
+    return K8, sc
 
 
 def prefill_flops(lens, Hq, D, q_len):
@@ -363,13 +402,18 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
 
     from workloads.synth import CONFIGS
-    spec = CONFIGS[args.workload]
+    base, q8k = split_workload(args.workload)
+    spec = CONFIGS[base]
     seed = rank_seed(spec.seed, rank)
-    wl = make_workload(args.workload, device, seed=seed, B=args.batch or None)
+    wl = make_workload(base, device, seed=seed, B=args.batch or None)
     q_len = spec.q_len
     Hq, Hkv, D, bs = spec.Hq, spec.Hkv, spec.D, spec.bs
+    k_bytes = 1 if q8k else 2
     n_distinct = min(args.warmup + args.steps, 64)
     steps = build_steps(pkv, wl, n_distinct, device, seed)
+    kq = ksc = None
+    if q8k:
+        kq, ksc = quantise_pool_device(pkv, wl)
     out = torch.empty((wl.B, q_len, Hq, D), dtype=torch.float16, device=device)
     ws = torch.empty(pkv.workspace_size(Hq, Hkv, q_len, D), dtype=torch.uint8, device=device)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
@@ -378,17 +422,8 @@ def run_ours(args):
 
     def step(i, ev=None):
         st = steps[i % n_distinct]
-        if st["pairs"] is not None:
-            pkv.paged_kv_copy_blocks(wl.k_pool, wl.v_pool, st["pairs"])
-        pkv.paged_kv_append(st["k_new"], st["v_new"], st["slots"], wl.k_pool, wl.v_pool)
-        if ev is not None:
-            ev.record(stream)
-        if q_len == 1:
-            pkv.paged_decode_attention(st["q"], wl.k_pool, wl.v_pool, st["tables"], st["lens"],
-                                       wl.scale, out=out, workspace=ws)
-        else:
-            pkv.paged_verify_attention(st["q"], wl.k_pool, wl.v_pool, st["tables"], st["lens"],
-                                       wl.scale, q_len, out=out, workspace=ws)
+        decode_step(pkv, wl, st["q"], st["k_new"], st["v_new"], st["slots"], st["tables"],
+                    st["lens"], st["pairs"], out, ws, q_len, kq, ksc, ev, stream)
 
     for i in range(args.warmup):
         step(i)
@@ -414,7 +449,7 @@ def run_ours(args):
             step(i, ev_a[k])
             ev_e[k].record(stream)
             launches += 3 + (1 if st["pairs"] is not None else 0)
-            kvb, allb = algorithmic_bytes(st["lens_host"], Hq, Hkv, D, bs, q_len)
+            kvb, allb = algorithmic_bytes(st["lens_host"], Hq, Hkv, D, bs, q_len, k_bytes)
             kv_bytes_total += kvb
             alg_attn.append(allb)
             th_tokens += int(st["lens_host"].sum()) * Hq * q_len
@@ -434,7 +469,7 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(pkv, wl, steps, n_distinct, args, out, ws, flush, stream, device, Hq, Hkv, D,
-                      bs, q_len, world)
+                      bs, q_len, world, kq, ksc)
 
     peak, peak_kind = measured_hbm_peak()
     attn_avg_ms = statistics.mean(attn_ms)
@@ -452,6 +487,8 @@ def run_ours(args):
                 "Hq": Hq, "Hkv": Hkv, "head_dim": D, "block_size": bs, "q_len": q_len,
                 "mean_context": float(np.mean(wl.lens)),
                 "step": "copy-on-write copies + append 1 token/sequence + paged attention + merge",
+                "k_pool": ("int8 codes, fp32 scale per (KV head, channel); V fp16" if q8k
+                           else "fp16"),
                 "l2": "flushed before every timed step (memset of 2x L2)",
                 "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "hbm_frac": round(value / peak, 4),
@@ -470,14 +507,39 @@ def run_ours(args):
         if world == 1 and args.cpu_seconds > 0:
             # the timed appends only wrote slots past each sequence's original
             # length, so the workload's original tokens are still in the pools
-            result["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+            result["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, q8k)
     if world > 1:
         dist.destroy_process_group()
     return result
 
 
+def decode_step(pkv, wl, q, k_new, v_new, slots, tables, lens, pairs, out, ws, q_len, kq, ksc,
+                ev=None, stream=None):
+    """One decode step through the public API: copy-on-write copies, append
+    of the new tokens, attention (int8 K pool when kq is given)."""
+    if kq is None:
+        if pairs is not None:
+            pkv.paged_kv_copy_blocks(wl.k_pool, wl.v_pool, pairs)
+        pkv.paged_kv_append(k_new, v_new, slots, wl.k_pool, wl.v_pool)
+    else:
+        if pairs is not None:
+            pkv.paged_kv_copy_blocks_q8k(kq, wl.v_pool, pairs)
+        pkv.paged_kv_append_q8k(k_new, v_new, slots, ksc, kq, wl.v_pool)
+    if ev is not None:
+        ev.record(stream)
+    if kq is not None:
+        pkv.paged_attention_q8k(q, kq, ksc, wl.v_pool, tables, lens, wl.scale, q_len, out=out,
+                                workspace=ws)
+    elif q_len == 1:
+        pkv.paged_decode_attention(q, wl.k_pool, wl.v_pool, tables, lens, wl.scale, out=out,
+                                   workspace=ws)
+    else:
+        pkv.paged_verify_attention(q, wl.k_pool, wl.v_pool, tables, lens, wl.scale, q_len, out=out,
+                                   workspace=ws)
+
+
 def run_e2e(pkv, wl, steps, n_distinct, args, out, ws, flush, stream, device, Hq, Hkv, D, bs, q_len,
-            world):
+            world, kq=None, ksc=None):
     import torch
     import torch.distributed as dist
     host = []
@@ -504,24 +566,19 @@ def run_e2e(pkv, wl, steps, n_distinct, args, out, ws, flush, stream, device, Hq
             nbytes += h[name].numel() * h[name].element_size()
         tables.copy_(h["tables"], non_blocking=True)
         nbytes += h["tables"].numel() * 4
+        pairs = None
         if h["pairs"] is not None:
             pairs = h["pairs"].to(device, non_blocking=True)
             nbytes += h["pairs"].numel() * 4
-            pkv.paged_kv_copy_blocks(wl.k_pool, wl.v_pool, pairs)
-        pkv.paged_kv_append(dev["k_new"], dev["v_new"], dev["slots"], wl.k_pool, wl.v_pool)
-        if q_len == 1:
-            pkv.paged_decode_attention(dev["q"], wl.k_pool, wl.v_pool, tables, dev["lens"],
-                                       wl.scale, out=out, workspace=ws)
-        else:
-            pkv.paged_verify_attention(dev["q"], wl.k_pool, wl.v_pool, tables, dev["lens"],
-                                       wl.scale, q_len, out=out, workspace=ws)
+        decode_step(pkv, wl, dev["q"], dev["k_new"], dev["v_new"], dev["slots"], tables,
+                    dev["lens"], pairs, out, ws, q_len, kq, ksc)
         out_host.copy_(out, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
         if k >= args.warmup:
             times.append(e0.elapsed_time(e1))
             kvb_total += algorithmic_bytes(steps[k % n_distinct]["lens_host"], Hq, Hkv, D, bs,
-                                           q_len)[0]
+                                           q_len, 1 if kq is not None else 2)[0]
             h2d = nbytes
     t = torch.tensor([sum(times)], dtype=torch.float64, device=device)
     kv = torch.tensor([float(kvb_total)], dtype=torch.float64, device=device)
@@ -542,6 +599,7 @@ def oracle_sample(workload, target_s, seed_offset=0):
     import oracle
     from workloads import make_workload
     from workloads.synth import CONFIGS
+    workload, _ = split_workload(workload)
     spec = CONFIGS[workload]
     probe = make_workload(workload, "cpu", B=1, seed=spec.seed + seed_offset)
     t0 = time.perf_counter()
@@ -552,11 +610,18 @@ def oracle_sample(workload, target_s, seed_offset=0):
     return make_workload(workload, "cpu", B=n, seed=spec.seed + seed_offset)
 
 
-def time_oracle(wl):
+def time_oracle(wl, k8=None):
+    """One oracle call over the workload (over int8 codes k8 = (codes, scales)
+    if given); seconds."""
     import oracle
     q, k, v = wl.q.numpy(), wl.k_pool.numpy(), wl.v_pool.numpy()
     t0 = time.perf_counter()
-    oracle.paged_attention(q, k, v, wl.block_tables, wl.lens, scale=wl.scale, q_len=wl.q.shape[1])
+    if k8 is None:
+        oracle.paged_attention(q, k, v, wl.block_tables, wl.lens, scale=wl.scale,
+                               q_len=wl.q.shape[1])
+    else:
+        oracle.paged_attention_q8k(q, k8[0], k8[1], v, wl.block_tables, wl.lens, scale=wl.scale,
+                                   q_len=wl.q.shape[1])
     return time.perf_counter() - t0
 
 
@@ -574,20 +639,28 @@ def host_copy(wl):
     return wl.q.cpu().numpy(), K, V, t2
 
 
-def cpu_baseline(wl, target_s):
+def cpu_baseline(wl, target_s, q8k=False):
     """The oracle, as it stands, over the whole workload of this run (its
-    sequences, blocks and queries copied to the host), repeated until about
-    target_s seconds of CPU time have been spent."""
+    sequences, blocks and queries copied to the host; int8 K codes made by
+    the oracle's own quantiser), repeated until about target_s seconds of CPU
+    time have been spent."""
     import oracle
     q, K, V, t2 = host_copy(wl)
     s = wl.spec
+    K8 = sc = None
+    if q8k:
+        K8, sc = quantise_pool_host(K)
     reps, spent = 0, 0.0
     while reps == 0 or spent < target_s:
         t0 = time.perf_counter()
-        oracle.paged_attention(q, K, V, t2, wl.lens, scale=wl.scale, q_len=q.shape[1])
+        if q8k:
+            oracle.paged_attention_q8k(q, K8, sc, V, t2, wl.lens, scale=wl.scale, q_len=q.shape[1])
+        else:
+            oracle.paged_attention(q, K, V, t2, wl.lens, scale=wl.scale, q_len=q.shape[1])
         spent += time.perf_counter() - t0
         reps += 1
-    kvb = algorithmic_bytes(wl.lens, q.shape[2], s.Hkv, q.shape[3], s.bs, q.shape[1])[0]
+    kvb = algorithmic_bytes(wl.lens, q.shape[2], s.Hkv, q.shape[3], s.bs, q.shape[1],
+                            1 if q8k else 2)[0]
     return {"value": round(kvb * reps / spent / 1e9, 4), "unit": "GB/s",
             "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"whole workload of this run ({wl.B} sequences, {int(wl.lens.sum())} "
@@ -600,13 +673,16 @@ def run_reference(args):
     if rank != 0:
         return None
     from workloads.synth import CONFIGS
-    spec = CONFIGS[args.workload]
+    base, q8k = split_workload(args.workload)
+    spec = CONFIGS[base]
     per_step = max(0.2, min(2.0, 120.0 / max(1, args.steps + args.warmup)))
     wl = oracle_sample(args.workload, per_step)
+    k8 = quantise_pool_host(wl.k_pool.numpy()) if q8k else None
     for _ in range(args.warmup):
-        time_oracle(wl)
-    times = [time_oracle(wl) for _ in range(args.steps)]
-    kvb = algorithmic_bytes(wl.lens, spec.Hq, spec.Hkv, spec.D, spec.bs, spec.q_len)[0]
+        time_oracle(wl, k8)
+    times = [time_oracle(wl, k8) for _ in range(args.steps)]
+    kvb = algorithmic_bytes(wl.lens, spec.Hq, spec.Hkv, spec.D, spec.bs, spec.q_len,
+                            1 if q8k else 2)[0]
     total = sum(times)
     value = kvb * args.steps / total / 1e9
     sample = (f"{wl.B} of {spec.B} sequences of {args.workload} per step (same length recipe), "
@@ -628,7 +704,7 @@ def main(argv=None):
     from workloads.synth import CONFIGS
     if args.impl == "reference":
         res = run_reference(args)
-    elif CONFIGS[args.workload].q_len > 32:
+    elif CONFIGS[split_workload(args.workload)[0]].q_len > 32:
         res = run_prefill(args)
     else:
         res = run_ours(args)

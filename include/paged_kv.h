@@ -206,6 +206,11 @@ int paged_kv_k_scales(const void* k, int64_t T, int32_t Hkv, int32_t head_dim, f
 int paged_kv_append_q8k(const void* k_new, const void* v_new, const int64_t* slot_mapping,
                         const float* k_scales, void* kq_pool, void* v_pool, int32_t T, int32_t Hkv,
                         int32_t head_dim, int32_t block_size, int32_t num_blocks, void* stream);
+/* paged_kv_copy_blocks_q8k: paged_kv_copy_blocks for an int8 K pool (K blocks
+ * of Hkv*bs*D bytes) and its fp16 V pool; head_dim a multiple of 16. */
+int paged_kv_copy_blocks_q8k(void* kq_pool, void* v_pool, const int32_t* pairs, int32_t n,
+                             int32_t Hkv, int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                             void* stream);
 /* paged_attention_q8k: paged_verify_attention (q_len = 1: decode) over an int8
  * K pool: scores use key t = code * k_scales[kvh][:].  The scales are folded
  * into q once per (sequence, kv head) segment (q_d * k_scales[d], rounded to

@@ -24,6 +24,7 @@ __all__ = ["KVPool", "KVError", "pool_bytes", "paged_kv_append", "paged_kv_copy_
            "workspace_size", "paged_decode_attention", "paged_verify_attention",
            "paged_attention", "paged_prefill_attention", "paged_kv_swap_out", "paged_kv_swap_in",
            "swap_staging_bytes", "paged_kv_k_scales", "paged_kv_append_q8k", "paged_attention_q8k",
+           "paged_kv_copy_blocks_q8k",
            "device_error", "lib"]
 
 _L = _abi.load()
@@ -343,6 +344,18 @@ def paged_kv_append_q8k(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: 
     check(_L.paged_kv_append_q8k(k_new.data_ptr(), v_new.data_ptr(), slot_mapping.data_ptr(),
                                  k_scales.data_ptr(), kq_pool.data_ptr(), v_pool.data_ptr(), T, Hkv,
                                  D, bs, nb, _stream(dev)), "paged_kv_append_q8k")
+
+
+def paged_kv_copy_blocks_q8k(kq_pool: torch.Tensor, v_pool: torch.Tensor, pairs: torch.Tensor) -> None:
+    """Copy-on-write block copies for an int8 K pool and its fp16 V pool."""
+    dev = v_pool.device
+    _need(kq_pool, "kq_pool", torch.int8, dev)
+    _need(v_pool, "v_pool", torch.float16, dev)
+    _need(pairs, "pairs", torch.int32, dev)
+    nb, Hkv, bs, D = kq_pool.shape
+    check(_L.paged_kv_copy_blocks_q8k(kq_pool.data_ptr(), v_pool.data_ptr(), pairs.data_ptr(),
+                                      pairs.numel() // 2, Hkv, D, bs, nb, _stream(dev)),
+          "paged_kv_copy_blocks_q8k")
 
 
 def paged_attention_q8k(q, kq_pool, k_scales, v_pool, block_tables, context_lens, scale, q_len=1,

@@ -74,6 +74,7 @@ SIGNATURES = {
     "paged_kv_swap_out": ([_P, _P, _P, _i32, _P, _P, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
     "paged_kv_swap_in": ([_P, _P, _P, _i32, _P, _P, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
     "paged_kv_k_scales": ([_P, ctypes.c_int64, _i32, _i32, _P, _P], ctypes.c_int),
+    "paged_kv_copy_blocks_q8k": ([_P, _P, _P, _i32, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
     "paged_kv_append_q8k": ([_P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
     "paged_attention_q8k": ([_P, _P, _P, _P, _P, _i32, _P, _i32, ctypes.c_float, _P, _i32, _i32, _i32,
                              _i32, _i32, _i32, _P, _sz, _P], ctypes.c_int),

@@ -54,7 +54,8 @@ __global__ void append_kernel(const uint4* __restrict__ k_new, const uint4* __re
 
 __global__ void copy_blocks_kernel(uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
                                    const int32_t* __restrict__ pairs, int32_t n,
-                                   int64_t chunks_per_block, int32_t num_blocks, int* err)
+                                   int64_t chunks_per_block, int32_t num_blocks, int* err,
+                                   int64_t k_chunks_per_block)
 {
     const int32_t pair = blockIdx.y;
     const int32_t src = __ldg(pairs + 2 * pair);
@@ -63,13 +64,14 @@ __global__ void copy_blocks_kernel(uint4* __restrict__ k_pool, uint4* __restrict
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(err, KV_DEV_BAD_BLOCK);
         return;
     }
-    const uint4* ks = k_pool + (int64_t)src * chunks_per_block;
+    // K blocks may be smaller than V blocks (int8 codes): k_chunks_per_block
+    const uint4* ks = k_pool + (int64_t)src * k_chunks_per_block;
     const uint4* vs = v_pool + (int64_t)src * chunks_per_block;
-    uint4* kd = k_pool + (int64_t)dst * chunks_per_block;
+    uint4* kd = k_pool + (int64_t)dst * k_chunks_per_block;
     uint4* vd = v_pool + (int64_t)dst * chunks_per_block;
     for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < chunks_per_block;
          c += (int64_t)gridDim.x * blockDim.x) {
-        kd[c] = ks[c];
+        if (c < k_chunks_per_block) kd[c] = ks[c];
         vd[c] = vs[c];
     }
 }
@@ -251,8 +253,10 @@ int paged_kv_append(const void* k_new, const void* v_new, const int64_t* slot_ma
     return kv_cuda_check(cudaGetLastError(), "paged_kv_append");
 }
 
-int paged_kv_copy_blocks(void* k_pool, void* v_pool, const int32_t* pairs, int32_t n, int32_t Hkv,
-                         int32_t head_dim, int32_t block_size, int32_t num_blocks, void* stream)
+
+static int copy_blocks_impl(void* k_pool, void* v_pool, const int32_t* pairs, int32_t n,
+                            int32_t Hkv, int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                            void* stream, bool k_int8)
 {
     if (n < 0 || Hkv <= 0 || head_dim <= 0 || head_dim % 8 != 0 || block_size <= 0 ||
         num_blocks <= 0 || n > 65535)
@@ -270,8 +274,25 @@ int paged_kv_copy_blocks(void* k_pool, void* v_pool, const int32_t* pairs, int32
     if (bx > 64) bx = 64;
     dim3 grid((unsigned)bx, (unsigned)n);
     copy_blocks_kernel<<<grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), pairs, n, cpb, num_blocks, err);
+        static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), pairs, n, cpb, num_blocks, err,
+        k_int8 ? cpb / 2 : cpb);
     return kv_cuda_check(cudaGetLastError(), "paged_kv_copy_blocks");
+}
+
+int paged_kv_copy_blocks(void* k_pool, void* v_pool, const int32_t* pairs, int32_t n, int32_t Hkv,
+                         int32_t head_dim, int32_t block_size, int32_t num_blocks, void* stream)
+{
+    return copy_blocks_impl(k_pool, v_pool, pairs, n, Hkv, head_dim, block_size, num_blocks, stream,
+                            false);
+}
+
+int paged_kv_copy_blocks_q8k(void* kq_pool, void* v_pool, const int32_t* pairs, int32_t n,
+                             int32_t Hkv, int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                             void* stream)
+{
+    if (head_dim % 16 != 0) return kv_fail(KV_ERR_INVALID, "paged_kv_copy_blocks_q8k: bad head_dim");
+    return copy_blocks_impl(kq_pool, v_pool, pairs, n, Hkv, head_dim, block_size, num_blocks, stream,
+                            true);
 }
 
 int paged_kv_append_q8k(const void* k_new, const void* v_new, const int64_t* slot_mapping,

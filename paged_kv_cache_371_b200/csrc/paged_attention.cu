@@ -172,60 +172,75 @@ __device__ __forceinline__ uint32_t tile_chunk_k8(int tok, int cg)
     return (uint32_t)((tok / C::BS) * C::K_TILE_BYTES + r * 128 + ((cg ^ (r & 7)) << 4));
 }
 
-// int8 codes -> exact fp16 integers: the byte x + 128 (x ^ 0x80) becomes the
-// low mantissa byte of an fp16 with exponent byte 0x64, i.e. 1024 + x + 128;
-// one half2 subtraction of 1152 leaves x.  Two codes (low 16 bits of w)
-// give one half2.
-__device__ __forceinline__ uint32_t i8x2_to_h2(uint32_t w)
-{
-    uint32_t r;
-    asm("prmt.b32 %0, %1, %2, 0x5140;" : "=r"(r) : "r"(w ^ 0x8080u), "r"(0x64646464u));
-    const __half2 v = __hsub2(*reinterpret_cast<const __half2*>(&r),
-                              __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480)));
-    return *reinterpret_cast<const uint32_t*>(&v);
-}
-
-// Four codes -> two half2 (bytes 0-1, bytes 2-3).
-__device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t& lo, uint32_t& hi)
-{
-    const uint32_t u = w ^ 0x80808080u;
-    uint32_t a, b;
-    asm("prmt.b32 %0, %1, %2, 0x5140;" : "=r"(a) : "r"(u), "r"(0x64646464u));
-    asm("prmt.b32 %0, %1, %2, 0x7362;" : "=r"(b) : "r"(u), "r"(0x64646464u));
-    const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
-    const __half2 va = __hsub2(*reinterpret_cast<const __half2*>(&a), bias);
-    const __half2 vb = __hsub2(*reinterpret_cast<const __half2*>(&b), bias);
-    lo = *reinterpret_cast<const uint32_t*>(&va);
-    hi = *reinterpret_cast<const uint32_t*>(&vb);
-}
-
-__device__ __forceinline__ uint32_t lds_u16(uint32_t addr)
-{
-    unsigned short v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-    return v;
-}
-
-// B fragments of k-step ks for the two n8 tiles (tokens t0 and t0 + 8) from an
-// int8 K stage: token t's codes of dims 16ks + 2tig, +1 (b0 / b2) and
-// 16ks + 8 + 2tig, +1 (b1 / b3), the m16n8k16 B layout.
-template <class C>
-__device__ __forceinline__ void k8_frag(uint32_t st, int t0, int ks, int tig, uint32_t& b0,
-                                        uint32_t& b1, uint32_t& b2, uint32_t& b3)
-{
-    const uint32_t a0 = st + tile_chunk_k8<C>(t0, ks) + 2 * tig;
-    const uint32_t a1 = st + tile_chunk_k8<C>(t0 + 8, ks) + 2 * tig;
-    b0 = i8x2_to_h2(lds_u16(a0));
-    b1 = i8x2_to_h2(lds_u16(a0 + 8));
-    b2 = i8x2_to_h2(lds_u16(a1));
-    b3 = i8x2_to_h2(lds_u16(a1 + 8));
-}
-
 // q times the channel scales of an int8 K pool (fp16 pair, round to nearest).
 __device__ __forceinline__ uint32_t scale_h2(uint32_t h2, float2 sc)
 {
     const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
     return pack_half2(f.x * sc.x, f.y * sc.y);
+}
+
+// int8 codes -> fp16: the byte x + 128 (x ^ 0x80) becomes the low mantissa
+// byte of an fp16 with exponent byte 0x64, whose value is 1024 + x + 128
+// exactly (1152 + x).
+
+// Biased form used on the hot path: four codes -> two half2 holding
+// 1152 + code exactly (no subtraction).  A dot product over biased keys
+// exceeds the true one by 1152 * (sum of the q entries), a per-row constant
+// subtracted once per score.
+__device__ __forceinline__ void i8x4_to_h2x2_biased(uint32_t w, uint32_t& lo, uint32_t& hi)
+{
+    const uint32_t u = w ^ 0x80808080u;
+    asm("prmt.b32 %0, %1, %2, 0x5140;" : "=r"(lo) : "r"(u), "r"(0x64646464u));
+    asm("prmt.b32 %0, %1, %2, 0x7362;" : "=r"(hi) : "r"(u), "r"(0x64646464u));
+}
+constexpr float kCodeBias = 1152.f;
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float h2_sum(uint32_t h2)
+{
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+    return f.x + f.y;
+}
+
+// B fragments of k-step ks for the two n8 tiles (tokens t0 and t0 + 8) from an
+// int8 K stage, biased.  The dims of each 16-dim chunk are taken in a
+// permuted order, so that one 32-bit word per token serves both registers:
+// lane tig's k positions (2tig, 2tig+1 | 2tig+8, 2tig+9) are dims
+// (4tig, 4tig+1 | 4tig+2, 4tig+3); the q fragments use the same order.
+template <class C>
+__device__ __forceinline__ void k8_frag(uint32_t st, int t0, int ks, int tig, uint32_t& b0,
+                                        uint32_t& b1, uint32_t& b2, uint32_t& b3)
+{
+    i8x4_to_h2x2_biased(lds_u32(st + tile_chunk_k8<C>(t0, ks) + 4 * tig), b0, b1);
+    i8x4_to_h2x2_biased(lds_u32(st + tile_chunk_k8<C>(t0 + 8, ks) + 4 * tig), b2, b3);
+}
+
+// q fragments (rows r and r + 8) of an int8-K segment in the permuted dim
+// order of k8_frag, times the channel scales; adds this lane's share of each
+// row's sum of the (rounded) fp16 entries to rsum.
+template <class C>
+__device__ __forceinline__ void q8_frags(const uint8_t* qrow_r, const uint8_t* qrow_r8,
+                                         const float* sc, int tig, uint32_t (&qa)[C::D / 16][4],
+                                         float (&rsum)[2])
+{
+#pragma unroll
+    for (int ks = 0; ks < C::D / 16; ++ks) {
+        const int d = 16 * ks + 4 * tig;
+        const float2 s01 = *reinterpret_cast<const float2*>(sc + d);
+        const float2 s23 = *reinterpret_cast<const float2*>(sc + d + 2);
+        qa[ks][0] = scale_h2(*reinterpret_cast<const uint32_t*>(qrow_r + d * 2), s01);
+        qa[ks][1] = scale_h2(*reinterpret_cast<const uint32_t*>(qrow_r8 + d * 2), s01);
+        qa[ks][2] = scale_h2(*reinterpret_cast<const uint32_t*>(qrow_r + d * 2 + 4), s23);
+        qa[ks][3] = scale_h2(*reinterpret_cast<const uint32_t*>(qrow_r8 + d * 2 + 4), s23);
+        rsum[0] += h2_sum(qa[ks][0]) + h2_sum(qa[ks][2]);
+        rsum[1] += h2_sum(qa[ks][1]) + h2_sum(qa[ks][3]);
+    }
 }
 
 // One TMA copy of the tile whose first row is `y` in the pool's row space.
@@ -658,6 +673,7 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
     float O[C::D / 8][4];
     uint32_t qa[C::D / 16][4];
     float m[2], l[2];
+    float corr[2] = {0.f, 0.f};  // int8 keys: bias * row sum of q
     int lim[2];
 
     int stage = 0;
@@ -676,22 +692,22 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
             const uint32_t qrow = st + C::Q_OFF +
                                   (mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * C::QROW;
             const int r0 = mt * 16 + gid;
+            if constexpr (!C::KQ) {
 #pragma unroll
-            for (int ks = 0; ks < C::D / 16; ++ks)
-                ldsm_x4(qrow + ((2 * ks + (lane >> 4)) << 4), qa[ks][0], qa[ks][1], qa[ks][2],
-                        qa[ks][3]);
-            if constexpr (C::KQ) {
-                // fold the channel scales of the int8 keys into q: (a0, a1) hold
-                // dims 16ks + 2tig, +1; (a2, a3) dims 16ks + 8 + 2tig, +1
-                const float* sc = p.k_scale + (int64_t)md.kvh * C::D + 2 * tig;
+                for (int ks = 0; ks < C::D / 16; ++ks)
+                    ldsm_x4(qrow + ((2 * ks + (lane >> 4)) << 4), qa[ks][0], qa[ks][1], qa[ks][2],
+                            qa[ks][3]);
+            } else {
+                // int8 keys: q fragments in the permuted dim order, times the
+                // channel scales; bias correction from the row sums
+                const uint8_t* qr = smem + stage * C::STAGE_BYTES + C::Q_OFF + (mt * 16 + gid) * C::QROW;
+                float rs[2] = {0.f, 0.f};
+                q8_frags<C>(qr, qr + 8 * C::QROW, p.k_scale + (int64_t)md.kvh * C::D, tig, qa, rs);
 #pragma unroll
-                for (int ks = 0; ks < C::D / 16; ++ks) {
-                    const float2 s_lo = *reinterpret_cast<const float2*>(sc + 16 * ks);
-                    const float2 s_hi = *reinterpret_cast<const float2*>(sc + 16 * ks + 8);
-                    qa[ks][0] = scale_h2(qa[ks][0], s_lo);
-                    qa[ks][1] = scale_h2(qa[ks][1], s_lo);
-                    qa[ks][2] = scale_h2(qa[ks][2], s_hi);
-                    qa[ks][3] = scale_h2(qa[ks][3], s_hi);
+                for (int rr = 0; rr < 2; ++rr) {
+                    rs[rr] += __shfl_xor_sync(0xffffffffu, rs[rr], 1);
+                    rs[rr] += __shfl_xor_sync(0xffffffffu, rs[rr], 2);
+                    corr[rr] = kCodeBias * rs[rr];
                 }
             }
 #pragma unroll
@@ -728,7 +744,7 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) S[nt][c] += T[nt][c];
+                for (int c = 0; c < 4; ++c) S[nt][c] += T[nt][c] - (C::KQ ? corr[c >> 1] : 0.f);
             // a token counts if its row may see it and this stage loaded it
             // (with 8-token blocks a warp's second block can lie past the run)
             const int pos0 = md.t0 + qw * 16 + tig * 2;
@@ -891,6 +907,7 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
     const int v_byte = (v_col % 8) * 2;  // byte offset inside that chunk
 
     uint32_t qh[NH][4];  // q columns h*64 + c*8 .. +8 (int8 keys: 16c + 8h ..) as fp16 pairs
+    float corr = 0.f;    // int8 keys: bias * sum of this lane's q entries
     float o[DPT];
     float m = kNegInf, l = 0.f;
 
@@ -920,6 +937,14 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
                         qh[h][e] = scale_h2(qh[h][e], *reinterpret_cast<const float2*>(sc + 2 * e));
                 }
             }
+            if constexpr (C::KQ) {  // bias correction of this lane's 16 dims
+                float qs = 0.f;
+#pragma unroll
+                for (int h = 0; h < NH; ++h)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) qs += h2_sum(qh[h][e]);
+                corr = kCodeBias * qs;
+            }
 #pragma unroll
             for (int i = 0; i < DPT; ++i) o[i] = 0.f;
             m = kNegInf;
@@ -939,7 +964,7 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
 #pragma unroll
                     for (int w = 0; w < 4; ++w) {
                         uint32_t lo, hi;
-                        i8x4_to_h2x2(kw8[w], lo, hi);
+                        i8x4_to_h2x2_biased(kw8[w], lo, hi);
                         const uint32_t qa_ = qh[w >> 1][(w & 1) * 2], qb_ = qh[w >> 1][(w & 1) * 2 + 1];
                         a0 = fma_h((uint16_t)(qa_ & 0xffff), (uint16_t)(lo & 0xffff), a0);
                         a1 = fma_h((uint16_t)(qa_ >> 16), (uint16_t)(lo >> 16), a1);
@@ -958,7 +983,7 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
                         }
                     }
                 }
-                acc[i] = a0 + a1;
+                acc[i] = C::KQ ? (a0 + a1) - corr : a0 + a1;
             }
 #pragma unroll
             for (int off = 1; off < 8; off <<= 1)
@@ -1081,6 +1106,7 @@ __device__ void consumer_mma_mt(const Params& p, uint8_t* smem, volatile int* ab
 
     float O[MT][C::D / 8][4];
     float m[MT][2], l[MT][2];
+    float corr[MT][2];  // int8 keys: bias * row sum of q
     int lim[MT][2];
 
     int stage = 0;
@@ -1097,22 +1123,45 @@ __device__ void consumer_mma_mt(const Params& p, uint8_t* smem, volatile int* ab
             // copy the segment's query rows out of the stage (it will be reused)
             const uint4* src = reinterpret_cast<const uint4*>(smem + stage * C::STAGE_BYTES + C::Q_OFF);
             uint4* dst = reinterpret_cast<uint4*>(smem + C::QP_OFF);
-            for (int i = threadIdx.x; i < C::RP * C::QROW / 16; i += C::NCW * 32) {
-                uint4 v = src[i];
-                if constexpr (C::KQ) {
-                    // fold the channel scales of the int8 keys into q
-                    const int col = i % (C::QROW / 16);  // 8 dims per 16-byte chunk
-                    if (col < C::D / 8) {
-                        const float* sc = p.k_scale + (int64_t)md.kvh * C::D + col * 8;
-                        v.x = scale_h2(v.x, *reinterpret_cast<const float2*>(sc));
-                        v.y = scale_h2(v.y, *reinterpret_cast<const float2*>(sc + 2));
-                        v.z = scale_h2(v.z, *reinterpret_cast<const float2*>(sc + 4));
-                        v.w = scale_h2(v.w, *reinterpret_cast<const float2*>(sc + 6));
-                    }
+            if constexpr (!C::KQ) {
+                for (int i = threadIdx.x; i < C::RP * C::QROW / 16; i += C::NCW * 32) dst[i] = src[i];
+            } else {
+                // int8 keys: q times the channel scales, each 16-dim chunk
+                // stored in the permuted order of k8_frag (dims 0,1,4,5,8,9,12,13
+                // then 2,3,6,7,10,11,14,15), so ldmatrix yields matching fragments
+                constexpr int CPR = C::QROW / 16;  // 16-byte chunks per row
+                const float* sc = p.k_scale + (int64_t)md.kvh * C::D;
+                for (int i = threadIdx.x; i < C::RP * (C::D / 16); i += C::NCW * 32) {
+                    const int row = i / (C::D / 16), ks = i % (C::D / 16);
+                    const uint4 a = src[row * CPR + 2 * ks], b = src[row * CPR + 2 * ks + 1];
+                    const float* s16 = sc + 16 * ks;
+                    const uint32_t pr[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+                    uint32_t q2[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        q2[e] = scale_h2(pr[e], *reinterpret_cast<const float2*>(s16 + 2 * e));
+                    dst[row * CPR + 2 * ks] = make_uint4(q2[0], q2[2], q2[4], q2[6]);
+                    dst[row * CPR + 2 * ks + 1] = make_uint4(q2[1], q2[3], q2[5], q2[7]);
                 }
-                dst[i] = v;
             }
             named_bar_sync(2, C::NCW * 32);
+            if constexpr (C::KQ) {
+                // bias corrections of this lane's rows: sums of their q entries
+                // (lane tig adds 32 of the 128 dims)
+#pragma unroll
+                for (int t = 0; t < MT; ++t)
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr) {
+                        const uint32_t* qr = reinterpret_cast<const uint32_t*>(
+                            smem + C::QP_OFF + (t * 16 + gid + rr * 8) * C::QROW) + tig * 16;
+                        float acc = 0.f;
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) acc += h2_sum(qr[e]);
+                        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+                        corr[t][rr] = kCodeBias * acc;
+                    }
+            }
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
 #pragma unroll
@@ -1163,7 +1212,8 @@ __device__ void consumer_mma_mt(const Params& p, uint8_t* smem, volatile int* ab
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         const int pos = pos0 + nt * 8 + (c & 1);
-                        const float v = pos < ((c >> 1) ? lim1 : lim0) ? S[t][nt][c] * sl2 : kNegInf;
+                        const float raw = C::KQ ? S[t][nt][c] - corr[t][c >> 1] : S[t][nt][c];
+                        const float v = pos < ((c >> 1) ? lim1 : lim0) ? raw * sl2 : kNegInf;
                         S[t][nt][c] = v;
                         mx[c >> 1] = fmaxf(mx[c >> 1], v);
                     }

@@ -157,3 +157,21 @@ def test_attention_q8k_edge_cases():
     out16 = pkv.paged_decode_attention(q, dev(kdq), dev(V), dev(tables), dev(lens), D ** -0.5)
     torch.cuda.synchronize()
     assert_close(out, out16.cpu().double().numpy(), "int8 vs fp16 keys")
+
+
+def test_copy_blocks_q8k_is_a_block_copy():
+    nb, Hkv, bs, D = 12, 4, 16, 128
+    rng = np.random.Generator(np.random.PCG64(3))
+    k0 = rng.integers(-128, 128, size=(nb, Hkv, bs, D)).astype(np.int8)
+    v0 = normal_fp16((nb, Hkv, bs, D), 4, "cpu").numpy()
+    kq, vq = torch.as_tensor(k0).cuda(), torch.as_tensor(v0).cuda()
+    pairs = np.array([[1, 7], [3, 0], [11, 5]], np.int32)
+    pkv.paged_kv_copy_blocks_q8k(kq, vq, torch.as_tensor(pairs).cuda())
+    torch.cuda.synchronize()
+    k_ref = k0.copy()
+    for src, dst in pairs:
+        k_ref[dst] = k0[src]
+    _, v_ref = oracle.copy_blocks(v0, v0, pairs)
+    assert np.array_equal(kq.cpu().numpy(), k_ref)
+    assert np.array_equal(vq.cpu().numpy().view(np.uint16), v_ref.view(np.uint16))
+
