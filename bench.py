@@ -281,6 +281,46 @@ def adopt_workload(pkv, wl, extra_cap):
     return pool, tables, nblk
 
 
+BEAMS = 8  # beams per prompt of the beam_search config
+
+
+def build_beam_steps(pkv, wl, n_steps, device, seed, width=BEAMS):
+    """Per-step inputs of beam search over the workload's prompts: each step
+    the survivors are drawn (seeded) within each prompt's beams, the host
+    block manager reorders the tables (kv_beam_reorder) and reserves one slot
+    per beam (copy-on-write pairs for shared partial last blocks)."""
+    import numpy as np
+    import torch
+    from workloads import normal_fp16
+    Hq, Hkv, D = wl.q.shape[-2], wl.spec.Hkv, wl.q.shape[-1]
+    pool, tables, nblk = adopt_workload(pkv, wl, extra_cap=n_steps // wl.spec.bs + 3)
+    rng = np.random.Generator(np.random.PCG64(seed + 7))
+    S = wl.B
+    parents = np.repeat(np.arange(S), width).astype(np.int32)
+    beam_len = wl.lens.astype(np.int32)
+    steps = []
+    for i in range(n_steps):
+        tables, nblk = pool.beam_reorder(tables, nblk, parents)
+        lens = beam_len[parents].astype(np.int32)
+        slots, pairs = pool.reserve_slots(tables, nblk, lens)
+        beam_len = lens + 1
+        n = S * width
+        steps.append({
+            "q": normal_fp16((n, 1, Hq, D), seed * 100003 + 3 * i, device),
+            "k_new": normal_fp16((n, Hkv, D), seed * 100003 + 3 * i + 1, device),
+            "v_new": normal_fp16((n, Hkv, D), seed * 100003 + 3 * i + 2, device),
+            "slots": torch.as_tensor(slots, device=device),
+            "pairs": torch.as_tensor(pairs, device=device) if len(pairs) else None,
+            "tables": torch.as_tensor(tables.copy(), device=device),
+            "lens": torch.as_tensor(beam_len.copy(), device=device),
+            "lens_host": beam_len.copy(),
+            "tables_host": tables.copy(),
+        })
+        parents = np.concatenate([g * width + rng.integers(0, width, size=width)
+                                  for g in range(S)]).astype(np.int32)
+    return steps
+
+
 def build_steps(pkv, wl, n_steps, device, seed):
     """Per-step inputs: slots / copy pairs from the host block manager, new
     K/V, queries, tables and lengths after the append."""
@@ -405,16 +445,20 @@ def run_ours(args):
     base, q8k = split_workload(args.workload)
     spec = CONFIGS[base]
     seed = rank_seed(spec.seed, rank)
-    wl = make_workload(base, device, seed=seed, B=args.batch or None)
+    beams = base == "beam_search"
+    n_distinct = min(args.warmup + args.steps, 64)
+    spare = (n_distinct // spec.bs + 3) * BEAMS * (args.batch or spec.B) * 2 if beams else 0
+    wl = make_workload(base, device, seed=seed, B=args.batch or None, spare_blocks=spare)
     q_len = spec.q_len
     Hq, Hkv, D, bs = spec.Hq, spec.Hkv, spec.D, spec.bs
     k_bytes = 1 if q8k else 2
-    n_distinct = min(args.warmup + args.steps, 64)
-    steps = build_steps(pkv, wl, n_distinct, device, seed)
+    steps = (build_beam_steps(pkv, wl, n_distinct, device, seed) if beams
+             else build_steps(pkv, wl, n_distinct, device, seed))
     kq = ksc = None
     if q8k:
         kq, ksc = quantise_pool_device(pkv, wl)
-    out = torch.empty((wl.B, q_len, Hq, D), dtype=torch.float16, device=device)
+    n_rows = steps[0]["q"].shape[0]  # sequences (beams) attended per step
+    out = torch.empty((n_rows, q_len, Hq, D), dtype=torch.float16, device=device)
     ws = torch.empty(pkv.workspace_size(Hq, Hkv, q_len, D), dtype=torch.uint8, device=device)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=device)
@@ -434,6 +478,7 @@ def run_ours(args):
     ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     launches = 0
+    n_cow = 0
     kv_bytes_total = 0
     alg_attn = []
     th_tokens = 0
@@ -449,6 +494,7 @@ def run_ours(args):
             step(i, ev_a[k])
             ev_e[k].record(stream)
             launches += 3 + (1 if st["pairs"] is not None else 0)
+            n_cow += 0 if st["pairs"] is None else int(st["pairs"].shape[0])
             kvb, allb = algorithmic_bytes(st["lens_host"], Hq, Hkv, D, bs, q_len, k_bytes)
             kv_bytes_total += kvb
             alg_attn.append(allb)
@@ -483,9 +529,10 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
             "config": {
                 "workload": args.workload + (f"[B={wl.B}]" if args.batch else ""),
-                "description": spec.description, "B": wl.B,
+                "description": spec.description, "B": n_rows,
                 "Hq": Hq, "Hkv": Hkv, "head_dim": D, "block_size": bs, "q_len": q_len,
-                "mean_context": float(np.mean(wl.lens)),
+                "mean_context": float(np.mean(steps[-1]["lens_host"])),
+                "cow_copies_per_step": round(n_cow / args.steps, 2),
                 "step": "copy-on-write copies + append 1 token/sequence + paged attention + merge",
                 "k_pool": ("int8 codes, fp32 scale per (KV head, channel); V fp16" if q8k
                            else "fp16"),
@@ -507,6 +554,10 @@ def run_ours(args):
         if world == 1 and args.cpu_seconds > 0:
             # the timed appends only wrote slots past each sequence's original
             # length, so the workload's original tokens are still in the pools
+            if beams:  # the oracle over the beams of the last step
+                wl.block_tables = steps[-1]["tables_host"]
+                wl.lens = steps[-1]["lens_host"]
+                wl.q = steps[-1]["q"]
             result["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, q8k)
     if world > 1:
         dist.destroy_process_group()

@@ -133,6 +133,20 @@ int kv_batch_reserve_slots(kv_pool* pool, int32_t B, int32_t* tables, int32_t ta
                            int64_t* slots_out /* [B] */, int32_t* cow_pairs_out /* [2B] */,
                            int32_t* n_cow_out, int32_t* n_done_out);
 
+/* Beam-search step ([T3] §2.3 (2): a fork copies only the block table; blocks
+ * stay shared until a beam writes, then copy-on-write).  tables [n_beams]
+ * [table_capacity] with n_blocks[b] live entries each; new beam i continues
+ * old beam parents[i]: new_tables[i] (same capacity, -1 padded; must not
+ * overlap tables) is a copy of its table and each of those blocks gets one
+ * more reference; then every old beam's references are dropped, beam by beam
+ * in order (a block reaching zero goes on the free list).  Nothing is copied
+ * on the device: the next kv_batch_reserve_slots emits the copy-on-write pairs
+ * for the beams whose shared last block is partial.  KV_ERR_INVALID (nothing
+ * changes) on a parent out of range or a table entry that is not live. */
+int kv_beam_reorder(kv_pool* pool, const int32_t* tables, const int32_t* n_blocks, int32_t n_beams,
+                    int32_t table_capacity, const int32_t* parents, int32_t n_new,
+                    int32_t* new_tables, int32_t* new_n_blocks);
+
 /* Prefix cache ([T3] §2.3 (3): requests sharing a prompt prefix are found by
  * hashing block contents and point their tables at the same physical blocks;
  * §2.3 (1): blocks nothing references are kept in LRU order).  A cached block

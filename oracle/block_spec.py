@@ -229,3 +229,31 @@ class PrefixCacheSpec:
             self.pool.free([b])
             out.append(b)
         return OK, out
+
+
+def beam_reorder(pool: BlockPoolSpec, tables, parents):
+    """One beam-search step over the pool's bookkeeping ([T3] §2.3 (2): a
+    fork copies only the block table; the blocks stay shared until a beam
+    writes into one).  New beam i continues old beam parents[i]: it gets a
+    copy of that table and one more reference on each of its blocks; then
+    every old beam's table is released, beam by beam in order (a block whose
+    count reaches zero goes on the free list).  References are added before
+    any is dropped, so a surviving block is never freed.  Returns
+    (status, new_tables); nothing changes on an error."""
+    n = len(tables)
+    if any(not 0 <= p < n for p in parents):
+        return ERR_INVALID, []
+    for t in tables:
+        for b in t:
+            if not 0 <= b < pool.num_blocks or pool.refcount[b] == 0:
+                return ERR_INVALID, []
+    new = [list(tables[p]) for p in parents]
+    for t in new:
+        for b in t:
+            pool.refcount[b] += 1
+    for t in tables:
+        for b in t:
+            pool.refcount[b] -= 1
+            if pool.refcount[b] == 0:
+                pool.free_stack.append(b)
+    return OK, new

@@ -149,6 +149,19 @@ class KVPool:
               "kv_batch_reserve_slots")
         return slots, pairs[:ncow.value].copy()
 
+    def beam_reorder(self, tables: np.ndarray, n_blocks: np.ndarray, parents):
+        """One beam-search step: new beam i continues old beam parents[i].
+        Returns (new_tables int32 [n_new][cap], new_n_blocks int32 [n_new])."""
+        assert tables.dtype == np.int32 and tables.flags["C_CONTIGUOUS"] and tables.ndim == 2
+        nb = np.ascontiguousarray(n_blocks, dtype=np.int32)
+        par = np.ascontiguousarray(parents, dtype=np.int32)
+        B, cap = tables.shape
+        new = np.full((max(par.size, 1), cap), -1, np.int32)
+        new_nb = np.zeros(max(par.size, 1), np.int32)
+        check(_L.kv_beam_reorder(self._h, _i32p(tables), _i32p(nb), B, cap, _i32p(par), par.size,
+                                 _i32p(new), _i32p(new_nb)), "kv_beam_reorder")
+        return new[:par.size].copy(), new_nb[:par.size].copy()
+
     # -- prefix cache --------------------------------------------------------
     def prefix_match(self, tokens) -> list:
         """Cached blocks holding the longest cached prefix of ``tokens`` (one

@@ -67,6 +67,7 @@ SIGNATURES = {
                                  _i32, _i32, _i32, _i32, _P], ctypes.c_int),
     "paged_decode_attention_static_ws": ([_P, _P, _P, _P, _i32, _P, ctypes.c_float, _P, _i32,
                                           _i32, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
+    "kv_beam_reorder": ([_P, _PI32, _PI32, _i32, _i32, _PI32, _i32, _PI32, _PI32], ctypes.c_int),
     "kv_prefix_match": ([_P, _PI32, _i32, _PI32, _i32, _PI32], ctypes.c_int),
     "kv_prefix_register": ([_P, _PI32, _i32, _PI32, _i32, _PI32], ctypes.c_int),
     "kv_prefix_evict": ([_P, _i32, _PI32, _PI32], ctypes.c_int),

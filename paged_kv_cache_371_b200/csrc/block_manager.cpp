@@ -208,3 +208,50 @@ int kv_batch_reserve_slots(kv_pool* pool, int32_t B, int32_t* tables, int32_t ta
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Beam-search step ("LLM 推理优化：KV Cache、PagedAttention 与量化" §2.3 (2): a
+// fork copies only the block table; blocks stay shared until a beam writes
+// into one, then copy-on-write).  New beam i continues old beam parents[i];
+// references are added for every new table before the old tables' are
+// dropped (old beams released in order), so surviving blocks are never freed.
+extern "C" int kv_beam_reorder(kv_pool* pool, const int32_t* tables, const int32_t* n_blocks,
+                               int32_t n_beams, int32_t table_capacity, const int32_t* parents,
+                               int32_t n_new, int32_t* new_tables, int32_t* new_n_blocks)
+{
+    if (!pool || n_beams < 0 || n_new < 0 || table_capacity < 1 ||
+        (n_beams > 0 && (!tables || !n_blocks)) || (n_new > 0 && (!parents || !new_tables || !new_n_blocks)))
+        return kv_fail(KV_ERR_INVALID, "kv_beam_reorder: bad argument");
+    const size_t cap = static_cast<size_t>(table_capacity);
+    if (n_new > 0 && n_beams > 0 && new_tables < tables + static_cast<size_t>(n_beams) * cap &&
+        tables < new_tables + static_cast<size_t>(n_new) * cap)
+        return kv_fail(KV_ERR_INVALID, "kv_beam_reorder: new_tables overlaps tables");
+    for (int32_t i = 0; i < n_new; ++i)
+        if (parents[i] < 0 || parents[i] >= n_beams)
+            return kv_fail(KV_ERR_INVALID, "kv_beam_reorder: parent out of range");
+    for (int32_t b = 0; b < n_beams; ++b) {
+        if (n_blocks[b] < 0 || n_blocks[b] > table_capacity)
+            return kv_fail(KV_ERR_INVALID, "kv_beam_reorder: bad block count");
+        for (int32_t k = 0; k < n_blocks[b]; ++k) {
+            const int32_t id = tables[b * cap + k];
+            if (id < 0 || id >= pool->cfg.num_blocks || pool->refcount[id] == 0)
+                return kv_fail(KV_ERR_INVALID, "kv_beam_reorder: table holds a block that is not live");
+        }
+    }
+    for (int32_t i = 0; i < n_new; ++i) {
+        const int32_t p = parents[i];
+        const int32_t nb = n_blocks[p];
+        for (int32_t k = 0; k < table_capacity; ++k) {
+            const int32_t id = k < nb ? tables[p * cap + k] : -1;
+            new_tables[i * cap + k] = id;
+            if (id >= 0) ++pool->refcount[id];
+        }
+        new_n_blocks[i] = nb;
+    }
+    for (int32_t b = 0; b < n_beams; ++b)
+        for (int32_t k = 0; k < n_blocks[b]; ++k) {
+            const int32_t id = tables[b * cap + k];
+            if (--pool->refcount[id] == 0) pool->free_stack.push_back(id);
+        }
+    return KV_OK;
+}

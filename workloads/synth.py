@@ -86,6 +86,14 @@ CONFIGS = {
         lens=_uniform(32, 512),
         description="64 requests sharing one 2048-token prefix (same physical blocks) plus "
                     "private suffixes U[32,512]; GQA 32/8, head_dim 128, block 16"),
+    "beam_search": ConfigSpec(
+        "beam_search", 7, B=32, Hq=32, Hkv=8, D=128, bs=16, q_len=1,
+        lens=_uniform(500, 2000),
+        description="beam search: 32 prompts U[500,2000] x 8 beams = 256 beams; per step the "
+                    "survivors are drawn within each prompt's beams (fork / reorder of block "
+                    "tables), shared partial last blocks are copied on write in one batched "
+                    "call, one token is appended per beam, then decode attention; GQA 32/8, "
+                    "head_dim 128, block 16"),
     "long_decode": ConfigSpec(
         "long_decode", 5, B=8, Hq=32, Hkv=8, D=128, bs=16, q_len=1, lens=_const(32768),
         description="8 sequences of 32768 tokens, GQA 32/8, head_dim 128, block 16"),
