@@ -405,9 +405,35 @@ def run_prefill(args):
     tot_fl, _, t_all = aggregate(fl * args.steps, 0, sum(step_ms), world, device)
     value = tot_fl / (t_all * 1e-3) / 1e12
     achieved = fl / (statistics.mean(attn_ms) * 1e-3) / 1e12
+
+    # e2e: the chunk's queries and K/V from pinned host memory, the output back
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hs = (x.cpu().pin_memory() for x in (wl.q, kn, vn, slots))
+        dq, dk, dv, ds = (torch.empty_like(x) for x in (wl.q, kn, vn, slots))
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hs))
+        times = []
+        for k in range(args.warmup + args.steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for d_, h_ in ((dq, hq), (dk, hk), (dv, hv), (ds, hs)):
+                d_.copy_(h_, non_blocking=True)
+            pkv.paged_kv_append(dk, dv, ds, wl.k_pool, wl.v_pool)
+            pkv.paged_prefill_attention(dq, wl.k_pool, wl.v_pool, bt, cl, wl.scale, q_len, out=out)
+            hout.copy_(out, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if k >= args.warmup:
+                times.append(e0.elapsed_time(e1))
+        e_fl, _, e_t = aggregate(fl * args.steps, 0, sum(times), world, device)
+        e2e = {"value": round(e_fl / (e_t * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout.numel() * hout.element_size()}
     if rank != 0:
         return None
-    return {
+    res = {
         "metric": "paged prefill attention TFLOP/s", "value": round(value, 2), "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(t_all / args.steps, 5), "higher_is_better": True, "scaling": "weak",
@@ -424,6 +450,49 @@ def run_prefill(args):
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }
+    if e2e:
+        res["e2e"] = e2e
+    if world == 1 and args.cpu_seconds > 0:
+        res["cpu_baseline"] = prefill_cpu_baseline(wl, q_len, args.cpu_seconds)
+    return res
+
+
+def prefill_window(wl, q_len, n_seq, n_pos):
+    """Host inputs of a bounded prefill sample: the first n_pos positions of
+    the chunks of the first n_seq sequences (their rows see exactly what they
+    see in the full chunk: lengths cut to L - q_len + n_pos)."""
+    import numpy as np
+    import torch
+    seqs = np.arange(n_seq)
+    tables = wl.block_tables[seqs]
+    lens = (wl.lens[seqs] - q_len + n_pos).astype(np.int32)
+    ids = np.unique(tables[tables >= 0])
+    idx = torch.as_tensor(ids, device=wl.k_pool.device, dtype=torch.long)
+    K = wl.k_pool[idx].cpu().numpy()
+    V = wl.v_pool[idx].cpu().numpy()
+    t2 = np.where(tables >= 0, np.searchsorted(ids, np.maximum(tables, 0)), -1).astype(np.int32)
+    q = wl.q[:n_seq, :n_pos].cpu().numpy().copy()
+    return q, K, V, t2, lens
+
+
+def prefill_cpu_baseline(wl, q_len, target_s):
+    """The oracle over a bounded sample of this run's chunked prefill,
+    repeated to about target_s seconds; reported in TFLOP/s."""
+    import oracle
+    Hq, D = wl.q.shape[-2], wl.q.shape[-1]
+    n_pos = 16
+    q, K, V, t2, lens = prefill_window(wl, q_len, 1, n_pos)
+    reps, spent = 0, 0.0
+    while reps == 0 or spent < target_s:
+        t0 = time.perf_counter()
+        oracle.paged_attention(q, K, V, t2, lens, scale=wl.scale, q_len=n_pos)
+        spent += time.perf_counter() - t0
+        reps += 1
+    fl = prefill_flops(lens, Hq, D, n_pos) * reps
+    return {"value": round(fl / spent / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"the first {n_pos} positions of sequence 0's chunk (all {Hq} heads, "
+                      f"{int(lens[0])} tokens) x {reps} repeat(s), fp64 C oracle, {spent:.2f} s"}
 
 
 def run_ours(args):
@@ -726,6 +795,8 @@ def run_reference(args):
     from workloads.synth import CONFIGS
     base, q8k = split_workload(args.workload)
     spec = CONFIGS[base]
+    if spec.q_len > 32:
+        return run_reference_prefill(args, base, spec, world)
     per_step = max(0.2, min(2.0, 120.0 / max(1, args.steps + args.warmup)))
     wl = oracle_sample(args.workload, per_step)
     k8 = quantise_pool_host(wl.k_pool.numpy()) if q8k else None
@@ -747,6 +818,37 @@ def run_reference(args):
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "kind": "oracle",
                              "cores": oracle.num_threads(), "sample": sample},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def run_reference_prefill(args, base, spec, world):
+    """The oracle on a bounded window of the chunked-prefill workload: the
+    first 16 positions of one sequence's chunk per step."""
+    import oracle
+    from workloads import make_workload
+    wl = make_workload(base, "cpu", B=1, seed=spec.seed)
+    n_pos = 16
+    q, K, V, t2, lens = prefill_window(wl, spec.q_len, 1, n_pos)
+
+    def once():
+        t0 = time.perf_counter()
+        oracle.paged_attention(q, K, V, t2, lens, scale=wl.scale, q_len=n_pos)
+        return time.perf_counter() - t0
+    for _ in range(args.warmup):
+        once()
+    times = [once() for _ in range(args.steps)]
+    fl = prefill_flops(lens, spec.Hq, spec.D, n_pos) * args.steps
+    value = fl / sum(times) / 1e12
+    sample = (f"first {n_pos} positions of one sequence's {spec.q_len}-token chunk per step "
+              f"({int(lens[0])} tokens, {spec.Hq} heads), fp64 C oracle")
+    return {"metric": "paged prefill attention TFLOP/s", "value": round(value, 6), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(sum(times) / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": {"workload": args.workload, "description": spec.description},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "kind": "oracle",
+                             "cores": oracle.num_threads(), "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 
