@@ -10,23 +10,26 @@
 // with the Attention(Q,K,V) formula of the same page's §2 and the tiled
 // online softmax of its §4.2.  Query head h reads KV head h / (Hq/Hkv).
 //
-// Design (sm_100a): one CTA per (sequence, kv head, tile of 128 query rows);
-// the rows of a tile are (position, head-in-group) pairs, so all of them share
-// the K/V tiles staged for their KV head.  Per 64-token stage:
-//   S = Q K^T   tcgen05.mma kind::f16, M128 N64 K128, fp32 in tensor memory
-//   softmax     4 warps, thread i owns row i (= TMEM lane i): no shuffles
-//   O += P V    tcgen05.mma, M128 N128 K64, P fp16 in tensor memory (it
-//               replaces the stage's S columns), V from shared memory
-// Warp roles: warps 0-3 softmax / epilogue, warp 4 TMA producer, warp 5 TMEM
-// allocation + MMA issue.  S is double-buffered so the next S = Q K^T runs
-// while the softmax of the previous stage is computed; K and V arrive through
-// separate two-slot rings, so a K slot refills as soon as its S is done (the
-// next K tile lands while this stage's softmax and P V run); two CTAs share an
-// SM (96 KB shared memory, 256 TMEM columns each) so one CTA's MMAs run while
-// the other's softmax does.  O is rescaled lazily:
-// only when a row's running maximum grows by more than 2^8 (weights stay below
-// 2^8 otherwise, well within fp16 and fp32).  Every wait is bounded; tensor
-// memory is released on every path out of the kernel.
+// Design (sm_100a): one CTA per SM-sized work item (sequence, kv head, two
+// consecutive tiles of 128 query rows); the rows of a tile are (position,
+// head-in-group) pairs, so both tiles share every K/V tile staged for their KV
+// head.  Per 128-token stage and tile t:
+//   S_t = Q_t K^T  tcgen05.mma kind::f16, M128 N128 K128, fp32 in tensor memory
+//   softmax        4 warps per tile, thread i owns row i (= TMEM lane i): no
+//                  shuffles; two passes over the 128 scores (max, then exp2)
+//   O_t += P_t V   tcgen05.mma, M128 N128 K128, P fp16 in tensor memory (it is
+//                  written over S_t), V from shared memory
+// Warp roles: warps 0-7 softmax / epilogue (4 per tile), warp 8 TMA producer,
+// warp 9 TMEM allocation + MMA issue.  Tensor memory: S_t and O_t for both
+// tiles (512 columns).  S is single-buffered per tile (S_t(j+1) waits for
+// P V_t(j)); the two tiles ping-pong: while one tile is in its softmax the
+// other's MMAs run, and the tiles' exp2 passes take turns so that each has the
+// MUFU pipe to itself.  K and V arrive through separate two-slot rings
+// (32 KB slots) shared by the tiles; the producer and the MMA warp poll their
+// barriers and issue whatever is ready.  O is rescaled lazily: only when a
+// row's running maximum grows by more than 2^8 (weights stay below 2^8
+// otherwise, well within fp16 and fp32).  Every wait is bounded; tensor memory
+// is released on every path out of the kernel.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -44,30 +47,39 @@ namespace pkv_prefill {
 using namespace pkv;
 
 constexpr int D = 128;          // head dim served by this kernel
-constexpr int M = 128;          // query rows per CTA (TMEM lanes)
-constexpr int TS = 64;          // tokens per stage (S columns)
+constexpr int M = 128;          // query rows per tile (TMEM lanes)
+constexpr int NT = 2;           // query tiles per CTA; they share every K/V stage
+constexpr int TS = 128;         // tokens per stage (S columns)
 constexpr int KV_SLOTS = 2;     // slots in each of the K and V rings
-constexpr int NTHREADS = 192;   // 4 softmax warps, producer, MMA warp
-constexpr int TMEM_COLS = 256;  // S0 [0,64) S1 [64,128) O [128,256)
+constexpr int SM_WARPS = 4 * NT;               // softmax warps: 4 per tile
+constexpr int PRODUCER_WARP = SM_WARPS;
+constexpr int MMA_WARP = SM_WARPS + 1;
+constexpr int NTHREADS = 32 * (SM_WARPS + 2);
+// tensor memory: tile t's S at t*TS (P is written over its first TS/2
+// columns), its O at O_COL + t*D: 2 * (128 + 128) = 512 columns
+constexpr int O_COL = NT * TS;
+constexpr int TMEM_COLS = O_COL + NT * D;
+static_assert(TMEM_COLS == 512, "tensor memory layout");
 constexpr uint64_t kWait = 2000000000ull;
 constexpr float kNegInf = -__builtin_huge_valf();
 constexpr float kRescaleThreshold = 8.f;  // log2 units
 
 // shared memory layout (bytes, from a 1024-aligned base)
-constexpr int Q_OFF = 0;                        // [2 halves][128 rows][128 B]
-constexpr int Q_BYTES = 2 * M * 128;            // 32 KB
-constexpr int KV_HALF = TS * 128;               // 8 KB: one 64-column half of 64 tokens
-constexpr int SLOT_BYTES = 2 * KV_HALF;         // 16 KB: K (or V) of one stage
+constexpr int Q_OFF = 0;                        // tile t: [2 halves][128 rows][128 B]
+constexpr int Q_TILE = 2 * M * 128;             // 32 KB
+constexpr int Q_BYTES = NT * Q_TILE;
+constexpr int KV_HALF = TS * 128;               // 16 KB: one 64-column half of a stage
+constexpr int SLOT_BYTES = 2 * KV_HALF;         // 32 KB: K (or V) of one stage
 constexpr int K_OFF = Q_OFF + Q_BYTES;          // K ring
 constexpr int V_OFF = K_OFF + KV_SLOTS * SLOT_BYTES;  // V ring
 constexpr int BAR_OFF = V_OFF + KV_SLOTS * SLOT_BYTES;
-// barriers: q_full, kfull[KS], kempty[KS], vfull[KS], vempty[KS], s_full[2],
-// s_free[2], p_full[2], drain
-constexpr int NBARS = 1 + 4 * KV_SLOTS + 2 + 2 + 2 + 1;
+// barriers: q_full, kfull[KS], kempty[KS], vfull[KS], vempty[KS], per tile
+// s_full, s_free, p_full; drain; exp turn per tile
+constexpr int NBARS = 1 + 4 * KV_SLOTS + 3 * NT + 1 + NT;
 constexpr int TMEM_SLOT_OFF = BAR_OFF + NBARS * 8;
 constexpr int SMEM_USED = TMEM_SLOT_OFF + 16;
 constexpr int SMEM_ALLOC = SMEM_USED + 1024;
-static_assert(2 * (SMEM_ALLOC + 1024) <= 233472, "two CTAs per SM must fit");
+static_assert(SMEM_ALLOC <= 232448, "one CTA per SM must fit");
 
 // Progress watchdog for the polling loops: true once kWait of wall time has
 // passed without progress (the clock is read every 1024 idle polls).
@@ -210,7 +222,7 @@ __host__ __device__ constexpr uint32_t idesc_f16(int m, int n, bool b_mn_major)
            | ((uint32_t)(m >> 4) << 24);       // M / 16
 }
 
-__global__ void __launch_bounds__(NTHREADS, 2)
+__global__ void __launch_bounds__(NTHREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ CUtensorMap tmQ, const Params p)
 {
@@ -222,36 +234,42 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t bar0 = sb + BAR_OFF;
     const uint32_t q_full = bar0;
-    // K and V rings are separate: a K slot is free once S = Q K^T of its
-    // stage is done, well before that stage's P V, so the K tile of a later
-    // stage is in flight while the softmax and P V of this one run.
+    // K and V rings are separate and shared by the NT query tiles: a K slot
+    // is free once every tile's S = Q K^T of its stage is done, a V slot once
+    // every tile's P V is.
     auto kfull = [&](int i) { return bar0 + 8 * (1 + i); };
     auto kempty = [&](int i) { return bar0 + 8 * (1 + KV_SLOTS + i); };
     auto vfull = [&](int i) { return bar0 + 8 * (1 + 2 * KV_SLOTS + i); };
     auto vempty = [&](int i) { return bar0 + 8 * (1 + 3 * KV_SLOTS + i); };
-    auto s_full = [&](int b) { return bar0 + 8 * (1 + 4 * KV_SLOTS + b); };
-    auto s_free = [&](int b) { return bar0 + 8 * (3 + 4 * KV_SLOTS + b); };
-    // one P barrier per S buffer: a softmax warp can run a stage ahead of the
-    // others, but not two (stage j+2 needs P V of stage j, hence every warp's
-    // arrive for stage j), so arrivals for different stages never share a phase
-    auto p_full = [&](int b) { return bar0 + 8 * (5 + 4 * KV_SLOTS + b); };
-    const uint32_t drain = bar0 + 8 * (7 + 4 * KV_SLOTS);
+    // per tile t: S full, S free (the P V that read P over it is done), P
+    // written.  S is single-buffered per tile: S_t(j+1) waits for P V_t(j),
+    // which needs all four warps' arrive for stage j, so a warp never passes
+    // stage j before the others of its tile arrived for it.
+    auto s_full = [&](int t) { return bar0 + 8 * (1 + 4 * KV_SLOTS + 3 * t); };
+    auto s_free = [&](int t) { return bar0 + 8 * (2 + 4 * KV_SLOTS + 3 * t); };
+    auto p_full = [&](int t) { return bar0 + 8 * (3 + 4 * KV_SLOTS + 3 * t); };
+    const uint32_t drain = bar0 + 8 * (1 + 4 * KV_SLOTS + 3 * NT);
+    // exp turns: the two tiles' exponential passes alternate (tile 0 for
+    // stage j, tile 1 for stage j, tile 0 for stage j+1, ...) so that one tile
+    // has the MUFU pipe while the other's MMAs run.  turn(t) completes a
+    // phase when the other tile's four warps finished an exp pass.
+    auto turn = [&](int t) { return bar0 + 8 * (2 + 4 * KV_SLOTS + 3 * NT + t); };
 
-    // work item
-    const int tile = blockIdx.x % p.tiles_per_head;
+    // work item: NT consecutive tiles of one (sequence, kv head)
+    const int pair = blockIdx.x % p.tiles_per_head;
     const int kvh = (blockIdx.x / p.tiles_per_head) % p.Hkv;
     const int s = blockIdx.x / (p.tiles_per_head * p.Hkv);
     const int pos_per_tile = M / p.G;
-    const int j0 = tile * pos_per_tile;                    // first window position
-    int jn = p.q_len - j0;
-    if (jn > pos_per_tile) jn = pos_per_tile;              // positions in this tile
+    const int jbase = pair * NT * pos_per_tile;            // first window position
+    int jn_all = p.q_len - jbase;
+    if (jn_all > NT * pos_per_tile) jn_all = NT * pos_per_tile;  // positions in this CTA
     int32_t L = __ldg(p.context_lens + s);
     if (L > p.max_blocks * p.bs) {
         if (threadIdx.x == 0) atomicOr(p.err, KV_DEV_BAD_BLOCK);
         L = p.max_blocks * p.bs;
     }
-    // last token any row of this tile may see (exclusive end)
-    int kv_end = L - p.q_len + j0 + jn;
+    // last token any row of this CTA may see (exclusive end)
+    int kv_end = L - p.q_len + jbase + jn_all;
     if (kv_end > L) kv_end = L;
     if (kv_end < 0) kv_end = 0;
     const int nst = (kv_end + TS - 1) / TS;
@@ -265,15 +283,16 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             mbar_init(vfull(i), 1);
             mbar_init(vempty(i), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(s_full(b), 1);
-            mbar_init(s_free(b), 1);
-            mbar_init(p_full(b), 4);
+        for (int t = 0; t < NT; ++t) {
+            mbar_init(s_full(t), 1);
+            mbar_init(s_free(t), 1);
+            mbar_init(p_full(t), 4);
         }
         mbar_init(drain, 1);
+        for (int t = 0; t < NT; ++t) mbar_init(turn(t), 4);
         fence_barrier_init();
     }
-    if (warp == 5) {
+    if (warp == MMA_WARP) {
         tmem_alloc(sb + TMEM_SLOT_OFF, TMEM_COLS);
         tmem_relinquish();
     }
@@ -282,24 +301,27 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + TMEM_SLOT_OFF);
 
-    if (warp == 4) {
+    if (warp == PRODUCER_WARP) {
         // ------------------------------------------------------------ producer
         const uint64_t pol = l2_policy_evict_first();
         if (lane == 0) {
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
             prefetch_tmap(&tmQ);
-            // Q tile: rows r = (j - j0) * G + g; one box per 64-column half,
-            // G heads x pos_per_tile positions (positions past q_len read zeros)
+            // Q tile t: rows r = (j - j0_t) * G + g; one box per 64-column half,
+            // G heads x pos_per_tile positions (positions past the chunk are
+            // never stored: their rows see no key)
             mbar_arrive_expect_tx(q_full, Q_BYTES);
-            const int z = s * p.q_len + j0;
-            for (int h = 0; h < 2; ++h)
-                asm volatile(
-                    "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-                    " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(sb + Q_OFF + h * M * 128),
-                    "l"(reinterpret_cast<uint64_t>(&tmQ)), "r"(h * 64), "r"(kvh * p.G), "r"(z),
-                    "r"(q_full)
-                    : "memory");
+            for (int t = 0; t < NT; ++t) {
+                const int z = s * p.q_len + jbase + t * pos_per_tile;
+                for (int h = 0; h < 2; ++h)
+                    asm volatile(
+                        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(sb + Q_OFF + t * Q_TILE + h * M * 128),
+                        "l"(reinterpret_cast<uint64_t>(&tmQ)), "r"(h * 64), "r"(kvh * p.G), "r"(z),
+                        "r"(q_full)
+                        : "memory");
+            }
         }
         // K (or V) of stage j into its (free) ring slot: block `lane` of the
         // stage -> rows [lane*bs, lane*bs+bs) of each 64-column half of the slot.
@@ -328,17 +350,15 @@ __global__ void __launch_bounds__(NTHREADS, 2)
                 tma_load_2d(dst + KV_HALF, tm, 64, y, fullb, pol);
             }
         };
-        // slot of stage j free?  (its previous use, stage j - KV_SLOTS, consumed;
-        // lane 0 decides for the warp)
+        // slot of stage j free?  (its previous use, stage j - KV_SLOTS, consumed
+        // by every tile; lane 0 decides for the warp)
         auto slot_free = [&](int j, bool is_v) {
             bool f = true;
             if (j >= KV_SLOTS)
                 f = mbar_test(is_v ? vempty(j % KV_SLOTS) : kempty(j % KV_SLOTS), ((j / KV_SLOTS) - 1) & 1);
             return __shfl_sync(0xffffffffu, f ? 1 : 0, 0) != 0;
         };
-        // Poll both rings and issue whichever slot frees first: a K slot frees
-        // when S of its stage is done, a V slot when P V is; neither waits
-        // behind the other.
+        // Poll both rings and issue whichever slot frees first.
         bool ok = true;
         int k_issued = 0, v_issued = 0;
         Idle idle;
@@ -378,60 +398,70 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             }
         }
         if (lane == 0 && !mbar_wait_bounded(q_full, 0, kWait)) atomicOr(p.err, KV_DEV_TIMEOUT);
-    } else if (warp == 5) {
+    } else if (warp == MMA_WARP) {
         // ------------------------------------------------------------ MMA issue
         if (lane == 0) {
             const uint32_t idS = idesc_f16(M, TS, false);
             const uint32_t idO = idesc_f16(M, D, true);
             bool ok = mbar_wait_bounded(q_full, 0, kWait);
             tc_fence_after();
-            const uint32_t qa = sb + Q_OFF;
-            // Poll and issue whichever is ready: S of the next stage (its K
-            // tile landed and the P V that last read its S buffer is done) or
-            // P V of the oldest stage with P written and V landed.
-            int ns = 0, np = 0;  // S issued, P V issued
+            // Poll and issue whatever is ready, per tile t: S_t of its next
+            // stage (K tile landed, and the P V that read the previous P over
+            // S_t done) or P V_t of its oldest stage with P written and V
+            // landed.  Within a stage the tiles go in order, so the last
+            // tile's issue releases the shared K (or V) slot.  While one tile
+            // is in its softmax, the other's MMAs keep the tensor pipe busy.
+            int ns[NT], np[NT];
+            for (int t = 0; t < NT; ++t) ns[t] = np[t] = 0;
             Idle idle;
-            while (ok && np < nst) {
+            while (ok && np[NT - 1] < nst) {
                 bool prog = false;
-                if (ns < nst && mbar_test(kfull(ns % KV_SLOTS), (ns / KV_SLOTS) & 1) &&
-                    (ns < 2 || mbar_test(s_free(ns & 1), ((ns >> 1) - 1) & 1))) {
-                    tc_fence_after();
-                    const int slot = ns % KV_SLOTS, b = ns & 1;
-                    const uint32_t kb = sb + K_OFF + slot * SLOT_BYTES;
-                    // S_b = Q K^T over 8 k-steps of 16 dims (4 per 64-column half)
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t off = (k & 3) * 32;
-                        const uint64_t a = smem_desc(qa + (k >> 2) * M * 128 + off, 16, 1024);
-                        const uint64_t bd = smem_desc(kb + (k >> 2) * KV_HALF + off, 16, 1024);
-                        umma_f16(tmem + b * TS, a, bd, idS, k > 0 ? 1u : 0u);
+                for (int t = 0; t < NT; ++t) {
+                    const int j = ns[t];
+                    if (j < nst && (t == 0 || j < ns[t - 1]) &&
+                        mbar_test(kfull(j % KV_SLOTS), (j / KV_SLOTS) & 1) &&
+                        (j < 1 || mbar_test(s_free(t), (j - 1) & 1))) {
+                        tc_fence_after();
+                        const uint32_t qa = sb + Q_OFF + t * Q_TILE;
+                        const uint32_t kb = sb + K_OFF + (j % KV_SLOTS) * SLOT_BYTES;
+                        // S = Q K^T, M128 N128, 8 k-steps of 16 dims (4 per half)
+                        for (int k = 0; k < 8; ++k) {
+                            const uint32_t off = (k & 3) * 32;
+                            const uint64_t a = smem_desc(qa + (k >> 2) * M * 128 + off, 16, 1024);
+                            const uint64_t bd = smem_desc(kb + (k >> 2) * KV_HALF + off, 16, 1024);
+                            umma_f16(tmem + t * TS, a, bd, idS, k > 0 ? 1u : 0u);
+                        }
+                        umma_commit(s_full(t));
+                        if (t == NT - 1) umma_commit(kempty(j % KV_SLOTS));  // K of stage j consumed
+                        ++ns[t];
+                        prog = true;
                     }
-                    umma_commit(s_full(b));
-                    umma_commit(kempty(slot));  // K of stage ns consumed
-                    ++ns;
-                    prog = true;
                 }
-                if (np < ns && mbar_test(p_full(np & 1), (np >> 1) & 1) &&
-                    mbar_test(vfull(np % KV_SLOTS), (np / KV_SLOTS) & 1)) {
-                    tc_fence_after();
-                    const int slot = np % KV_SLOTS;
-                    const uint32_t vb = sb + V_OFF + slot * SLOT_BYTES;
-                    // O += P V over 4 k-steps of 16 tokens.  P: fp16 pairs in the
-                    // first 32 columns of S buffer (np & 1).  V is MN-major (dims
-                    // contiguous): 64-dim groups 8 KB apart, 8-token groups 1 KB apart
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t bd = smem_desc(vb + k * 16 * 128, KV_HALF, 1024);
-                        umma_f16_ts(tmem + 2 * TS, tmem + (np & 1) * TS + k * 8, bd, idO,
-                                    (np > 0 || k > 0) ? 1u : 0u);
+                for (int t = 0; t < NT; ++t) {
+                    const int j = np[t];
+                    if (j < ns[t] && (t == 0 || j < np[t - 1]) && mbar_test(p_full(t), j & 1) &&
+                        mbar_test(vfull(j % KV_SLOTS), (j / KV_SLOTS) & 1)) {
+                        tc_fence_after();
+                        const uint32_t vb = sb + V_OFF + (j % KV_SLOTS) * SLOT_BYTES;
+                        // O += P V over 8 k-steps of 16 tokens.  P: fp16 pairs in the
+                        // first 64 columns of S_t.  V is MN-major (dims contiguous):
+                        // 64-dim groups KV_HALF apart, 8-token groups 1 KB apart
+                        for (int k = 0; k < 8; ++k) {
+                            const uint64_t bd = smem_desc(vb + k * 16 * 128, KV_HALF, 1024);
+                            umma_f16_ts(tmem + O_COL + t * D, tmem + t * TS + k * 8, bd, idO,
+                                        (j > 0 || k > 0) ? 1u : 0u);
+                        }
+                        umma_commit(s_free(t));  // P V_t of stage j done: S_t free
+                        if (t == NT - 1) umma_commit(vempty(j % KV_SLOTS));  // V of stage j consumed
+                        ++np[t];
+                        prog = true;
                     }
-                    umma_commit(s_free(np & 1));  // P V of stage np done: S buffer free
-                    umma_commit(vempty(slot));    // V of stage np consumed
-                    ++np;
-                    prog = true;
                 }
-                if (prog)
+                if (prog) {
                     idle.reset();
-                else if (*reinterpret_cast<volatile int*>(&abort_flag) || idle.expired())
-                    ok = false;
+                } else {
+                    if (*reinterpret_cast<volatile int*>(&abort_flag) || idle.expired()) ok = false;
+                }
             }
             if (!ok) {
                 atomicOr(p.err, KV_DEV_TIMEOUT);
@@ -444,71 +474,72 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax
-        const int r = threadIdx.x;  // row = TMEM lane
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-        const int jr = r / p.G;                       // position within the tile
-        const bool row_ok = jr < jn;
-        const int lim = L - p.q_len + j0 + jr;        // last visible token (inclusive)
+        // warps 4t .. 4t+3 serve tile t; thread row r = TMEM lane r
+        const int t = warp >> 2;
+        const int r = (warp & 3) * 32 + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const uint32_t s_col = (uint32_t)(t * TS), o_col = (uint32_t)(O_COL + t * D);
+        const int jr = t * pos_per_tile + r / p.G;    // position within this CTA's window
+        const bool row_ok = jr < jn_all;
+        const int lim = L - p.q_len + jbase + jr;     // last visible token (inclusive)
+        const float sl2 = p.scale_log2;
         float m = kNegInf, l = 0.f;
         bool ok = true;
+        // 64 scores of half h of the stage, masked past what the row sees
+        auto load_half = [&](int h, int vis, bool full, float (&sv)[64]) {
+            float t32[32];
+            tmem_ld32(lane_base + s_col + 64 * h, t32);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sv[i] = t32[i];
+            tmem_ld32(lane_base + s_col + 64 * h + 32, t32);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sv[32 + i] = t32[i];
+            tmem_wait_ld();
+            if (!full) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) sv[c] = 64 * h + c < vis ? sv[c] : kNegInf;
+            }
+        };
         for (int j = 0; j < nst && ok; ++j) {
-            const int b = j & 1, slot = j % KV_SLOTS;
-            ok = mbar_wait_bounded(s_full(b), (j >> 1) & 1, kWait);
+            const int slot = j % KV_SLOTS;
+            ok = mbar_wait_bounded(s_full(t), j & 1, kWait);
             if (!ok) break;
             tc_fence_after();
-            float sv[TS];
-            {
-                float t32[32];
-                tmem_ld32(lane_base + b * TS, t32);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) sv[i] = t32[i];
-                tmem_ld32(lane_base + b * TS + 32, t32);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) sv[32 + i] = t32[i];
-            }
-            tmem_wait_ld();
             const int t0 = j * TS;
             int ntok = kv_end - t0;                   // staged tokens (< TS: last stage)
             if (ntok > TS) ntok = TS;
             int vis = lim - t0 + 1;                   // columns this row may see
             if (vis > ntok) vis = ntok;
             if (!row_ok) vis = 0;
-            // raw scores stay unscaled; scale > 0 commutes with the maximum
-            if (!__all_sync(0xffffffffu, vis >= TS)) {  // boundary stage: mask
-#pragma unroll
-                for (int c = 0; c < TS; ++c) sv[c] = c < vis ? sv[c] : kNegInf;
-            }
+            const bool full = __all_sync(0xffffffffu, vis >= TS);
+            // pass 1: the row maximum (raw scores; scale > 0 commutes with it)
             float mx4[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
+            for (int h = 0; h < 2; ++h) {
+                float sv[64];
+                load_half(h, vis, full, sv);
 #pragma unroll
-            for (int c = 0; c < TS; c += 4) {
-                mx4[0] = fmaxf(mx4[0], sv[c]);
-                mx4[1] = fmaxf(mx4[1], sv[c + 1]);
-                mx4[2] = fmaxf(mx4[2], sv[c + 2]);
-                mx4[3] = fmaxf(mx4[3], sv[c + 3]);
+                for (int c = 0; c < 64; c += 4) {
+                    mx4[0] = fmaxf(mx4[0], sv[c]);
+                    mx4[1] = fmaxf(mx4[1], sv[c + 1]);
+                    mx4[2] = fmaxf(mx4[2], sv[c + 2]);
+                    mx4[3] = fmaxf(mx4[3], sv[c + 3]);
+                }
             }
-            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * p.scale_log2;
-            // P of this stage goes to its own S buffer, which no pending P V
-            // reads, so the exponentials need not wait for the previous P V;
-            // only a rescale of O does.
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
+            // S_t(j) was issued after P V_t(j-1) finished and P V_t(j) waits for
+            // this warp's arrive: O is quiet, a rescale needs no wait.
             const bool grow = mx > m + kRescaleThreshold;
             if (__any_sync(0xffffffffu, grow)) {
                 const float mn = grow ? mx : m;
                 const float alpha = mn == kNegInf ? 1.f : ex2(m - mn);
                 if (j >= 1) {
-                    // P V of stage j-1 (the last one issued) must be done: the
-                    // ((j-1)/2)-th phase of its S buffer's barrier.  The phase
-                    // before it (stage j-3) completed before S(j-1) was issued,
-                    // and the one after needs this warp's arrive below.
-                    ok = mbar_wait_bounded(s_free((j - 1) & 1), ((j - 1) >> 1) & 1, kWait);
-                    if (!ok) break;
-                    tc_fence_after();
                     for (int c0 = 0; c0 < D; c0 += 32) {
                         float o32[32];
-                        tmem_ld32(lane_base + 2 * TS + c0, o32);
+                        tmem_ld32(lane_base + o_col + c0, o32);
                         tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 32; ++i) o32[i] *= alpha;
-                        tmem_st32(lane_base + 2 * TS + c0, o32);
+                        tmem_st32(lane_base + o_col + c0, o32);
                     }
                     tmem_wait_st();
                 }
@@ -516,12 +547,20 @@ __global__ void __launch_bounds__(NTHREADS, 2)
                 m = mn;
             }
             const float mu = m == kNegInf ? 0.f : m;
-            // P row: fp16 weights packed in pairs into the first 32 columns of
-            // this stage's S buffer (the tensor-memory A operand of P V)
+            // wait for this tile's exp turn: tile 0's pass of stage j follows
+            // tile 1's pass of stage j-1, tile 1's follows tile 0's of stage j.
+            // Neither side can run two phases ahead of the other.
+            if (t == 1 || j >= 1) {
+                ok = mbar_wait_bounded(turn(t), (t == 1 ? j : j - 1) & 1, kWait);
+                if (!ok) break;
+            }
+            // pass 2: fp16 weights packed in pairs into the first 64 columns of
+            // S_t (half h -> columns 32h ..; those S columns are already read)
             float ps4[4] = {0.f, 0.f, 0.f, 0.f};
-            {
+            for (int h = 0; h < 2; ++h) {
+                float sv[64];
+                load_half(h, vis, full, sv);
                 float pw[32];
-                const float sl2 = p.scale_log2;
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const float a = ex2(fmaf(sv[2 * e], sl2, -mu));
@@ -529,17 +568,21 @@ __global__ void __launch_bounds__(NTHREADS, 2)
                     ps4[e & 3] += a + bq;
                     pw[e] = __uint_as_float(pack_half2(a, bq));
                 }
-                tmem_st32(lane_base + b * TS, pw);
+                tmem_st32(lane_base + s_col + 32 * h, pw);
             }
             l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(turn(1 - t));  // the other tile's exp turn
             // V rows past the staged tokens must be finite zeros for the MMA
-            // (the copy of this stage's V must have landed first; V of stage
-            // j+2 cannot start before this stage's P V, so the phase is this one)
-            if (ntok < TS) {
+            // (tile 0 writes them; tile 1's P V is issued after tile 0's, which
+            // waited for these writes).  The copy of this stage's V must have
+            // landed first; V of stage j+KS cannot start before P V of stage j,
+            // so the phase is this one.
+            if (t == 0 && ntok < TS) {
                 ok = mbar_wait_bounded(vfull(slot), (j / KV_SLOTS) & 1, kWait);
                 if (!ok) break;
                 uint8_t* vb = smem + V_OFF + slot * SLOT_BYTES;
-                for (int i = r; i < (TS - ntok) * 16; i += 128) {
+                for (int i = r; i < (TS - ntok) * 16; i += M) {
                     const int row = ntok + i / 16, ch = i % 16;  // 16 chunks: 2 halves x 8
                     *reinterpret_cast<uint4*>(vb + (ch >> 3) * KV_HALF + row * 128 + ((ch & 7) << 4)) =
                         make_uint4(0, 0, 0, 0);
@@ -548,9 +591,9 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             fence_proxy_async();  // the V zeros above are read by the tensor core
             tmem_wait_st();
             tc_fence_before();
-            // all 128 softmax threads wrote their part: one arrive per warp
+            // the tile's 128 softmax threads wrote their part: one arrive per warp
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full(b));
+            if (lane == 0) mbar_arrive(p_full(t));
         }
         // epilogue: O / l, fp16, one 256-byte row per thread
         // (the MMA warp commits `drain` once, after the last P V)
@@ -563,11 +606,11 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         } else {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            __half* dst = p.out + (((int64_t)s * p.q_len + j0 + jr) * p.Hq + (int64_t)kvh * p.G +
+            __half* dst = p.out + (((int64_t)s * p.q_len + jbase + jr) * p.Hq + (int64_t)kvh * p.G +
                                    (r % p.G)) * D;
             for (int c0 = 0; c0 < D; c0 += 32) {
                 float o32[32];
-                tmem_ld32(lane_base + 2 * TS + c0, o32);
+                tmem_ld32(lane_base + o_col + c0, o32);
                 tmem_wait_ld();
                 if (nst == 0) {  // nothing visible (context shorter than the window)
 #pragma unroll
@@ -589,7 +632,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == MMA_WARP) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
@@ -664,7 +707,8 @@ extern "C" int paged_prefill_attention(const void* q, const void* k_pool, const 
     if (rc != KV_OK) return rc;
     const int ppt = M / G;
     const int tiles = (q_len + ppt - 1) / ppt;
-    const uint64_t grid = (uint64_t)B * Hkv * tiles;
+    const int groups = (tiles + NT - 1) / NT;  // CTAs per (sequence, kv head)
+    const uint64_t grid = (uint64_t)B * Hkv * groups;
     if (grid >= (1ull << 31)) return kv_fail(KV_ERR_INVALID, "paged_prefill_attention: grid too large");
     // K / V pools as [rows][128] fp16, box = [bs rows][64 columns]
     CUtensorMap tk, tv, tq;
@@ -694,7 +738,7 @@ extern "C" int paged_prefill_attention(const void* q, const void* k_pool, const 
     prm.G = G;
     prm.bs = block_size;
     prm.num_blocks = num_blocks;
-    prm.tiles_per_head = tiles;
+    prm.tiles_per_head = groups;
     prm.scale_log2 = scale * 1.4426950408889634f;
     static std::mutex amu;
     static unsigned long long configured = 0;
