@@ -405,7 +405,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const uint32_t idO = idesc_f16(M, D, true);
             bool ok = mbar_wait_bounded(q_full, 0, kWait);
             tc_fence_after();
-            // Poll and issue whatever is ready, per tile t: S_t of its next
+            // Poll and issue whatever is ready (P V first: it frees the S
+            // buffer its tile's next S needs), per tile t: S_t of its next
             // stage (K tile landed, and the P V that read the previous P over
             // S_t done) or P V_t of its oldest stage with P written and V
             // landed.  Within a stage the tiles go in order, so the last
@@ -416,6 +417,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             Idle idle;
             while (ok && np[NT - 1] < nst) {
                 bool prog = false;
+                for (int t = 0; t < NT; ++t) {
+                    const int j = np[t];
+                    if (j < ns[t] && (t == 0 || j < np[t - 1]) && mbar_test(p_full(t), j & 1) &&
+                        mbar_test(vfull(j % KV_SLOTS), (j / KV_SLOTS) & 1)) {
+                        tc_fence_after();
+                        const uint32_t vb = sb + V_OFF + (j % KV_SLOTS) * SLOT_BYTES;
+                        // O += P V over 8 k-steps of 16 tokens.  P: fp16 pairs in the
+                        // first 64 columns of S_t.  V is MN-major (dims contiguous):
+                        // 64-dim groups KV_HALF apart, 8-token groups 1 KB apart
+                        for (int k = 0; k < 8; ++k) {
+                            const uint64_t bd = smem_desc(vb + k * 16 * 128, KV_HALF, 1024);
+                            umma_f16_ts(tmem + O_COL + t * D, tmem + t * TS + k * 8, bd, idO,
+                                        (j > 0 || k > 0) ? 1u : 0u);
+                        }
+                        umma_commit(s_free(t));  // P V_t of stage j done: S_t free
+                        if (t == NT - 1) umma_commit(vempty(j % KV_SLOTS));  // V of stage j consumed
+                        ++np[t];
+                        prog = true;
+                    }
+                }
                 for (int t = 0; t < NT; ++t) {
                     const int j = ns[t];
                     if (j < nst && (t == 0 || j < ns[t - 1]) &&
@@ -434,26 +455,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         umma_commit(s_full(t));
                         if (t == NT - 1) umma_commit(kempty(j % KV_SLOTS));  // K of stage j consumed
                         ++ns[t];
-                        prog = true;
-                    }
-                }
-                for (int t = 0; t < NT; ++t) {
-                    const int j = np[t];
-                    if (j < ns[t] && (t == 0 || j < np[t - 1]) && mbar_test(p_full(t), j & 1) &&
-                        mbar_test(vfull(j % KV_SLOTS), (j / KV_SLOTS) & 1)) {
-                        tc_fence_after();
-                        const uint32_t vb = sb + V_OFF + (j % KV_SLOTS) * SLOT_BYTES;
-                        // O += P V over 8 k-steps of 16 tokens.  P: fp16 pairs in the
-                        // first 64 columns of S_t.  V is MN-major (dims contiguous):
-                        // 64-dim groups KV_HALF apart, 8-token groups 1 KB apart
-                        for (int k = 0; k < 8; ++k) {
-                            const uint64_t bd = smem_desc(vb + k * 16 * 128, KV_HALF, 1024);
-                            umma_f16_ts(tmem + O_COL + t * D, tmem + t * TS + k * 8, bd, idO,
-                                        (j > 0 || k > 0) ? 1u : 0u);
-                        }
-                        umma_commit(s_free(t));  // P V_t of stage j done: S_t free
-                        if (t == NT - 1) umma_commit(vempty(j % KV_SLOTS));  // V of stage j consumed
-                        ++np[t];
                         prog = true;
                     }
                 }
