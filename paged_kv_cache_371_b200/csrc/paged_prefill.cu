@@ -25,9 +25,12 @@
 // P V_t(j)); the two tiles ping-pong: while one tile is in its softmax the
 // other's MMAs run, and the tiles' exp2 passes take turns so that each has the
 // MUFU pipe to itself.  K and V arrive through separate two-slot rings
-// (32 KB slots) shared by the tiles; the producer and the MMA warp poll their
-// barriers and issue whatever is ready.  O is rescaled lazily: only when a
-// row's running maximum grows by more than 2^8 (weights stay below 2^8
+// (32 KB slots) shared by the tiles; the producer polls both rings and fills
+// whichever slot frees first.  The MMA warp issues in the one order in which
+// the tiles' work becomes ready (S_0 and S_1 of the first stage, then per
+// stage P V_0, the next S_0, P V_1, the next S_1), blocking on each barrier so
+// that it wakes as soon as the barrier completes.  O is rescaled lazily: only
+// when a row's running maximum grows by more than 2^8 (weights stay below 2^8
 // otherwise, well within fp16 and fp32).  Every wait is bounded; tensor memory
 // is released on every path out of the kernel.
 #include <cuda.h>
@@ -81,8 +84,8 @@ constexpr int SMEM_USED = TMEM_SLOT_OFF + 16;
 constexpr int SMEM_ALLOC = SMEM_USED + 1024;
 static_assert(SMEM_ALLOC <= 232448, "one CTA per SM must fit");
 
-// Progress watchdog for the polling loops: true once kWait of wall time has
-// passed without progress (the clock is read every 1024 idle polls).
+// Progress watchdog for the producer's polling loop: true once kWait of wall
+// time has passed without progress (the clock is read every 1024 idle polls).
 struct Idle {
     uint32_t n = 0;
     uint64_t t0 = 0;
@@ -405,63 +408,58 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const uint32_t idO = idesc_f16(M, D, true);
             bool ok = mbar_wait_bounded(q_full, 0, kWait);
             tc_fence_after();
-            // Poll and issue whatever is ready (P V first: it frees the S
-            // buffer its tile's next S needs), per tile t: S_t of its next
-            // stage (K tile landed, and the P V that read the previous P over
-            // S_t done) or P V_t of its oldest stage with P written and V
-            // landed.  Within a stage the tiles go in order, so the last
-            // tile's issue releases the shared K (or V) slot.  While one tile
-            // is in its softmax, the other's MMAs keep the tensor pipe busy.
-            int ns[NT], np[NT];
-            for (int t = 0; t < NT; ++t) ns[t] = np[t] = 0;
-            Idle idle;
-            while (ok && np[NT - 1] < nst) {
-                bool prog = false;
-                for (int t = 0; t < NT; ++t) {
-                    const int j = np[t];
-                    if (j < ns[t] && (t == 0 || j < np[t - 1]) && mbar_test(p_full(t), j & 1) &&
-                        mbar_test(vfull(j % KV_SLOTS), (j / KV_SLOTS) & 1)) {
-                        tc_fence_after();
-                        const uint32_t vb = sb + V_OFF + (j % KV_SLOTS) * SLOT_BYTES;
-                        // O += P V over 8 k-steps of 16 tokens.  P: fp16 pairs in the
-                        // first 64 columns of S_t.  V is MN-major (dims contiguous):
-                        // 64-dim groups KV_HALF apart, 8-token groups 1 KB apart
-                        for (int k = 0; k < 8; ++k) {
-                            const uint64_t bd = smem_desc(vb + k * 16 * 128, KV_HALF, 1024);
-                            umma_f16_ts(tmem + O_COL + t * D, tmem + t * TS + k * 8, bd, idO,
-                                        (j > 0 || k > 0) ? 1u : 0u);
-                        }
-                        umma_commit(s_free(t));  // P V_t of stage j done: S_t free
-                        if (t == NT - 1) umma_commit(vempty(j % KV_SLOTS));  // V of stage j consumed
-                        ++np[t];
-                        prog = true;
-                    }
+            // S_t(j): S = Q_t K^T, M128 N128, 8 k-steps of 16 dims (4 per
+            // 64-dim half); the last tile's issue releases the shared K slot.
+            auto issue_S = [&](int t, int j) {
+                tc_fence_after();
+                const uint32_t qa = sb + Q_OFF + t * Q_TILE;
+                const uint32_t kb = sb + K_OFF + (j % KV_SLOTS) * SLOT_BYTES;
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t off = (k & 3) * 32;
+                    const uint64_t a = smem_desc(qa + (k >> 2) * M * 128 + off, 16, 1024);
+                    const uint64_t bd = smem_desc(kb + (k >> 2) * KV_HALF + off, 16, 1024);
+                    umma_f16(tmem + t * TS, a, bd, idS, k > 0 ? 1u : 0u);
                 }
-                for (int t = 0; t < NT; ++t) {
-                    const int j = ns[t];
-                    if (j < nst && (t == 0 || j < ns[t - 1]) &&
-                        mbar_test(kfull(j % KV_SLOTS), (j / KV_SLOTS) & 1) &&
-                        (j < 1 || mbar_test(s_free(t), (j - 1) & 1))) {
-                        tc_fence_after();
-                        const uint32_t qa = sb + Q_OFF + t * Q_TILE;
-                        const uint32_t kb = sb + K_OFF + (j % KV_SLOTS) * SLOT_BYTES;
-                        // S = Q K^T, M128 N128, 8 k-steps of 16 dims (4 per half)
-                        for (int k = 0; k < 8; ++k) {
-                            const uint32_t off = (k & 3) * 32;
-                            const uint64_t a = smem_desc(qa + (k >> 2) * M * 128 + off, 16, 1024);
-                            const uint64_t bd = smem_desc(kb + (k >> 2) * KV_HALF + off, 16, 1024);
-                            umma_f16(tmem + t * TS, a, bd, idS, k > 0 ? 1u : 0u);
-                        }
-                        umma_commit(s_full(t));
-                        if (t == NT - 1) umma_commit(kempty(j % KV_SLOTS));  // K of stage j consumed
-                        ++ns[t];
-                        prog = true;
-                    }
+                umma_commit(s_full(t));
+                if (t == NT - 1) umma_commit(kempty(j % KV_SLOTS));  // K of stage j consumed
+            };
+            // P V_t(j): O_t += P V over 8 k-steps of 16 tokens.  P: fp16 pairs in
+            // the first 64 columns of S_t.  V is MN-major (dims contiguous):
+            // 64-dim groups KV_HALF apart, 8-token groups 1 KB apart.  Its
+            // completion frees S_t for the tile's next S.
+            auto issue_PV = [&](int t, int j) {
+                tc_fence_after();
+                const uint32_t vb = sb + V_OFF + (j % KV_SLOTS) * SLOT_BYTES;
+                for (int k = 0; k < 8; ++k) {
+                    const uint64_t bd = smem_desc(vb + k * 16 * 128, KV_HALF, 1024);
+                    umma_f16_ts(tmem + O_COL + t * D, tmem + t * TS + k * 8, bd, idO,
+                                (j > 0 || k > 0) ? 1u : 0u);
                 }
-                if (prog) {
-                    idle.reset();
-                } else {
-                    if (*reinterpret_cast<volatile int*>(&abort_flag) || idle.expired()) ok = false;
+                umma_commit(s_free(t));
+                if (t == NT - 1) umma_commit(vempty(j % KV_SLOTS));  // V of stage j consumed
+            };
+            // The softmax tiles take their exp turns in order, so the work
+            // becomes ready in one fixed order: S_0(0), S_1(0), then per stage
+            // j: P V_0(j), S_0(j+1), P V_1(j), S_1(j+1).  Issuing in that order
+            // with blocking waits wakes on each barrier as it completes; while
+            // one tile is in its softmax, the other's MMAs keep the tensor
+            // pipe busy.
+            if (ok && nst > 0) ok = mbar_wait_bounded(kfull(0), 0, kWait);
+            if (ok && nst > 0) {
+                for (int t = 0; t < NT; ++t) issue_S(t, 0);
+            }
+            for (int j = 0; j < nst && ok; ++j) {
+                for (int t = 0; t < NT && ok; ++t) {
+                    ok = mbar_wait_bounded(p_full(t), j & 1, kWait) &&
+                         mbar_wait_bounded(vfull(j % KV_SLOTS), (j / KV_SLOTS) & 1, kWait);
+                    if (!ok) break;
+                    issue_PV(t, j);
+                    if (j + 1 < nst) {
+                        ok = mbar_wait_bounded(kfull((j + 1) % KV_SLOTS), ((j + 1) / KV_SLOTS) & 1, kWait) &&
+                             mbar_wait_bounded(s_free(t), j & 1, kWait);
+                        if (!ok) break;
+                        issue_S(t, j + 1);
+                    }
                 }
             }
             if (!ok) {
