@@ -23,7 +23,9 @@
 //  * One producer warp streams K and V tiles with 2-D TMA (128-byte swizzle)
 //    into a ring of shared-memory stages (mbarrier complete_tx), plus the
 //    query rows with a 1-D bulk copy at each segment start.  Consumer warps
-//    take 16 tokens each per 64-token stage.
+//    take 16 tokens each of a stage: 8 warps per 128-token stage on the FMA
+//    path (twice the loads in flight for its latency-bound matrix-vector
+//    work), 4 warps per 64-token stage on the tensor-core paths.
 //  * When the rows sharing a KV head (GQA group x window) make the products a
 //    dense contraction (rows > 1), q K^T and P V run on tensor cores
 //    (mma.sync m16n8k16, fp16 in, fp32 accumulate), fed by conflict-free
@@ -46,8 +48,6 @@
 
 namespace pkv {
 
-constexpr int kTS = 64;                     // tokens per pipeline stage
-constexpr int kTokWarps = 4;                // consumer warps along the tokens of a stage
 constexpr int kMaxMT = 2;                   // m16 tiles of rows per KV head (rows <= 32)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kSmemBudget = 225 * 1024;
@@ -82,9 +82,16 @@ struct Cfg {
     static constexpr bool KQ = KQ_;  // K pool of int8 codes with per-channel scales
     static_assert(!KQ || D == 128, "int8 K pools are served at head_dim 128");
     static constexpr int NH = D / 64;                       // 64-column halves per row
-    static constexpr int NBS = kTS / BS;                    // blocks per stage
+    // consumer warps along the tokens of a stage (16 tokens each) and tokens
+    // per stage: the FMA consumers run latency-bound matrix-vector work and
+    // gain from twice the warps; the tensor-core consumers keep 4 (with 9
+    // warps their register cap would drop to 168 and the merge at each
+    // segment end would take twice the rounds)
+    static constexpr int TW = FMA ? 8 : 4;
+    static constexpr int TS = 16 * TW;                      // tokens per pipeline stage
+    static constexpr int NBS = TS / BS;                     // blocks per stage
     static constexpr int RP = FMA ? 1 : 16 * MT;            // padded rows
-    static constexpr int NCW = kTokWarps;                   // consumer warps
+    static constexpr int NCW = TW;                          // consumer warps
     static constexpr int THREADS = (NCW + 1) * 32;
     // registers per thread for one CTA per SM: warps are spread over the 4
     // SM sub-partitions, each with a 16K-register file
@@ -92,9 +99,9 @@ struct Cfg {
     static constexpr int MAXREG_RAW = (16384 / (32 * WARPS_PER_SUBPART)) / 8 * 8;
     static constexpr int MAXREG = MAXREG_RAW > 255 ? 255 : MAXREG_RAW;
     static constexpr int TILE_BYTES = BS * D * 2;           // one (block, kv-head) fp16 tile
-    static constexpr int KV_BYTES = kTS * D * 2;            // fp16 K (or V) bytes per stage
+    static constexpr int KV_BYTES = TS * D * 2;             // fp16 K (or V) bytes per stage
     static constexpr int K_TILE_BYTES = KQ ? BS * D : TILE_BYTES;
-    static constexpr int K_BYTES = KQ ? kTS * D : KV_BYTES;
+    static constexpr int K_BYTES = KQ ? TS * D : KV_BYTES;
     static constexpr int V_OFF = K_BYTES;                   // stage: K, V, query rows
     // query rows of a segment, one per 16-byte-padded row (conflict-free ldmatrix)
     static constexpr int QROW = D * 2 + 16;
@@ -104,7 +111,7 @@ struct Cfg {
     static constexpr int OB_STRIDE = D + 8;                 // floats per obuf row
     static constexpr int OBUF_SLICE = RP * OB_STRIDE;               // floats
     static constexpr int OBUF_BYTES = 2 * OBUF_SLICE * 4;           // two merge slices
-    static constexpr int ML_BYTES = kTokWarps * RP * 2 * 4;
+    static constexpr int ML_BYTES = TW * RP * 2 * 4;
     static constexpr int QP_BYTES = MT > 1 ? RP * QROW : 0;   // CTA copy of the query rows
     static constexpr int FIXED = OBUF_BYTES + ML_BYTES + QP_BYTES + 256 + 16 * 64;
     static constexpr int STAGES_RAW = (kSmemBudget - FIXED) / STAGE_BYTES;
@@ -114,7 +121,7 @@ struct Cfg {
     static constexpr int BAR_OFF = META_OFF + STAGES * 32;  // full[S], empty[S]
     static constexpr int ZERO_OFF = BAR_OFF + STAGES * 16;  // 128 zero bytes
     static constexpr int PB_OFF = ZERO_OFF + 128;           // per-warp fp16 weights (FMA path)
-    static constexpr int ML_OFF = PB_OFF + 128;
+    static constexpr int ML_OFF = PB_OFF + TW * 32;
     static constexpr int OBUF_OFF = ML_OFF + ML_BYTES;
     static constexpr int QP_OFF = OBUF_OFF + OBUF_BYTES;
     static constexpr int SMEM_USED = QP_OFF + QP_BYTES;
@@ -618,11 +625,11 @@ __device__ void store_segment(const Params& p, const StageMeta& md, const float*
         for (int R = tid; R < rows; R += C::NCW * 32) {
             float M = kNegInf;
 #pragma unroll
-            for (int w = 0; w < kTokWarps; ++w) M = fmaxf(M, mlb[(w * C::RP + R) * 2]);
+            for (int w = 0; w < C::TW; ++w) M = fmaxf(M, mlb[(w * C::RP + R) * 2]);
             const float Mu = M == kNegInf ? 0.f : M;
             float Ls = 0.f;
 #pragma unroll
-            for (int w = 0; w < kTokWarps; ++w)
+            for (int w = 0; w < C::TW; ++w)
                 Ls += mlb[(w * C::RP + R) * 2 + 1] * ex2(mlb[(w * C::RP + R) * 2] - Mu);
             p.part_lse[pbase + R] = Ls > 0.f ? Mu + lg2(Ls) : kNegInf;
         }
@@ -636,11 +643,11 @@ __device__ __forceinline__ float row_factor(const float* mlb, int R, float m_w)
 {
     float M = kNegInf;
 #pragma unroll
-    for (int w = 0; w < kTokWarps; ++w) M = fmaxf(M, mlb[(w * C::RP + R) * 2]);
+    for (int w = 0; w < C::TW; ++w) M = fmaxf(M, mlb[(w * C::RP + R) * 2]);
     const float Mu = M == kNegInf ? 0.f : M;
     float Ls = 0.f;
 #pragma unroll
-    for (int w = 0; w < kTokWarps; ++w)
+    for (int w = 0; w < C::TW; ++w)
         Ls += mlb[(w * C::RP + R) * 2 + 1] * ex2(mlb[(w * C::RP + R) * 2] - Mu);
     return Ls > 0.f ? ex2(m_w - Mu) / Ls : 0.f;
 }
@@ -652,7 +659,7 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
 {
     const int cw = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int mt = cw / kTokWarps, qw = cw % kTokWarps;
+    const int mt = cw / C::TW, qw = cw % C::TW;
     const int gid = lane >> 2, tig = lane & 3;
     const uint32_t sbase = smem_u32(smem);
     const StageMeta* smeta = reinterpret_cast<const StageMeta*>(smem + C::META_OFF);
@@ -828,12 +835,12 @@ __device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort
             float f[2];
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) f[rr] = row_factor<C>(mlb, mt * 16 + gid + rr * 8, m[rr]);
-            // token-warps 0 and 1 write slices 0 and 1, then 2 and 3 add to them
+            // token-warps 0 and 1 write slices 0 and 1, then each later pair adds to them
             const bool row0 = mt * 16 + gid < p.rows, row1 = mt * 16 + gid + 8 < p.rows;
             float* slice = obuf + (qw & 1) * C::OBUF_SLICE;
             float* r0p = slice + (mt * 16 + gid) * C::OB_STRIDE + tig * 2;
             float* r1p = r0p + 8 * C::OB_STRIDE;
-            for (int round = 0; round < 2; ++round) {
+            for (int round = 0; round < C::TW / 2; ++round) {
                 if ((qw >> 1) == round) {
                     // round 1 adds to round 0's values: read them all first so the
                     // loads pipeline instead of waiting behind each store
@@ -1055,7 +1062,7 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
             named_bar_sync(1, C::NCW * 32);
             const float f = row_factor<C>(mlb, 0, m);
             float* slice = obuf + (qw & 1) * C::OBUF_SLICE;
-            for (int round = 0; round < 2; ++round) {  // fixed order: deterministic sums
+            for (int round = 0; round < C::TW / 2; ++round) {  // fixed order: deterministic sums
                 if ((qw >> 1) == round) {
 #pragma unroll
                     for (int i = 0; i < DPT; ++i)
@@ -1075,7 +1082,7 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
 
 // ---------------------------------------------------------------------------
 // Tensor-core consumer for more than 16 rows per KV head (verify windows):
-// each of the four token warps covers every m16 row tile for its 16 tokens,
+// each of the token warps covers every m16 row tile for its 16 tokens,
 // so K and V fragments are loaded once and reused by all row tiles.  The
 // query fragments are re-read each stage (conflict-free ldmatrix) from a
 // per-CTA copy of the segment's query rows, which keeps registers for the
@@ -1289,7 +1296,7 @@ __device__ void consumer_mma_mt(const Params& p, uint8_t* smem, volatile int* ab
                 }
             named_bar_sync(1, C::NCW * 32);
             float* slice = obuf + (qw & 1) * C::OBUF_SLICE;
-            for (int round = 0; round < 2; ++round) {
+            for (int round = 0; round < C::TW / 2; ++round) {
                 if ((qw >> 1) == round) {
 #pragma unroll
                     for (int t = 0; t < MT; ++t) {
