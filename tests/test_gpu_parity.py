@@ -179,14 +179,15 @@ def test_forced_splits_full_compare(Hq, Hkv, D, bs, q_len, grid, min_split):
 
 @pytest.mark.parametrize("seg_cost", [-1, 1, 4, 13])
 @pytest.mark.parametrize("grid", [0, 61])
-def test_segment_cost_partition(seg_cost, grid):
+@pytest.mark.parametrize("Hq,Hkv", [(16, 4), (8, 8)])  # tensor-core path, FMA path
+def test_segment_cost_partition(seg_cost, grid, Hq, Hkv):
     """Many short sequences: CTA runs that start or end inside a segment's
     virtual cost units, splits and merges all give the oracle's result."""
     rng = np.random.Generator(np.random.PCG64(17))
-    lens = rng.integers(1, 120, size=40).astype(np.int32)
-    wl = make_workload("llama70b_gqa", "cuda", lens=lens, seed=19, Hq=16, Hkv=4, D=128)
+    lens = rng.integers(1, 300, size=40).astype(np.int32)
+    wl = make_workload("llama70b_gqa", "cuda", lens=lens, seed=19, Hq=Hq, Hkv=Hkv, D=128)
     out = _run(wl, 1, grid_ctas=grid, min_split_blocks=1, seg_cost_blocks=seg_cost)
-    assert_close(out, oracle_subset(wl, list(range(wl.B))), f"seg_cost {seg_cost} grid {grid}")
+    assert_close(out, oracle_subset(wl, list(range(wl.B))), f"Hq{Hq} Hkv{Hkv} seg_cost {seg_cost} grid {grid}")
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,maxlen,grid", [
