@@ -120,6 +120,7 @@ int block_free(kv_pool* pool, const int32_t* ids, int32_t n)
             return kv_fail(KV_ERR_DOUBLE_FREE, "block_free: reference count would go below zero");
     for (int32_t i = 0; i < n; ++i) {
         if (--pool->refcount[ids[i]] == 0) pool->free_stack.push_back(ids[i]);
+        kv_cache_recheck(pool, ids[i]);
     }
     return KV_OK;
 }
@@ -130,7 +131,10 @@ int block_fork(kv_pool* pool, const int32_t* ids, int32_t n)
     for (int32_t i = 0; i < n; ++i)
         if (ids[i] < 0 || ids[i] >= pool->cfg.num_blocks || pool->refcount[ids[i]] == 0)
             return kv_fail(KV_ERR_INVALID, "block_fork: id is not a live block");
-    for (int32_t i = 0; i < n; ++i) ++pool->refcount[ids[i]];
+    for (int32_t i = 0; i < n; ++i) {
+        ++pool->refcount[ids[i]];
+        kv_cache_recheck(pool, ids[i]);
+    }
     return KV_OK;
 }
 
@@ -173,6 +177,7 @@ int kv_seq_reserve_slot(kv_pool* pool, int32_t* table, int32_t table_capacity, i
         int rc = alloc_ids(pool, 1, &id);
         if (rc != KV_OK) return rc;
         --pool->refcount[last];
+        kv_cache_recheck(pool, last);
         table[nb - 1] = id;
         *cow_src_out = last;
         *cow_dst_out = id;
@@ -244,7 +249,10 @@ extern "C" int kv_beam_reorder(kv_pool* pool, const int32_t* tables, const int32
         for (int32_t k = 0; k < table_capacity; ++k) {
             const int32_t id = k < nb ? tables[p * cap + k] : -1;
             new_tables[i * cap + k] = id;
-            if (id >= 0) ++pool->refcount[id];
+            if (id >= 0) {
+                ++pool->refcount[id];
+                kv_cache_recheck(pool, id);
+            }
         }
         new_n_blocks[i] = nb;
     }
@@ -252,6 +260,7 @@ extern "C" int kv_beam_reorder(kv_pool* pool, const int32_t* tables, const int32
         for (int32_t k = 0; k < n_blocks[b]; ++k) {
             const int32_t id = tables[b * cap + k];
             if (--pool->refcount[id] == 0) pool->free_stack.push_back(id);
+            kv_cache_recheck(pool, id);
         }
     return KV_OK;
 }

@@ -25,6 +25,13 @@ struct kv_pool {
     std::vector<int32_t> key_tokens;
     std::unordered_multimap<uint64_t, int32_t> by_hash;  // key hash -> block
     std::set<std::pair<uint64_t, int32_t>> lru;         // (last use, block), cached blocks
+    // (last use, block) of exactly the cached blocks that eviction may take:
+    // no cached children and no reference but the cache's own
+    std::set<std::pair<uint64_t, int32_t>> evictable;
     uint64_t clock = 0;
     int32_t n_cached = 0;
 };
+
+// Brings block b's membership of `evictable` up to date; called after any
+// change to its reference count (a no-op while nothing was ever cached).
+void kv_cache_recheck(kv_pool* p, int32_t b);

@@ -72,15 +72,20 @@ int32_t find(const kv_pool* p, uint64_t h, int32_t parent, const int32_t* tokens
 // Mark a block (cached, or about to be) as the most recently used.
 void use(kv_pool* p, int32_t b)
 {
-    if (p->cached[b]) p->lru.erase({p->last_use[b], b});
+    if (p->cached[b]) {
+        p->lru.erase({p->last_use[b], b});
+        p->evictable.erase({p->last_use[b], b});
+    }
     p->last_use[b] = ++p->clock;
     p->lru.insert({p->last_use[b], b});
+    kv_cache_recheck(p, b);
 }
 
 void uncache(kv_pool* p, int32_t b)
 {
     const int32_t bs = p->cfg.block_size;
     p->lru.erase({p->last_use[b], b});
+    p->evictable.erase({p->last_use[b], b});
     const uint64_t h = key_hash(p->parent[b], &p->key_tokens[static_cast<size_t>(b) * bs], bs);
     const auto range = p->by_hash.equal_range(h);
     for (auto it = range.first; it != range.second; ++it)
@@ -88,13 +93,25 @@ void uncache(kv_pool* p, int32_t b)
             p->by_hash.erase(it);
             break;
         }
-    if (p->parent[b] >= 0) --p->children[p->parent[b]];
+    const int32_t up = p->parent[b];
+    if (up >= 0) --p->children[up];
     p->cached[b] = 0;
     p->parent[b] = -1;
     --p->n_cached;
+    if (up >= 0) kv_cache_recheck(p, up);  // it may have become a leaf
 }
 
 }  // namespace
+
+void kv_cache_recheck(kv_pool* p, int32_t b)
+{
+    if (p->cached.empty() || b < 0) return;
+    const std::pair<uint64_t, int32_t> k{p->last_use[b], b};
+    if (p->cached[b] && p->children[b] == 0 && p->refcount[b] == 1)
+        p->evictable.insert(k);
+    else
+        p->evictable.erase(k);
+}
 
 extern "C" {
 
@@ -149,6 +166,8 @@ int kv_prefix_register(kv_pool* pool, const int32_t* tokens, int32_t n_tokens, c
             use(pool, b);
             pool->cached[b] = 1;
             ++pool->n_cached;
+            kv_cache_recheck(pool, b);
+            if (parent >= 0) kv_cache_recheck(pool, parent);  // no longer a leaf
         } else if (have == b) {
             use(pool, b);
         } else {
@@ -167,16 +186,10 @@ int kv_prefix_evict(kv_pool* pool, int32_t n, int32_t* ids_out, int32_t* n_evict
     *n_evicted_out = 0;
     if (pool->cached.empty()) return KV_OK;
     int32_t k = 0;
-    while (k < n) {
-        int32_t victim = -1;
-        for (const auto& e : pool->lru) {
-            const int32_t b = e.second;
-            if (pool->children[b] == 0 && pool->refcount[b] == 1) {
-                victim = b;
-                break;
-            }
-        }
-        if (victim < 0) break;
+    // the least recently used unreferenced leaf, each time: freeing a leaf
+    // can make its parent one
+    while (k < n && !pool->evictable.empty()) {
+        const int32_t victim = pool->evictable.begin()->second;
         uncache(pool, victim);
         pool->refcount[victim] = 0;
         pool->free_stack.push_back(victim);

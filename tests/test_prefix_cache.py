@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 
 from conftest import read_golden
-from oracle.block_spec import OK, BlockPoolSpec, PrefixCacheSpec
+from oracle.block_spec import OK, BlockPoolSpec, PrefixCacheSpec, beam_reorder
 
 import paged_kv_cache_371_b200 as pkv
 
@@ -225,6 +225,106 @@ def test_cpp_prefix_cache_matches_spec(seed, bs):
     for tokens, table in live:
         spool.free(table)
         impl.free(table)
+    assert impl.prefix_evict(nb) == scache.evict(nb)[1]
+    assert impl.num_free() == nb and impl.num_cached() == 0
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_cpp_eviction_tracks_forks_appends_and_beams(seed):
+    """Cached blocks whose references also move through forks, appends
+    (copy-on-write) and beam steps: the C++ cache evicts exactly the blocks
+    the spec does, in the same order, with the same reference counts."""
+    rng = np.random.Generator(np.random.PCG64(300 + seed))
+    nb, bs = 128, 8
+    order = rng.permutation(nb)
+    spool = BlockPoolSpec(nb, bs, order)
+    scache = PrefixCacheSpec(spool)
+    impl = pkv.KVPool(nb, bs, order=order)
+    systems = [list(rng.integers(0, 40, size=int(rng.integers(2, 6)) * bs)) for _ in range(3)]
+    live = []   # [tokens, table]: the same ids on both sides
+    extra = []  # references taken directly on cached blocks (no request)
+    n_evicted = 0
+    for step in range(1200):
+        op = int(rng.integers(0, 13))
+        if op <= 3 or not live:
+            sysp = systems[int(rng.integers(len(systems)))]
+            cut = int(rng.integers(0, len(sysp) + 1))
+            tokens = [int(x) for x in sysp[:cut]] + [int(x) for x in rng.integers(0, 3, size=int(rng.integers(1, 2 * bs)))]
+            st, stab = scache.match(tokens)
+            assert impl.prefix_match(tokens) == stab
+            need = -(-len(tokens) // bs) - len(stab)
+            st2, ids = spool.alloc(need)
+            if st2 != OK:
+                spool.free(stab)
+                impl.free(stab)
+                continue
+            assert impl.alloc(need) == ids
+            live.append([tokens, stab + ids])
+        elif op <= 5:
+            tokens, table = live[int(rng.integers(len(live)))]
+            assert impl.prefix_register(tokens, table) == scache.register(tokens, table)[1]
+        elif op == 6:
+            tokens, table = live[int(rng.integers(len(live)))]
+            assert spool.fork(table) == OK
+            impl.fork(table)
+            live.append([list(tokens), list(table)])
+        elif op == 7:
+            tokens, table = live[int(rng.integers(len(live)))]
+            before = list(table)
+            st, slot, src, dst = spool.reserve_slot(table, len(tokens))
+            if st != OK:
+                continue
+            t = np.full(len(before) + 1, -1, np.int32)
+            t[:len(before)] = before
+            assert impl.reserve_slot(t, len(before), len(tokens)) == (slot, len(table), src, dst)
+            assert t[:len(table)].tolist() == table
+            tokens.append(int(rng.integers(0, 3)))
+        elif op == 8:
+            k = int(rng.integers(1, min(3, len(live)) + 1))
+            pick = sorted(rng.choice(len(live), size=k, replace=False).tolist())
+            group = [live[i] for i in pick]
+            parents = rng.integers(0, k, size=int(rng.integers(1, 4))).tolist()
+            st, new = beam_reorder(spool, [g[1] for g in group], parents)
+            assert st == OK
+            cap = max(len(g[1]) for g in group)
+            tabs = np.full((k, cap), -1, np.int32)
+            for i, g in enumerate(group):
+                tabs[i, :len(g[1])] = g[1]
+            got, got_nb = impl.beam_reorder(tabs, np.array([len(g[1]) for g in group], np.int32), parents)
+            assert [got[i, :got_nb[i]].tolist() for i in range(len(parents))] == new
+            for i in reversed(pick):
+                live.pop(i)
+            live.extend([list(group[p][0]), list(t)] for p, t in zip(parents, new))
+        elif op == 9:
+            tokens, table = live.pop(int(rng.integers(len(live))))
+            assert spool.free(table) == OK
+            impl.free(table)
+        elif op == 10:
+            k = int(rng.integers(0, 8))
+            got = impl.prefix_evict(k)
+            assert got == scache.evict(k)[1]
+            n_evicted += len(got)
+        elif op == 11 and scache.key_of:
+            # one more reference on cached blocks only the cache may hold
+            ids = sorted(rng.choice(sorted(scache.key_of), size=min(3, len(scache.key_of)), replace=False).tolist())
+            assert spool.fork(ids) == OK
+            impl.fork(ids)
+            extra.append(ids)
+        elif op == 12 and extra:
+            ids = extra.pop(int(rng.integers(len(extra))))
+            assert spool.free(ids) == OK
+            impl.free(ids)
+        assert impl.num_free() == spool.num_free()
+        assert impl.num_cached() == scache.num_cached()
+        if step % 25 == 0:
+            assert [impl.refcount(b) for b in range(nb)] == spool.refcount
+    assert n_evicted >= 10   # eviction really ran against forked and beamed references
+    for tokens, table in live:
+        spool.free(table)
+        impl.free(table)
+    for ids in extra:
+        spool.free(ids)
+        impl.free(ids)
     assert impl.prefix_evict(nb) == scache.evict(nb)[1]
     assert impl.num_free() == nb and impl.num_cached() == 0
 
