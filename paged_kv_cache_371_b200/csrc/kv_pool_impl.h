@@ -24,7 +24,6 @@ struct kv_pool {
     std::vector<uint64_t> last_use;
     std::vector<int32_t> key_tokens;
     std::unordered_multimap<uint64_t, int32_t> by_hash;  // key hash -> block
-    std::set<std::pair<uint64_t, int32_t>> lru;         // (last use, block), cached blocks
     // (last use, block) of exactly the cached blocks that eviction may take:
     // no cached children and no reference but the cache's own
     std::set<std::pair<uint64_t, int32_t>> evictable;

@@ -48,6 +48,7 @@ bool ensure_cache(kv_pool* p)
         p->children.assign(n, 0);
         p->last_use.assign(n, 0);
         p->key_tokens.assign(n * bs, 0);
+        p->by_hash.reserve(n);
     } catch (...) {
         p->cached.clear();
         return false;
@@ -72,19 +73,14 @@ int32_t find(const kv_pool* p, uint64_t h, int32_t parent, const int32_t* tokens
 // Mark a block (cached, or about to be) as the most recently used.
 void use(kv_pool* p, int32_t b)
 {
-    if (p->cached[b]) {
-        p->lru.erase({p->last_use[b], b});
-        p->evictable.erase({p->last_use[b], b});
-    }
+    if (p->cached[b]) p->evictable.erase({p->last_use[b], b});
     p->last_use[b] = ++p->clock;
-    p->lru.insert({p->last_use[b], b});
     kv_cache_recheck(p, b);
 }
 
 void uncache(kv_pool* p, int32_t b)
 {
     const int32_t bs = p->cfg.block_size;
-    p->lru.erase({p->last_use[b], b});
     p->evictable.erase({p->last_use[b], b});
     const uint64_t h = key_hash(p->parent[b], &p->key_tokens[static_cast<size_t>(b) * bs], bs);
     const auto range = p->by_hash.equal_range(h);
