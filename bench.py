@@ -5,8 +5,12 @@ One step = one decode step of one attention layer over a batch:
   copy-on-write block copies (when the step has any) -> cache append of one
   new token per sequence -> paged decode (or verify) attention over the
   grown contexts (+ the split-context merge).
-Host bookkeeping (slot reservation) for every step is done before timing;
-the e2e figure repeats the steps through the public API with host buffers.
+The device-timed steps replay slots and tables the host block manager
+reserved before timing; the e2e figure runs the whole step through the
+public API with host buffers, the host reservation (and, for beam search,
+the beam reorder) of every step inside its timed region.  The default run
+also times the Llama-2-70B-shaped GQA decode at block sizes 16 and 8
+(`targets` in the JSON line).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                        [--impl ours|reference]
@@ -49,6 +53,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-targets", action="store_true",
+                    help="skip the 70B GQA decode lines reported beside the default workload")
     ap.add_argument("--batch", type=int, default=0,
                     help="use only the first B sequences of the workload (profiling runs)")
     return ap.parse_args(argv)
@@ -294,12 +300,12 @@ def build_beam_steps(pkv, wl, n_steps, device, seed, width=BEAMS):
     from workloads import normal_fp16
     Hq, Hkv, D = wl.q.shape[-2], wl.spec.Hkv, wl.q.shape[-1]
     pool, tables, nblk = adopt_workload(pkv, wl, extra_cap=n_steps // wl.spec.bs + 3)
-    rng = np.random.Generator(np.random.PCG64(seed + 7))
     S = wl.B
-    parents = np.repeat(np.arange(S), width).astype(np.int32)
+    all_parents = beam_parents(S, width, n_steps, seed)
     beam_len = wl.lens.astype(np.int32)
     steps = []
     for i in range(n_steps):
+        parents = all_parents[i]
         tables, nblk = pool.beam_reorder(tables, nblk, parents)
         lens = beam_len[parents].astype(np.int32)
         slots, pairs = pool.reserve_slots(tables, nblk, lens)
@@ -316,8 +322,6 @@ def build_beam_steps(pkv, wl, n_steps, device, seed, width=BEAMS):
             "lens_host": beam_len.copy(),
             "tables_host": tables.copy(),
         })
-        parents = np.concatenate([g * width + rng.integers(0, width, size=width)
-                                  for g in range(S)]).astype(np.int32)
     return steps
 
 
@@ -345,6 +349,7 @@ def build_steps(pkv, wl, n_steps, device, seed):
             "tables": torch.as_tensor(tables.copy(), device=device),
             "lens": torch.as_tensor(lens.copy(), device=device),
             "lens_host": lens.copy(),
+            "tables_host": tables.copy(),
         }
         steps.append(st)
     return steps
@@ -374,7 +379,7 @@ def run_prefill(args):
     kn = normal_fp16((len(slots), Hkv, D), 901, device)
     vn = normal_fp16((len(slots), Hkv, D), 902, device)
     out = torch.empty_like(wl.q)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     stream = torch.cuda.current_stream(device)
 
     def step(ev=None):
@@ -392,7 +397,7 @@ def run_prefill(args):
     ee = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     with ClockSampler(local) as clk:
         for k in range(args.steps):
-            flush.zero_()
+            flush()
             es[k].record(stream)
             step(ea[k])
             ee[k].record(stream)
@@ -415,7 +420,7 @@ def run_prefill(args):
         h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hs))
         times = []
         for k in range(args.warmup + args.steps):
-            flush.zero_()
+            flush()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
@@ -442,7 +447,8 @@ def run_prefill(args):
                    "Hq": Hq, "Hkv": Hkv, "head_dim": D, "block_size": bs, "q_len": q_len,
                    "mean_context": float(np.mean(wl.lens)),
                    "step": "append the chunk's K/V + causal paged prefill attention",
-                   "l2": "flushed before every timed step (256 MB memset)"},
+                   "l2": f"flushed before every timed step by reading {flush.bytes >> 20} MiB "
+                         "(a sum into one word: no dirty lines left)"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "traffic": ncu_traffic(args.workload, "paged_prefill.cu"),
@@ -490,18 +496,65 @@ def prefill_cpu_baseline(wl, q_len, target_s):
         reps += 1
     fl = prefill_flops(lens, Hq, D, n_pos) * reps
     return {"value": round(fl / spent / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
+            "kind": "oracle", "cpu_model": cpu_model(),
             "sample": f"the first {n_pos} positions of sequence 0's chunk (all {Hq} heads, "
                       f"{int(lens[0])} tokens) x {reps} repeat(s), fp64 C oracle, {spent:.2f} s"}
 
 
-def run_ours(args):
+def beam_parents(S, width, n_steps, seed):
+    """The beams each step continues: step 0 forks every prompt into `width`
+    beams; later steps draw the survivors (seeded) within each prompt's beams
+    (the sampler's decision, made by the caller, not by the library)."""
     import numpy as np
+    rng = np.random.Generator(np.random.PCG64(seed + 7))
+    out = [np.repeat(np.arange(S), width).astype(np.int32)]
+    for _ in range(n_steps - 1):
+        out.append(np.concatenate([g * width + rng.integers(0, width, size=width)
+                                   for g in range(S)]).astype(np.int32))
+    return out
+
+
+class L2Flush:
+    """Evicts L2 between timed steps by READING a buffer of twice its size
+    into a one-word sum: no dirty lines are left behind for the next timed
+    step to write back."""
+
+    def __init__(self, device):
+        import torch
+        l2 = torch.cuda.get_device_properties(device).L2_cache_size
+        n = max(2 * l2, 256 << 20) // 4
+        self.buf = torch.zeros(n, dtype=torch.float32, device=device)
+        self.acc = torch.zeros((), dtype=torch.float32, device=device)
+        self.bytes = n * 4
+
+    def __call__(self):
+        import torch
+        torch.sum(self.buf, 0, out=self.acc)
+
+
+def unique_kv_bytes(tables, lens, bs, Hkv, D, k_bytes=2):
+    """K/V bytes of the distinct cache rows one launch reads: a block shared
+    by several sequences (a common prefix, beams) counts once, with the most
+    rows any of them reads from it."""
+    import numpy as np
+    rows = {}
+    for s in range(len(lens)):
+        L = int(lens[s])
+        n = -(-L // bs)
+        for b in range(n):
+            blk = int(tables[s, b])
+            used = min(bs, L - b * bs)
+            if rows.get(blk, 0) < used:
+                rows[blk] = used
+    return sum(rows.values()) * Hkv * D * (k_bytes + 2)
+
+
+TARGET_WORKLOADS = ("llama70b_gqa", "llama70b_gqa_bs8")
+
+
+def run_ours(args):
     import torch
     import torch.distributed as dist
-
-    import paged_kv_cache_371_b200 as pkv
-    from workloads import make_workload
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
@@ -509,14 +562,50 @@ def run_ours(args):
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    try:
+        result = measure_decode(args, args.workload, rank, world, local, device, full=True)
+        if args.workload == DEFAULT_WORKLOAD and not args.no_targets and not args.batch:
+            # the Llama-2-70B-shaped GQA decode at both block sizes, same
+            # steps and warm-up, reported beside the headline
+            targets = {}
+            for name in TARGET_WORKLOADS:
+                torch.cuda.empty_cache()
+                r = measure_decode(args, name, rank, world, local, device, full=False)
+                if rank == 0:
+                    targets[name] = {k: r[k] for k in ("value", "unit", "ms_per_step", "hbm_frac",
+                                                       "tokens_heads_per_s", "roofline", "clocks",
+                                                       "gpu_launches", "config")}
+            if rank == 0:
+                result["targets"] = targets
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    return result if rank == 0 else None
 
+
+def measure_decode(args, workload, rank, world, local, device, full=True):
+    """Device-timed decode steps of one workload (+ with `full`: the
+    end-to-end serving loop and, on one GPU, the oracle baseline)."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_371_b200 as pkv
+    from workloads import make_workload
     from workloads.synth import CONFIGS
-    base, q8k = split_workload(args.workload)
+
+    base, q8k = split_workload(workload)
     spec = CONFIGS[base]
     seed = rank_seed(spec.seed, rank)
     beams = base == "beam_search"
     n_distinct = min(args.warmup + args.steps, 64)
-    spare = (n_distinct // spec.bs + 3) * BEAMS * (args.batch or spec.B) * 2 if beams else 0
+    do_e2e = full and not args.no_e2e
+    n_host = args.warmup + args.steps if do_e2e else n_distinct  # steps the host pool must fit
+    B = args.batch or spec.B
+    if beams:
+        spare = (n_host // spec.bs + 3) * BEAMS * B * 2
+    else:
+        spare = (n_host // spec.bs + 2) * B
     wl = make_workload(base, device, seed=seed, B=args.batch or None, spare_blocks=spare)
     q_len = spec.q_len
     Hq, Hkv, D, bs = spec.Hq, spec.Hkv, spec.D, spec.bs
@@ -529,8 +618,7 @@ def run_ours(args):
     n_rows = steps[0]["q"].shape[0]  # sequences (beams) attended per step
     out = torch.empty((n_rows, q_len, Hq, D), dtype=torch.float16, device=device)
     ws = torch.empty(pkv.workspace_size(Hq, Hkv, q_len, D), dtype=torch.uint8, device=device)
-    l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     stream = torch.cuda.current_stream(device)
 
     def step(i, ev=None):
@@ -539,6 +627,7 @@ def run_ours(args):
                     st["lens"], st["pairs"], out, ws, q_len, kq, ksc, ev, stream)
 
     for i in range(args.warmup):
+        flush()
         step(i)
     torch.cuda.synchronize()
     assert pkv.device_error() == 0, "device error during warm-up"
@@ -558,7 +647,7 @@ def run_ours(args):
         for k in range(args.steps):
             i = args.warmup + k
             st = steps[i % n_distinct]
-            flush.zero_()
+            flush()
             ev_s[k].record(stream)
             step(i, ev_a[k])
             ev_e[k].record(stream)
@@ -580,47 +669,60 @@ def run_ours(args):
     kv_all, th_all, t_all = aggregate(kv_bytes_total, th_tokens, total_ms, world, device)
     value = kv_all / (t_all * 1e-3) / 1e9
 
-    # e2e: same steps through the public API with pinned host buffers
     e2e = None
-    if not args.no_e2e:
-        e2e = run_e2e(pkv, wl, steps, n_distinct, args, out, ws, flush, stream, device, Hq, Hkv, D,
-                      bs, q_len, world, kq, ksc)
+    if do_e2e:
+        e2e = run_e2e(pkv, wl, steps, n_distinct, args, ws, stream, device, Hq, Hkv, D, bs, q_len,
+                      world, kq, ksc, beams, seed)
 
     peak, peak_kind = measured_hbm_peak()
     attn_avg_ms = statistics.mean(attn_ms)
     achieved = statistics.mean(alg_attn) / (attn_avg_ms * 1e-3) / 1e9
     result = None
     if rank == 0:
+        st_last = steps[-1]
+        tables_last = st_last["tables_host"]
+        shared = base in ("prefix_beam", "beam_search")
         result = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(t_all / args.steps, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
             "config": {
-                "workload": args.workload + (f"[B={wl.B}]" if args.batch else ""),
+                "workload": workload + (f"[B={wl.B}]" if args.batch else ""),
                 "description": spec.description, "B": n_rows,
                 "Hq": Hq, "Hkv": Hkv, "head_dim": D, "block_size": bs, "q_len": q_len,
-                "mean_context": float(np.mean(steps[-1]["lens_host"])),
+                "mean_context": float(np.mean(st_last["lens_host"])),
                 "cow_copies_per_step": round(n_cow / args.steps, 2),
                 "step": "copy-on-write copies + append 1 token/sequence + paged attention + merge",
                 "k_pool": ("int8 codes, fp32 scale per (KV head, channel); V fp16" if q8k
                            else "fp16"),
-                "l2": "flushed before every timed step (memset of 2x L2)",
+                "l2": f"flushed before every timed step by reading {flush.bytes >> 20} MiB "
+                      "(a sum into one word: no dirty lines left)",
                 "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "hbm_frac": round(value / peak, 4),
             "hbm_peak_gbs": peak, "hbm_peak_kind": peak_kind,
             "tokens_heads_per_s": round(th_all / (t_all * 1e-3), 1),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "traffic": ncu_traffic(args.workload),
+                         "traffic": ncu_traffic(workload),
                          "kernel": "paged_attention_kernel + lse_merge_kernel",
+                         "attention_ms": round(attn_avg_ms, 5),
                          "peak_kind": peak_kind},
             "gpu_launches": launches,
             "clocks": clk.summary(),
         }
+        if shared:
+            # the same launch counted in distinct cache rows (shared blocks once)
+            ub = unique_kv_bytes(tables_last, st_last["lens_host"], bs, Hkv, D, k_bytes)
+            lb = algorithmic_bytes(st_last["lens_host"], Hq, Hkv, D, bs, q_len, k_bytes)[0]
+            u_gbs = ub / (attn_avg_ms * 1e-3) / 1e9
+            result["roofline"]["unique_kv_bytes"] = ub
+            result["roofline"]["logical_kv_bytes"] = lb
+            result["roofline"]["unique_gbs"] = round(u_gbs, 2)
+            result["roofline"]["unique_frac"] = round(u_gbs / peak, 4)
         if e2e:
             result["e2e"] = e2e
-        if world == 1 and args.cpu_seconds > 0:
+        if full and world == 1 and args.cpu_seconds > 0:
             # the timed appends only wrote slots past each sequence's original
             # length, so the workload's original tokens are still in the pools
             if beams:  # the oracle over the beams of the last step
@@ -628,8 +730,7 @@ def run_ours(args):
                 wl.lens = steps[-1]["lens_host"]
                 wl.q = steps[-1]["q"]
             result["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, q8k)
-    if world > 1:
-        dist.destroy_process_group()
+    del steps, wl, kq, ksc, out, ws, flush
     return result
 
 
@@ -658,58 +759,102 @@ def decode_step(pkv, wl, q, k_new, v_new, slots, tables, lens, pairs, out, ws, q
                                    workspace=ws)
 
 
-def run_e2e(pkv, wl, steps, n_distinct, args, out, ws, flush, stream, device, Hq, Hkv, D, bs, q_len,
-            world, kq=None, ksc=None):
-    """Decode steps through the public API with host buffers, pipelined the
-    way a serving loop runs: step k+1's inputs go host -> device on one
-    stream and step k's output device -> host on another while step k
-    computes (double-buffered inputs and outputs).  Every step's copies are
-    inside the timed region (first input copy to last output copy).  No L2
+def run_e2e(pkv, wl, steps, n_distinct, args, ws, stream, device, Hq, Hkv, D, bs, q_len, world,
+            kq=None, ksc=None, beams=False, seed=0):
+    """The whole decode step through the public API with host buffers, run
+    the way a serving loop runs it.  Every step, inside the timed region:
+    the host block manager reserves one slot per sequence (for beam search,
+    after reordering the beams' tables), emitting copy-on-write pairs; the
+    slots, pairs, tables, lengths and the step's q / K / V go host -> device
+    from pinned memory; copy-on-write copies, append, attention and merge run;
+    the output comes back device -> host.  Step k+1's host work and input
+    copies overlap step k's kernels (double-buffered inputs and outputs, two
+    side streams).  The host pool starts from the workload's placement, so
+    the first steps reserve the slots the device-timed steps used.  No L2
     flush: each step reads far more K/V than the 126 MB L2."""
+    import numpy as np
     import torch
     import torch.distributed as dist
-    names = ("q", "k_new", "v_new", "slots", "lens", "tables")
-    host = []
-    for st in steps:
-        h = {k: st[k].cpu().pin_memory() for k in names}
-        h["pairs"] = st["pairs"].cpu().pin_memory() if st["pairs"] is not None else None
-        host.append(h)
-    max_pairs = max((h["pairs"].shape[0] for h in host if h["pairs"] is not None), default=0)
-    bufs = []
+    n_total = args.warmup + args.steps
+    pool, tables, nblk = adopt_workload(pkv, wl, extra_cap=n_total // bs + 3)
+    lens = wl.lens.astype(np.int32).copy()
+    parents = beam_parents(wl.B, BEAMS, n_total, seed) if beams else None
+    n = steps[0]["q"].shape[0]
+    cap = tables.shape[1]
+    # per-step q / K / V in pinned host memory (the model's outputs of the step)
+    host_qkv = [{k: st[k].cpu().pin_memory() for k in ("q", "k_new", "v_new")} for st in steps]
+    names = ("slots", "pairs", "tables", "lens")
+    stage = [{"slots": torch.empty(n, dtype=torch.int64).pin_memory(),
+              "pairs": torch.empty((n, 2), dtype=torch.int32).pin_memory(),
+              "tables": torch.empty((n, cap), dtype=torch.int32).pin_memory(),
+              "lens": torch.empty(n, dtype=torch.int32).pin_memory()} for _ in range(2)]
+    dbuf = []
     for _ in range(2):
-        d = {k: torch.empty_like(steps[0][k]) for k in names}
-        d["pairs"] = torch.empty((max(max_pairs, 1), 2), dtype=torch.int32, device=device)
-        bufs.append(d)
-    outs = [out, torch.empty_like(out)]
-    houts = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+        d = {k: torch.empty_like(steps[0][k]) for k in ("q", "k_new", "v_new")}
+        d.update({k: torch.empty(v.shape, dtype=v.dtype, device=device)
+                  for k, v in stage[0].items()})
+        dbuf.append(d)
+    out0 = torch.empty((n, q_len, Hq, D), dtype=torch.float16, device=device)
+    outs = [out0, torch.empty_like(out0)]
+    houts = [torch.empty(out0.shape, dtype=out0.dtype).pin_memory() for _ in range(2)]
     s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_done = [torch.cuda.Event() for _ in range(2)]
     ev_read = [torch.cuda.Event() for _ in range(2)]
+    state = {"tables": tables, "nblk": nblk, "lens": lens, "beam_len": lens.copy()}
 
-    def run(k0, n):
+    def host_step(k, b):
+        """Host bookkeeping of step k into staging buffer b; returns (pairs,
+        bytes copied host -> device this step)."""
+        if beams:
+            state["tables"], state["nblk"] = pool.beam_reorder(state["tables"], state["nblk"],
+                                                               parents[k])
+            cur = state["beam_len"][parents[k]].astype(np.int32)
+        else:
+            cur = state["lens"]
+        slots, pairs = pool.reserve_slots(state["tables"], state["nblk"], cur)
+        cur = cur + 1
+        if beams:
+            state["beam_len"] = cur
+        else:
+            state["lens"] = cur
+        if k >= 2:
+            ev_in[b].synchronize()  # step k-2's copies out of staging b are done
+        sg = stage[b]
+        sg["slots"].numpy()[:] = slots
+        sg["tables"].numpy()[:] = state["tables"]
+        sg["lens"].numpy()[:] = cur
+        npairs = len(pairs)
+        if npairs:
+            sg["pairs"].numpy()[:npairs] = pairs
+        return npairs
+
+    def run(k0, cnt):
         nbytes = 0
-        for k in range(k0, k0 + n):
+        for k in range(k0, k0 + cnt):
             b = k % 2
-            h, d = host[k % n_distinct], bufs[b]
+            npairs = host_step(k, b)
+            h, sg, d = host_qkv[k % n_distinct], stage[b], dbuf[b]
             if k - k0 >= 2:
                 s_in.wait_event(ev_done[b])      # step k-2 finished reading buffer b
             with torch.cuda.stream(s_in):
                 nbytes = 0
-                for name in names:
-                    d[name].copy_(h[name], non_blocking=True)
-                    nbytes += h[name].numel() * h[name].element_size()
+                for name, src in (("q", h["q"]), ("k_new", h["k_new"]), ("v_new", h["v_new"]),
+                                  ("slots", sg["slots"]), ("tables", sg["tables"]),
+                                  ("lens", sg["lens"])):
+                    d[name].copy_(src, non_blocking=True)
+                    nbytes += src.numel() * src.element_size()
                 pairs = None
-                if h["pairs"] is not None:
-                    pairs = d["pairs"][:h["pairs"].shape[0]]
-                    pairs.copy_(h["pairs"], non_blocking=True)
-                    nbytes += h["pairs"].numel() * 4
+                if npairs:
+                    pairs = d["pairs"][:npairs]
+                    pairs.copy_(sg["pairs"][:npairs], non_blocking=True)
+                    nbytes += npairs * 8
                 ev_in[b].record(s_in)
             stream.wait_event(ev_in[b])
             if k - k0 >= 2:
                 stream.wait_event(ev_read[b])    # step k-2's output was copied out
-            decode_step(pkv, wl, d["q"], d["k_new"], d["v_new"], d["slots"], d["tables"], d["lens"],
-                        pairs, outs[b], ws, q_len, kq, ksc)
+            decode_step(pkv, wl, d["q"], d["k_new"], d["v_new"], d["slots"], d["tables"],
+                        d["lens"], pairs, outs[b], ws, q_len, kq, ksc)
             ev_done[b].record(stream)
             s_out.wait_event(ev_done[b])
             with torch.cuda.stream(s_out):
@@ -721,6 +866,7 @@ def run_e2e(pkv, wl, steps, n_distinct, args, out, ws, flush, stream, device, Hq
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    lens_at_start = (state["beam_len"] if beams else state["lens"]).copy()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(s_in)
@@ -728,19 +874,25 @@ def run_e2e(pkv, wl, steps, n_distinct, args, out, ws, flush, stream, device, Hq
     s_out.wait_stream(stream)
     e1.record(s_out)
     torch.cuda.synchronize()
-    kvb_total = sum(algorithmic_bytes(steps[k % n_distinct]["lens_host"], Hq, Hkv, D, bs, q_len,
-                                      1 if kq is not None else 2)[0]
-                    for k in range(args.warmup, args.warmup + args.steps))
+    assert pkv.device_error() == 0, "device error in the end-to-end loop"
+    # K/V bytes attended: every sequence grows by one token per step
+    L0 = lens_at_start.astype(np.int64)
+    kvb_total = sum(algorithmic_bytes(L0 + 1 + k, Hq, Hkv, D, bs, q_len, 1 if kq is not None else 2)[0]
+                    for k in range(args.steps))
     t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
     kv = torch.tensor([float(kvb_total)], dtype=torch.float64, device=device)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         dist.all_reduce(kv, op=dist.ReduceOp.SUM)
+    pool.close()
     return {"value": round(kv.item() / (t.item() * 1e-3) / 1e9, 2), "unit": "GB/s",
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(out.numel() * out.element_size()),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(out0.numel() * 2),
             "ms_per_step": round(t.item() / args.steps, 5),
-            "pipelining": "inputs of step k+1 and output of step k copied on two streams while "
-                          "step k computes (double buffers); L2 not flushed (K/V per step >> L2)"}
+            "host_work": ("kv_beam_reorder + " if beams else "") +
+                         "kv_batch_reserve_slots every step, inside the timed region",
+            "pipelining": "host bookkeeping and input copies of step k+1, and the output copy of "
+                          "step k, overlap step k's kernels (double buffers, two side streams); "
+                          "L2 not flushed (K/V per step >> L2)"}
 
 
 # ---------------------------------------------------------------------------
@@ -792,32 +944,70 @@ def host_copy(wl):
     return wl.q.cpu().numpy(), K, V, t2
 
 
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def cpu_baseline(wl, target_s, q8k=False):
     """The oracle, as it stands, over the whole workload of this run (its
     sequences, blocks and queries copied to the host; int8 K codes made by
     the oracle's own quantiser), repeated until about target_s seconds of CPU
-    time have been spent."""
+    time have been spent, on all host threads; then on one thread over the
+    first sequences of the same workload (about target_s / 2 seconds)."""
+    import numpy as np
     import oracle
     q, K, V, t2 = host_copy(wl)
     s = wl.spec
     K8 = sc = None
     if q8k:
         K8, sc = quantise_pool_host(K)
+
+    def call(nseq):
+        if q8k:
+            oracle.paged_attention_q8k(q[:nseq], K8, sc, V, t2[:nseq], wl.lens[:nseq],
+                                       scale=wl.scale, q_len=q.shape[1])
+        else:
+            oracle.paged_attention(q[:nseq], K, V, t2[:nseq], wl.lens[:nseq], scale=wl.scale,
+                                   q_len=q.shape[1])
+
+    def kvb(nseq):
+        return algorithmic_bytes(wl.lens[:nseq], q.shape[2], s.Hkv, q.shape[3], s.bs, q.shape[1],
+                                 1 if q8k else 2)[0]
+
+    B = int(wl.lens.shape[0])
     reps, spent = 0, 0.0
     while reps == 0 or spent < target_s:
         t0 = time.perf_counter()
-        if q8k:
-            oracle.paged_attention_q8k(q, K8, sc, V, t2, wl.lens, scale=wl.scale, q_len=q.shape[1])
-        else:
-            oracle.paged_attention(q, K, V, t2, wl.lens, scale=wl.scale, q_len=q.shape[1])
+        call(B)
         spent += time.perf_counter() - t0
         reps += 1
-    kvb = algorithmic_bytes(wl.lens, q.shape[2], s.Hkv, q.shape[3], s.bs, q.shape[1],
-                            1 if q8k else 2)[0]
-    return {"value": round(kvb * reps / spent / 1e9, 4), "unit": "GB/s",
-            "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"whole workload of this run ({wl.B} sequences, {int(wl.lens.sum())} "
-                      f"tokens) x {reps} repeat(s), fp64 C oracle, {spent:.2f} s"}
+    threads = oracle.num_threads()
+    res = {"value": round(kvb(B) * reps / spent / 1e9, 4), "unit": "GB/s", "cores": threads,
+           "kind": "oracle", "cpu_model": cpu_model(),
+           "sample": f"whole workload of this run ({B} sequences, {int(wl.lens.sum())} "
+                     f"tokens) x {reps} repeat(s), fp64 C oracle, {spent:.2f} s"}
+    # one thread: as many leading sequences as fit in about target_s / 2
+    per_seq = spent / reps / B * threads
+    n1 = int(max(1, min(B, (target_s / 2) / max(per_seq, 1e-6))))
+    oracle.set_num_threads(1)
+    try:
+        t0 = time.perf_counter()
+        call(n1)
+        t1 = time.perf_counter() - t0
+    finally:
+        oracle.set_num_threads(threads)
+    res["single_thread"] = {"value": round(kvb(n1) / t1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                            "sample": f"first {n1} of {B} sequences "
+                                      f"({int(np.sum(wl.lens[:n1]))} tokens), {t1:.2f} s"}
+    return res
 
 
 def run_reference(args):
@@ -849,7 +1039,8 @@ def run_reference(args):
             "impl": "reference",
             "config": {"workload": args.workload, "description": spec.description},
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "kind": "oracle",
-                             "cores": oracle.num_threads(), "sample": sample},
+                             "cores": oracle.num_threads(), "cpu_model": cpu_model(),
+                             "sample": sample},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -880,7 +1071,8 @@ def run_reference_prefill(args, base, spec, world):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference", "config": {"workload": args.workload, "description": spec.description},
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "kind": "oracle",
-                             "cores": oracle.num_threads(), "sample": sample},
+                             "cores": oracle.num_threads(), "cpu_model": cpu_model(),
+                             "sample": sample},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 

@@ -319,13 +319,24 @@ int paged_prefill_attention(const void* q, const void* k_pool, const void* v_poo
  *                    (default), -1: plain launch;
  *   seg_cost_blocks  fixed cost, in blocks, charged to every (sequence,
  *                    kv-head) when work is divided among CTAs (default 8;
- *                    -1 for none). */
+ *                    -1 for none);
+ *   producer_wait_ns limit, in nanoseconds, of the loading warp's waits for
+ *                    a free pipeline stage (default 2 s).  Meant for failure-
+ *                    detection tests: with a limit shorter than a stage's
+ *                    turnaround the loader gives up, the CTA finishes the
+ *                    stages already loaded and stops, KV_DEV_TIMEOUT is set
+ *                    in the device error word and the output is undefined;
+ *                    the call still returns and later calls are unaffected.
+ *                    The compute warps' waits keep the default limit (they
+ *                    meet at a barrier at the end of every sequence, so they
+ *                    must all stop at the same stage). */
 typedef struct paged_attention_opts {
     int32_t grid_ctas;
     int32_t min_split_blocks;
     int32_t use_pdl;
     int32_t seg_cost_blocks;
-    int32_t reserved[4];
+    int32_t producer_wait_ns;
+    int32_t reserved[3];
 } paged_attention_opts;
 
 int paged_attention_ex(const void* q, const void* k_pool, const void* v_pool,
@@ -334,6 +345,16 @@ int paged_attention_ex(const void* q, const void* k_pool, const void* v_pool,
                        int32_t B, int32_t Hq, int32_t Hkv, int32_t head_dim, int32_t block_size,
                        int32_t num_blocks, void* workspace, size_t workspace_bytes,
                        const paged_attention_opts* opts, void* stream);
+
+/* paged_attention_q8k with the launch knobs of paged_attention_ex (opts may
+ * be NULL: defaults). */
+int paged_attention_q8k_ex(const void* q, const void* kq_pool, const float* k_scales,
+                           const void* v_pool, const int32_t* block_tables,
+                           int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t q_len,
+                           float scale, void* out, int32_t B, int32_t Hq, int32_t Hkv,
+                           int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                           void* workspace, size_t workspace_bytes,
+                           const paged_attention_opts* opts, void* stream);
 
 /* paged_decode_attention without a workspace argument: for callers that may
  * not allocate device memory themselves (their device memory is owned by

@@ -27,7 +27,7 @@ class KvPoolConfig(ctypes.Structure):
 class PagedAttentionOpts(ctypes.Structure):
     _fields_ = [("grid_ctas", ctypes.c_int32), ("min_split_blocks", ctypes.c_int32),
                 ("use_pdl", ctypes.c_int32), ("seg_cost_blocks", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 4)]
+                ("producer_wait_ns", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
 
 
 _P = ctypes.c_void_p
@@ -79,6 +79,9 @@ SIGNATURES = {
     "paged_kv_append_q8k": ([_P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
     "paged_attention_q8k": ([_P, _P, _P, _P, _P, _i32, _P, _i32, ctypes.c_float, _P, _i32, _i32, _i32,
                              _i32, _i32, _i32, _P, _sz, _P], ctypes.c_int),
+    "paged_attention_q8k_ex": ([_P, _P, _P, _P, _P, _i32, _P, _i32, ctypes.c_float, _P, _i32, _i32,
+                                _i32, _i32, _i32, _i32, _P, _sz, ctypes.POINTER(PagedAttentionOpts),
+                                _P], ctypes.c_int),
 }
 
 

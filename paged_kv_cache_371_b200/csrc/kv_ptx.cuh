@@ -88,6 +88,17 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
+// Bounded wait for short limits: a non-blocking test and a clock read on
+// every poll, so that the limit holds to within a poll.
+__device__ __forceinline__ bool mbar_wait_fine(uint32_t bar, uint32_t parity, uint64_t limit_ns)
+{
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_test(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+
 // ---- copies -------------------------------------------------------------------
 // L2 policy for data read exactly once (K/V tiles).
 __device__ __forceinline__ uint64_t l2_policy_evict_first()

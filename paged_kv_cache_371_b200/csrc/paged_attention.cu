@@ -73,6 +73,7 @@ struct Params {
     int32_t max_blocks, B, q_len, Hq, Hkv, G, rows, num_blocks, min_share;
     int32_t seg_cost;  // virtual blocks charged per (sequence, kv-head) segment
     float scale_log2;
+    uint64_t slot_wait_ns;  // limit of the producer's waits for a free ring slot
 };
 
 template <int D_, int BS_, int MT_, bool FMA_, bool KQ_ = false>
@@ -413,6 +414,17 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
     w.win_len = 0;
     bool ok = true;
     int k_issued = 0;  // stages issued so far (the end marker included)
+    // Wait for ring slot `stage` to be free again (its previous use, `round`
+    // - 1, consumed).  Every lane waits; lane 0's outcome (and its reading of
+    // the abort flag) decides for the warp, so the lanes never disagree.
+    auto slot_wait = [&](int stage, int round, uint64_t limit) -> bool {
+        const uint32_t bar = empty0 + stage * 8;
+        const uint32_t par = (uint32_t)(round - 1) & 1u;
+        bool got = limit >= kWaitLimitNs ? mbar_wait_bounded(bar, par, limit)
+                                         : mbar_wait_fine(bar, par, limit);
+        got = got && !*abort_flag;
+        return __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+    };
 
     if (u0 < u1) {
         // Pass 2: the sequence holding unit u0.
@@ -490,12 +502,9 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
                 const StageDesc& d = cur[k];
                 const int stage = k_issued % C::STAGES;
                 const int round = k_issued / C::STAGES;
-                if (round > 0) {
-                    if (!mbar_wait_bounded(empty0 + stage * 8, (round - 1) & 1, kWaitLimitNs) ||
-                        *abort_flag) {
-                        ok = false;
-                        break;
-                    }
+                if (round > 0 && !slot_wait(stage, round, p.slot_wait_ns)) {
+                    ok = false;
+                    break;
                 }
                 const int32_t id = cid[k];
                 const bool has_tok = lane < d.nbl && d.t0 + lane * C::BS < d.L;
@@ -555,13 +564,19 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
     }
     if (lane == 0) p.meta[blockIdx.x] = w.merge_meta;
 
-    // End marker.
-    if (ok) {
+    // End marker, also after giving up: the consumers then finish the stages
+    // already issued and stop at the marker instead of waiting out their own
+    // limit on a stage that never comes.  After a give-up the slot wait uses
+    // the full limit (the consumers are still draining the ring), unless a
+    // consumer has already stopped.
+    {
         const int stage = k_issued % C::STAGES;
         const int round = k_issued / C::STAGES;
-        if (round > 0 && !mbar_wait_bounded(empty0 + stage * 8, (round - 1) & 1, kWaitLimitNs))
-            ok = false;
-        if (ok) {
+        bool slot_ok = round == 0;
+        if (!slot_ok && ok) slot_ok = slot_wait(stage, round, p.slot_wait_ns);
+        if (!slot_ok) ok = false;
+        if (!slot_ok) slot_ok = slot_wait(stage, round, kWaitLimitNs);
+        if (slot_ok) {
             if (lane == 0) {
                 smeta[stage].flags = F_END;
                 mbar_arrive(full0 + stage * 8);
@@ -1657,6 +1672,8 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
     prm.seg_cost = (opts && opts->seg_cost_blocks != 0) ? (opts->seg_cost_blocks > 0 ? opts->seg_cost_blocks : 0)
                                                         : kDefaultSegCost;
     prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.slot_wait_ns = (opts && opts->producer_wait_ns > 0) ? (uint64_t)opts->producer_wait_ns
+                                                            : kWaitLimitNs;
     const bool pdl = !(opts && opts->use_pdl < 0);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (k_scale)
@@ -1722,6 +1739,20 @@ int paged_attention_q8k(const void* q, const void* kq_pool, const float* k_scale
     return attention_impl(q, kq_pool, v_pool, block_tables, max_blocks_per_seq, context_lens, q_len,
                           scale, out, B, Hq, Hkv, head_dim, block_size, num_blocks, workspace,
                           workspace_bytes, nullptr, stream, k_scales);
+}
+
+int paged_attention_q8k_ex(const void* q, const void* kq_pool, const float* k_scales,
+                           const void* v_pool, const int32_t* block_tables,
+                           int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t q_len,
+                           float scale, void* out, int32_t B, int32_t Hq, int32_t Hkv,
+                           int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                           void* workspace, size_t workspace_bytes,
+                           const paged_attention_opts* opts, void* stream)
+{
+    if (!k_scales) return kv_fail(KV_ERR_INVALID, "paged_attention_q8k_ex: null k_scales");
+    return attention_impl(q, kq_pool, v_pool, block_tables, max_blocks_per_seq, context_lens, q_len,
+                          scale, out, B, Hq, Hkv, head_dim, block_size, num_blocks, workspace,
+                          workspace_bytes, opts, stream, k_scales);
 }
 
 int paged_attention_ex(const void* q, const void* k_pool, const void* v_pool,

@@ -53,3 +53,88 @@ def test_prefill_matches_verify_for_short_windows():
     ref = oracle_subset(wl, [0, 1], q_len=5)
     assert_close(a, ref, "prefill")
     assert_close(b, ref, "verify")
+
+
+def _stage_max_jumps(wl, s, q_len, stage=128):
+    """log2-unit growth of each row's running score maximum at the start of
+    every later stage, from the inputs (fp64): used to show that a case
+    really makes the maximum jump after the first stage."""
+    bs = wl.k_pool.shape[2]
+    L = int(wl.lens[s])
+    n = -(-L // bs)
+    ids = torch.as_tensor(wl.block_tables[s, :n].astype(np.int64), device=wl.k_pool.device)
+    K = wl.k_pool[ids].double().permute(1, 0, 2, 3).reshape(wl.k_pool.shape[1], n * bs, -1)[:, :L]
+    q = wl.q[s].double()                                   # [q_len][Hq][D]
+    G = q.shape[1] // K.shape[0]
+    sc = torch.einsum("jhd,htd->jht", q, K.repeat_interleave(G, 0)) * wl.scale / np.log(2.0)
+    pos = torch.arange(L, device=sc.device)
+    lim = L - q_len + torch.arange(q_len, device=sc.device)
+    sc = sc.masked_fill(pos[None, None, :] > lim[:, None, None], float("-inf"))
+    best = 0.0
+    m = sc[:, :, :stage].amax(-1)
+    for t0 in range(stage, L, stage):
+        mn = torch.maximum(m, sc[:, :, t0:t0 + stage].amax(-1))
+        best = max(best, float((mn - m)[torch.isfinite(m)].max()))
+        m = mn
+    return best
+
+
+@pytest.mark.parametrize("Hq,Hkv,bs,q_len,lens", [
+    (8, 8, 16, 200, [1031, 700]),      # MHA rows, 16-token blocks
+    (64, 8, 8, 48, [1100, 600]),       # G=8, 8-token blocks
+    (64, 8, 16, 160, [900, 1200]),     # G=8, 16-token blocks, two tiles per CTA
+])
+def test_prefill_planted_late_maxima(Hq, Hkv, bs, q_len, lens):
+    """Keys aligned with the queries planted in stage 1, stage 3 and the last
+    (partial) stage, each dominating everything before it by > 2^8 in weight:
+    every stage-j >= 1 rescale of O in tensor memory runs, and the output
+    must still be the oracle's."""
+    from planted import plant
+    wl = make_workload("llama70b_gqa", "cuda", lens=np.array(lens, np.int32), bs=bs, q_len=q_len,
+                       Hq=Hq, Hkv=Hkv, D=128, seed=q_len + 7 * Hq)
+    plan = {}
+    for s, L in enumerate(lens):
+        plan[s] = [(200, 40.0), (450, 80.0), (L - q_len + 5, 120.0), (L - 2, 160.0)]
+    plant(wl, plan, seed=q_len)
+    assert _stage_max_jumps(wl, 0, q_len) > 8.0
+    bt, cl = device_inputs(wl)
+    out = pkv.paged_prefill_attention(wl.q, wl.k_pool, wl.v_pool, bt, cl, wl.scale, q_len)
+    torch.cuda.synchronize()
+    assert pkv.device_error() == 0
+    ref = oracle_subset(wl, list(range(wl.B)), q_len=q_len)
+    assert_close(out, ref, f"planted prefill Hq{Hq} Hkv{Hkv} bs{bs}")
+
+
+@pytest.mark.parametrize("Hq,Hkv,bs", [(8, 8, 16), (64, 8, 8), (64, 8, 16)])
+def test_prefill_ramped_keys(Hq, Hkv, bs):
+    """Key norms growing along the context (x(1 + t/150)): the row maxima
+    climb stage after stage and the lazy rescale fires repeatedly."""
+    from planted import ramp
+    q_len = 96
+    lens = [1000, 777]
+    wl = make_workload("llama70b_gqa", "cuda", lens=np.array(lens, np.int32), bs=bs, q_len=q_len,
+                       Hq=Hq, Hkv=Hkv, D=128, seed=5 + Hq + bs)
+    ramp(wl, 150.0)
+    assert _stage_max_jumps(wl, 0, q_len) > 2.0
+    bt, cl = device_inputs(wl)
+    out = pkv.paged_prefill_attention(wl.q, wl.k_pool, wl.v_pool, bt, cl, wl.scale, q_len)
+    torch.cuda.synchronize()
+    assert pkv.device_error() == 0
+    ref = oracle_subset(wl, list(range(wl.B)), q_len=q_len)
+    assert_close(out, ref, f"ramped prefill Hq{Hq} bs{bs}")
+
+
+def test_prefill_chunk_full_size_whole_sequences():
+    """The benchmark's chunked-prefill workload at full size (8 sequences, a
+    512-token chunk each on prefixes of 1-4K tokens, GQA 64/8), launched as
+    the benchmark launches it; every row of every head of the shortest and
+    the longest sequence compared with the oracle."""
+    wl = make_workload("prefill_chunk", "cuda")
+    q_len = wl.spec.q_len
+    bt, cl = device_inputs(wl)
+    out = pkv.paged_prefill_attention(wl.q, wl.k_pool, wl.v_pool, bt, cl, wl.scale, q_len)
+    torch.cuda.synchronize()
+    assert pkv.device_error() == 0
+    seqs = sorted({int(np.argmin(wl.lens)), int(np.argmax(wl.lens))})
+    ref = oracle_subset(wl, seqs, q_len=q_len)
+    assert_close(out[torch.as_tensor(seqs, device="cuda")], ref, "prefill_chunk full size")

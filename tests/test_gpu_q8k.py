@@ -175,3 +175,54 @@ def test_copy_blocks_q8k_is_a_block_copy():
     assert np.array_equal(kq.cpu().numpy(), k_ref)
     assert np.array_equal(vq.cpu().numpy().view(np.uint16), v_ref.view(np.uint16))
 
+
+
+def _pool_scales(wl):
+    """Channel scales from every token of the pool (unused rows, which hold
+    NaN, count as zeros), computed by the oracle on the host."""
+    K = np.nan_to_num(wl.k_pool.cpu().numpy())
+    nb, Hkv, bs, D = K.shape
+    return oracle.k_scales(K.transpose(0, 2, 1, 3).reshape(nb * bs, Hkv, D))
+
+
+@pytest.mark.parametrize("name", ["llama7b_mha", "llama70b_gqa", "llama70b_gqa_bs8", "long_verify"])
+def test_attention_q8k_full_size_every_sequence(name):
+    """The int8-K forms of the benchmark's workloads at full size (scales from
+    the whole pool, as the benchmark sets them), launched as the benchmark
+    launches them: device codes bit-exact against the oracle's, and every
+    output element of every sequence within tolerance."""
+    wl = make_workload(name, "cuda")
+    q_len = wl.q.shape[1]
+    scales = _pool_scales(wl)
+    kq, vq, sc = _quantise_on_device(wl, scales)
+    bt, cl = torch.as_tensor(wl.block_tables, device="cuda"), torch.as_tensor(wl.lens, device="cuda")
+    out = pkv.paged_attention_q8k(wl.q, kq, sc, vq, bt, cl, wl.scale, q_len=q_len)
+    torch.cuda.synchronize()
+    assert pkv.device_error() == 0
+    ref = _oracle_subset_q8k(wl, kq, scales, np.arange(wl.B), wl.q, q_len)
+    assert_close(out, ref, f"q8k {name} full size")
+
+
+@pytest.mark.parametrize("Hq,Hkv,bs,q_len", [(8, 8, 16, 1), (64, 8, 16, 1), (64, 8, 8, 1),
+                                             (32, 8, 16, 5)])
+@pytest.mark.parametrize("grid,min_split", [(0, 0), (300, 1), (7, 1)])
+def test_attention_q8k_planted_late_maxima(Hq, Hkv, bs, q_len, grid, min_split):
+    """Dominant keys planted after the first stage (see planted.py) over an
+    int8 K pool: FMA, one-tile and two-tile tensor-core consumers, with and
+    without forced context splits."""
+    from planted import plant
+    lens = np.array([1500, 700, 333], np.int32)
+    wl = make_workload("llama70b_gqa", "cuda", lens=lens, bs=bs, q_len=q_len, Hq=Hq, Hkv=Hkv,
+                       D=128, seed=29 + Hq + bs + q_len)
+    plan = {s: [(70, 40.0), (300, 80.0), (int(L) - 10, 120.0), (int(L) - 1, 160.0)]
+            for s, L in enumerate(lens)}
+    plant(wl, plan, seed=3 + Hq)
+    scales = _pool_scales(wl)
+    kq, vq, sc = _quantise_on_device(wl, scales)
+    bt, cl = torch.as_tensor(wl.block_tables, device="cuda"), torch.as_tensor(wl.lens, device="cuda")
+    out = pkv.paged_attention_q8k(wl.q, kq, sc, vq, bt, cl, wl.scale, q_len=q_len, grid_ctas=grid,
+                                  min_split_blocks=min_split)
+    torch.cuda.synchronize()
+    assert pkv.device_error() == 0
+    ref = _oracle_subset_q8k(wl, kq, scales, np.arange(wl.B), wl.q, q_len)
+    assert_close(out, ref, f"q8k planted Hq{Hq} bs{bs} q{q_len}")

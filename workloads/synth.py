@@ -188,8 +188,11 @@ def make_workload(name: str, device="cpu", *, B: Optional[int] = None,
         num_blocks = max(spec.pool_blocks, total_need)
     else:
         num_blocks = int(math.ceil(spec.pool_factor * total_need))
+    # spare blocks go after the permuted pool, so that the placement of the
+    # sequences does not depend on how much room is added for appends
+    order = np.concatenate([rng.permutation(num_blocks),
+                            num_blocks + np.arange(int(spare_blocks))]).astype(np.int32)
     num_blocks += int(spare_blocks)
-    order = rng.permutation(num_blocks).astype(np.int32)
 
     max_blocks = max(1, max(need) if need else 1)
     tables = np.full((B, max_blocks), -1, dtype=np.int32)
