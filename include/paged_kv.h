@@ -321,9 +321,12 @@ int paged_prefill_attention(const void* q, const void* k_pool, const void* v_poo
  *                    kv-head) when work is divided among CTAs (default 8;
  *                    -1 for none);
  *   producer_wait_ns limit, in nanoseconds, of the loading warp's waits for
- *                    a free pipeline stage (default 2 s).  Meant for failure-
- *                    detection tests: with a limit shorter than a stage's
- *                    turnaround the loader gives up, the CTA finishes the
+ *                    a free pipeline stage (default 2 s; below 1000 the
+ *                    loader gives up at the first stage that is not already
+ *                    free, as the device timer is too coarse to measure
+ *                    less).  Meant for failure-detection tests: with a limit
+ *                    shorter than a stage's turnaround the loader gives up,
+ *                    the CTA finishes the
  *                    stages already loaded and stops, KV_DEV_TIMEOUT is set
  *                    in the device error word and the output is undefined;
  *                    the call still returns and later calls are unaffected.

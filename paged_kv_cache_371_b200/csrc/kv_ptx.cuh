@@ -89,9 +89,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 }
 
 // Bounded wait for short limits: a non-blocking test and a clock read on
-// every poll, so that the limit holds to within a poll.
+// every poll.  The global timer advances in steps of up to a microsecond or
+// more, so a limit below kFineWaitNs gives up at once when the phase is not
+// already complete (a deterministic form for failure-detection tests).
+constexpr uint64_t kFineWaitNs = 1000;
 __device__ __forceinline__ bool mbar_wait_fine(uint32_t bar, uint32_t parity, uint64_t limit_ns)
 {
+    if (mbar_test(bar, parity)) return true;
+    if (limit_ns < kFineWaitNs) return false;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         if (mbar_test(bar, parity)) return true;
@@ -162,6 +167,15 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                  : "r"(addr));
+}
+
+// Transpose of an 8x8 b16 matrix held as one 32-bit register per lane (lane
+// l: row l/4, columns 2*(l%4), +1) into the same layout.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)
+{
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
 }
 
 // D = A(16x16, row) * B(16x8, col) + D, fp16 operands, fp32 accumulators.

@@ -76,11 +76,15 @@ struct Params {
     uint64_t slot_wait_ns;  // limit of the producer's waits for a free ring slot
 };
 
-template <int D_, int BS_, int MT_, bool FMA_, bool KQ_ = false>
+template <int D_, int BS_, int MT_, bool FMA_, bool KQ_ = false, int NR8_ = 0, int TW_ = 0,
+          int SUBS_ = 1>
 struct Cfg {
     static constexpr int D = D_, BS = BS_, MT = MT_;
     static constexpr bool FMA = FMA_;
     static constexpr bool KQ = KQ_;  // K pool of int8 codes with per-channel scales
+    // NR8 > 0: tensor-core consumer over S^T = K Q^T (tokens as the MMA's M
+    // dimension, query rows as N, in NR8 tiles of 8 rows)
+    static constexpr int NR8 = NR8_;
     static_assert(!KQ || D == 128, "int8 K pools are served at head_dim 128");
     static constexpr int NH = D / 64;                       // 64-column halves per row
     // consumer warps along the tokens of a stage (16 tokens each) and tokens
@@ -88,10 +92,15 @@ struct Cfg {
     // gain from twice the warps; the tensor-core consumers keep 4 (with 9
     // warps their register cap would drop to 168 and the merge at each
     // segment end would take twice the rounds)
-    static constexpr int TW = FMA ? 8 : 4;
-    static constexpr int TS = 16 * TW;                      // tokens per pipeline stage
+    static constexpr int TW = TW_ ? TW_ : (FMA ? 8 : 4);
+    // 16-token sub-tiles each consumer warp takes per stage (the transposed
+    // tensor-core consumer only): larger stages at the same register count
+    static constexpr int SUBS = SUBS_;
+    static_assert(SUBS == 1 || NR8 > 0, "sub-tiles need the transposed consumer");
+    static constexpr int TS = 16 * TW * SUBS;               // tokens per pipeline stage
+    static_assert(TS / BS <= 32, "one producer lane per block of a stage");
     static constexpr int NBS = TS / BS;                     // blocks per stage
-    static constexpr int RP = FMA ? 1 : 16 * MT;            // padded rows
+    static constexpr int RP = FMA ? 1 : (NR8 ? 8 * NR8 : 16 * MT);  // padded rows
     static constexpr int NCW = TW;                          // consumer warps
     static constexpr int THREADS = (NCW + 1) * 32;
     // registers per thread for one CTA per SM: warps are spread over the 4
@@ -109,11 +118,18 @@ struct Cfg {
     static constexpr int Q_BYTES = (RP * QROW + 1023) / 1024 * 1024;
     static constexpr int Q_OFF = K_BYTES + KV_BYTES;
     static constexpr int STAGE_BYTES = Q_OFF + Q_BYTES;
-    static constexpr int OB_STRIDE = D + 8;                 // floats per obuf row
+    // floats per obuf row (the transposed consumer's scalar stores of rows
+    // 2*tig, 2*tig+1 are conflict-free when 2 * OB_STRIDE = 8 mod 32)
+    static constexpr int OB_STRIDE = NR8 ? D + 4 : D + 8;
     static constexpr int OBUF_SLICE = RP * OB_STRIDE;               // floats
     static constexpr int OBUF_BYTES = 2 * OBUF_SLICE * 4;           // two merge slices
     static constexpr int ML_BYTES = TW * RP * 2 * 4;
-    static constexpr int QP_BYTES = MT > 1 ? RP * QROW : 0;   // CTA copy of the query rows
+    // CTA copy of the query rows (read again every stage)
+    static constexpr bool QPERSIST = NR8 ? NR8 > 2 : MT > 1;
+    // rows of that copy: whole pairs of 8-row tiles (B fragments of two row
+    // tiles come from one ldmatrix)
+    static constexpr int QP_ROWS = NR8 ? 16 * ((NR8 + 1) / 2) : RP;
+    static constexpr int QP_BYTES = QPERSIST ? QP_ROWS * QROW : 0;
     static constexpr int FIXED = OBUF_BYTES + ML_BYTES + QP_BYTES + 256 + 16 * 64;
     static constexpr int STAGES_RAW = (kSmemBudget - FIXED) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
@@ -1352,6 +1368,342 @@ __device__ void consumer_mma_mt(const Params& p, uint8_t* smem, volatile int* ab
     }
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core consumer with the tokens as the MMA's M dimension: per warp and
+// stage, S^T (16 tokens x 8*NR8 rows) = K Q^T and O^T (head dims x rows) +=
+// V^T P^T, mma.sync m16n8k16.  No row padding to 16 (a GQA group of 8 fills
+// one n8 tile), half the MMAs and half the accumulator registers of the
+// rows-as-M form.  P^T reaches the B-operand layout of the P V product with
+// movmatrix (an 8x8 transpose in registers).  Each thread owns rows 2*tig,
+// 2*tig+1 of every row tile for two tokens (gid, gid + 8): a row's softmax
+// maximum and sum reduce over the 8 lanes of one tig.
+template <class C>
+__device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_flag)
+{
+    constexpr int NR = C::NR8;
+    constexpr int KS = C::D / 16;
+    const int qw = threadIdx.x >> 5;  // token warp
+    const int lane = threadIdx.x & 31;
+    const int gid = lane >> 2, tig = lane & 3;
+    const uint32_t sbase = smem_u32(smem);
+    const StageMeta* smeta = reinterpret_cast<const StageMeta*>(smem + C::META_OFF);
+    const uint32_t full0 = sbase + C::BAR_OFF;
+    const uint32_t empty0 = full0 + C::STAGES * 8;
+    const uint32_t zero_row = sbase + C::ZERO_OFF;
+    float* mlb = reinterpret_cast<float*>(smem + C::ML_OFF);
+    float* obuf = reinterpret_cast<float*>(smem + C::OBUF_OFF);
+    const float sl2 = p.scale_log2;
+
+    // ldmatrix lane geometry.  K as the A operand: matrices (tokens 0-7 |
+    // 8-15) x (dims lo | hi); V^T as the A operand (transposed load):
+    // matrices (dims lo | hi) x (tokens 0-7 | 8-15); query rows as the B
+    // operand: row lane & 7 of a row tile, 16-byte chunk lane >> 3.
+    const int a_i = ((lane >> 3) & 1) * 8 + (lane & 7);
+    const int a_sel = lane >> 4;
+    const int v_i = (lane >> 4) * 8 + (lane & 7);
+    const int v_sel = (lane >> 3) & 1;
+
+    float O[KS][NR][4];  // O^T tile (dims 16*np.., rows 8*nt..): d = gid(+8), r = 2tig(+1)
+    uint32_t qb[C::QPERSIST ? 1 : KS][NR][2];  // B fragments of the query rows
+    float m[NR][2], l[NR][2];
+    float corr[NR][2];  // int8 keys: bias * row sum of the scaled q
+    int lim[NR][2];
+
+    // B fragments of k-steps ks, ks+1 of row tile nt from padded query rows at `rows`
+    auto load_qb2 = [&](uint32_t rows, int nt, int ks, uint32_t (&b)[4]) {
+        ldsm_x4(rows + (nt * 8 + (lane & 7)) * C::QROW + ((2 * ks + (lane >> 3)) << 4), b[0], b[1],
+                b[2], b[3]);
+    };
+
+    int stage = 0;
+    uint32_t phase = 0;
+    for (;;) {
+        if (!mbar_wait_bounded(full0 + stage * 8, phase, kWaitLimitNs)) {
+            *abort_flag = 1;
+            break;
+        }
+        const StageMeta md = smeta[stage];
+        if (md.flags & F_END) break;
+        const uint32_t st = sbase + stage * C::STAGE_BYTES;
+        if (md.flags & F_FIRST) {
+            uint32_t qsrc = st + C::Q_OFF;
+            if constexpr (C::QPERSIST) {
+                // copy the segment's query rows out of the stage (read every stage)
+                const uint4* src = reinterpret_cast<const uint4*>(smem + stage * C::STAGE_BYTES + C::Q_OFF);
+                uint4* dst = reinterpret_cast<uint4*>(smem + C::QP_OFF);
+                constexpr int CPR = C::QROW / 16;  // 16-byte chunks per padded row
+                if constexpr (!C::KQ) {
+                    for (int i = threadIdx.x; i < C::RP * CPR; i += C::NCW * 32) dst[i] = src[i];
+                } else {
+                    // q times the channel scales, each 16-dim chunk stored in the
+                    // permuted order of the int8 key fragments (dims 0,1,4,5,8,9,
+                    // 12,13 then 2,3,6,7,10,11,14,15)
+                    const float* sc = p.k_scale + (int64_t)md.kvh * C::D;
+                    for (int i = threadIdx.x; i < C::RP * KS; i += C::NCW * 32) {
+                        const int row = i / KS, ks = i % KS;
+                        const uint4 a = src[row * CPR + 2 * ks], b = src[row * CPR + 2 * ks + 1];
+                        const float* s16 = sc + 16 * ks;
+                        const uint32_t pr[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+                        uint32_t q2[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            q2[e] = scale_h2(pr[e], *reinterpret_cast<const float2*>(s16 + 2 * e));
+                        dst[row * CPR + 2 * ks] = make_uint4(q2[0], q2[2], q2[4], q2[6]);
+                        dst[row * CPR + 2 * ks + 1] = make_uint4(q2[1], q2[3], q2[5], q2[7]);
+                    }
+                }
+                named_bar_sync(2, C::NCW * 32);
+                qsrc = sbase + C::QP_OFF;
+            } else if constexpr (!C::KQ) {
+#pragma unroll
+                for (int nt = 0; nt < NR; ++nt)
+#pragma unroll
+                    for (int ks = 0; ks < KS; ks += 2) {
+                        uint32_t b[4];
+                        load_qb2(qsrc, nt, ks, b);
+                        qb[ks][nt][0] = b[0];
+                        qb[ks][nt][1] = b[1];
+                        qb[ks + 1][nt][0] = b[2];
+                        qb[ks + 1][nt][1] = b[3];
+                    }
+            } else {
+                // int8 keys: q of row nt*8+gid times the channel scales, in the
+                // permuted dim order (lane tig: dims 4tig, 4tig+1 | 4tig+2, 4tig+3)
+                const float* sc = p.k_scale + (int64_t)md.kvh * C::D;
+#pragma unroll
+                for (int nt = 0; nt < NR; ++nt) {
+                    const uint8_t* qr = smem + stage * C::STAGE_BYTES + C::Q_OFF + (nt * 8 + gid) * C::QROW;
+#pragma unroll
+                    for (int ks = 0; ks < KS; ++ks) {
+                        const int d = 16 * ks + 4 * tig;
+                        qb[ks][nt][0] = scale_h2(*reinterpret_cast<const uint32_t*>(qr + d * 2),
+                                                 *reinterpret_cast<const float2*>(sc + d));
+                        qb[ks][nt][1] = scale_h2(*reinterpret_cast<const uint32_t*>(qr + d * 2 + 4),
+                                                 *reinterpret_cast<const float2*>(sc + d + 2));
+                    }
+                }
+            }
+            if constexpr (C::KQ) {
+                // bias corrections of this thread's rows 8nt + 2tig (+1): sums of
+                // their scaled q entries (lane tig adds 32 of the 128 dims of row
+                // 8nt + gid, then the row sums are fetched from lane 4*row)
+#pragma unroll
+                for (int nt = 0; nt < NR; ++nt) {
+                    float acc = 0.f;
+                    if constexpr (C::QPERSIST) {
+                        const uint32_t* qr = reinterpret_cast<const uint32_t*>(
+                            smem + C::QP_OFF + (nt * 8 + gid) * C::QROW) + tig * 16;
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) acc += h2_sum(qr[e]);
+                    } else {
+#pragma unroll
+                        for (int ks = 0; ks < KS; ++ks) acc += h2_sum(qb[ks][nt][0]) + h2_sum(qb[ks][nt][1]);
+                    }
+                    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+                    corr[nt][0] = kCodeBias * __shfl_sync(0xffffffffu, acc, (2 * tig) * 4);
+                    corr[nt][1] = kCodeBias * __shfl_sync(0xffffffffu, acc, (2 * tig + 1) * 4);
+                }
+            }
+#pragma unroll
+            for (int np = 0; np < KS; ++np)
+#pragma unroll
+                for (int nt = 0; nt < NR; ++nt) O[np][nt][0] = O[np][nt][1] = O[np][nt][2] = O[np][nt][3] = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < NR; ++nt)
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int R = nt * 8 + 2 * tig + i;
+                    m[nt][i] = kNegInf;
+                    l[nt][i] = 0.f;
+                    lim[nt][i] = R < p.rows ? md.L - p.q_len + R / p.G + 1 : md.L;
+                }
+        }
+#pragma unroll 1
+        for (int sub = 0; sub < C::SUBS; ++sub) {
+        const int tb = (qw * C::SUBS + sub) * 16;  // first stage token of this sub-tile
+        const int nv = md.ntok - tb;
+        if (nv > 0) {
+            const int a_tok = tb + a_i, v_tok = tb + v_i;
+            // S^T = K Q^T for my 16 tokens; the k-steps accumulate into NCH
+            // separate chains (fewer dependent MMAs in a row), summed after
+            constexpr int NCH = NR == 1 ? 4 : 2;
+            float Sc[NCH][NR][4];
+#pragma unroll
+            for (int c = 0; c < NCH; ++c)
+#pragma unroll
+                for (int nt = 0; nt < NR; ++nt) Sc[c][nt][0] = Sc[c][nt][1] = Sc[c][nt][2] = Sc[c][nt][3] = 0.f;
+            const uint32_t qrows = sbase + C::QP_OFF;
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                float (&S)[NR][4] = Sc[ks % NCH];
+                uint32_t a[4];
+                if constexpr (C::KQ) {
+                    // tokens gid and gid + 8, dims 16ks + 4tig .. +3 (permuted order)
+                    i8x4_to_h2x2_biased(lds_u32(st + tile_chunk_k8<C>(tb + gid, ks) + 4 * tig), a[0], a[2]);
+                    i8x4_to_h2x2_biased(lds_u32(st + tile_chunk_k8<C>(tb + gid + 8, ks) + 4 * tig), a[1], a[3]);
+                } else {
+                    ldsm_x4(st + tile_chunk<C>(a_tok, 2 * ks + a_sel), a[0], a[1], a[2], a[3]);
+                }
+                if constexpr (C::QPERSIST) {
+#pragma unroll
+                    for (int nt = 0; nt < NR; nt += 2) {
+                        // two row tiles per load: (tile nt | nt+1) x (chunk 2ks | 2ks+1)
+                        uint32_t b[4];
+                        const int row = nt * 8 + (lane & 7) + ((lane >> 4) & 1) * 8;
+                        ldsm_x4(qrows + row * C::QROW + ((2 * ks + ((lane >> 3) & 1)) << 4), b[0], b[1], b[2],
+                                b[3]);
+                        mma_16816(S[nt], a, b[0], b[1]);
+                        if (nt + 1 < NR) mma_16816(S[nt + 1], a, b[2], b[3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int nt = 0; nt < NR; ++nt) mma_16816(S[nt], a, qb[ks][nt][0], qb[ks][nt][1]);
+                }
+            }
+            float S[NR][4];
+#pragma unroll
+            for (int nt = 0; nt < NR; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float v = Sc[0][nt][e];
+#pragma unroll
+                    for (int c = 1; c < NCH; ++c) v += Sc[c][nt][e];
+                    S[nt][e] = v;
+                }
+            // mask: a token counts if the row may see it and this stage loaded it
+            const int pos0 = md.t0 + tb + gid;
+            const int st_end = md.t0 + md.ntok;
+            bool rescale = false;
+            float alpha[NR][2], mu[NR][2];
+#pragma unroll
+            for (int nt = 0; nt < NR; ++nt) {
+                float mx[2];
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int lm = min(lim[nt][i], st_end);
+                    const float c0 = C::KQ ? S[nt][i] - corr[nt][i] : S[nt][i];
+                    const float c1 = C::KQ ? S[nt][2 + i] - corr[nt][i] : S[nt][2 + i];
+                    S[nt][i] = pos0 < lm ? c0 * sl2 : kNegInf;
+                    S[nt][2 + i] = pos0 + 8 < lm ? c1 * sl2 : kNegInf;
+                    mx[i] = fmaxf(S[nt][i], S[nt][2 + i]);
+                }
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1)
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], off));
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float mn = fmaxf(m[nt][i], mx[i]);
+                    mu[nt][i] = mn == kNegInf ? 0.f : mn;
+                    alpha[nt][i] = ex2(m[nt][i] - mu[nt][i]);
+                    m[nt][i] = mn;
+                    rescale |= alpha[nt][i] != 1.f;
+                }
+            }
+            uint32_t pb[NR][2];
+#pragma unroll
+            for (int nt = 0; nt < NR; ++nt) {
+                const float e0 = ex2(S[nt][0] - mu[nt][0]), e1 = ex2(S[nt][1] - mu[nt][1]);
+                const float e2 = ex2(S[nt][2] - mu[nt][0]), e3 = ex2(S[nt][3] - mu[nt][1]);
+                l[nt][0] = l[nt][0] * alpha[nt][0] + (e0 + e2);
+                l[nt][1] = l[nt][1] * alpha[nt][1] + (e1 + e3);
+                // P^T (tokens x rows) -> P (rows x tokens) fragments: b0 = P[gid][2tig..],
+                // b1 = P[gid][8 + 2tig..]
+                pb[nt][0] = movmatrix_trans(pack_half2(e0, e1));
+                pb[nt][1] = movmatrix_trans(pack_half2(e2, e3));
+            }
+            if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                for (int np = 0; np < KS; ++np)
+#pragma unroll
+                    for (int nt = 0; nt < NR; ++nt) {
+                        O[np][nt][0] *= alpha[nt][0];
+                        O[np][nt][1] *= alpha[nt][1];
+                        O[np][nt][2] *= alpha[nt][0];
+                        O[np][nt][3] *= alpha[nt][1];
+                    }
+            }
+            // O^T += V^T P^T; rows of V past the valid tokens read a zero row
+            const bool v_ok = v_i < nv;
+#pragma unroll
+            for (int np = 0; np < KS; ++np) {
+                const uint32_t addr = v_ok ? st + C::V_OFF + tile_chunk<C>(v_tok, 2 * np + v_sel) : zero_row;
+                uint32_t a[4];
+                ldsm_x4_trans(addr, a[0], a[1], a[2], a[3]);
+#pragma unroll
+                for (int nt = 0; nt < NR; ++nt) mma_16816(O[np][nt], a, pb[nt][0], pb[nt][1]);
+            }
+        }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + stage * 8);
+
+        if (md.flags & F_LAST) {
+            // merge the token-warps (fixed order), then store
+            const int tid = threadIdx.x;
+#pragma unroll
+            for (int nt = 0; nt < NR; ++nt)
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    float lr = l[nt][i];
+                    lr += __shfl_xor_sync(0xffffffffu, lr, 4);
+                    lr += __shfl_xor_sync(0xffffffffu, lr, 8);
+                    lr += __shfl_xor_sync(0xffffffffu, lr, 16);
+                    if (gid == 0) {
+                        const int R = nt * 8 + 2 * tig + i;
+                        mlb[(qw * C::RP + R) * 2] = m[nt][i];
+                        mlb[(qw * C::RP + R) * 2 + 1] = lr;
+                    }
+                }
+            named_bar_sync(1, C::NCW * 32);
+            float f[NR][2];
+#pragma unroll
+            for (int nt = 0; nt < NR; ++nt)
+#pragma unroll
+                for (int i = 0; i < 2; ++i) f[nt][i] = row_factor<C>(mlb, nt * 8 + 2 * tig + i, m[nt][i]);
+            // token-warps 0 and 1 write slices 0 and 1, then each later pair adds to them
+            float* slice = obuf + (qw & 1) * C::OBUF_SLICE;
+            for (int round = 0; round < C::TW / 2; ++round) {
+                if ((qw >> 1) == round) {
+#pragma unroll
+                    for (int nt = 0; nt < NR; ++nt) {
+                        float* r0 = slice + (nt * 8 + 2 * tig) * C::OB_STRIDE + gid;
+                        float* r1 = r0 + C::OB_STRIDE;
+                        const bool ok0 = nt * 8 + 2 * tig < p.rows, ok1 = nt * 8 + 2 * tig + 1 < p.rows;
+                        float x[KS][4];  // loads first, then stores
+#pragma unroll
+                        for (int np = 0; np < KS; ++np) {
+                            x[np][0] = round && ok0 ? r0[16 * np] : 0.f;
+                            x[np][1] = round && ok1 ? r1[16 * np] : 0.f;
+                            x[np][2] = round && ok0 ? r0[16 * np + 8] : 0.f;
+                            x[np][3] = round && ok1 ? r1[16 * np + 8] : 0.f;
+                        }
+#pragma unroll
+                        for (int np = 0; np < KS; ++np) {
+                            if (ok0) {
+                                r0[16 * np] = x[np][0] + O[np][nt][0] * f[nt][0];
+                                r0[16 * np + 8] = x[np][2] + O[np][nt][2] * f[nt][0];
+                            }
+                            if (ok1) {
+                                r1[16 * np] = x[np][1] + O[np][nt][1] * f[nt][1];
+                                r1[16 * np + 8] = x[np][3] + O[np][nt][3] * f[nt][1];
+                            }
+                        }
+                    }
+                }
+                named_bar_sync(1, C::NCW * 32);
+            }
+            store_segment<C>(p, md, obuf, mlb, tid);
+            named_bar_sync(1, C::NCW * 32);
+        }
+        if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+        }
+    }
+}
+
 template <class C>
 __global__ void __maxnreg__(C::MAXREG)
     paged_attention_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -1389,6 +1741,8 @@ __global__ void __maxnreg__(C::MAXREG)
         producer<C>(&tmK, &tmV, p, smem, &abort_flag);
     } else if constexpr (C::FMA) {
         consumer_fma<C>(p, smem, &abort_flag);
+    } else if constexpr (C::NR8 > 0) {
+        consumer_tc<C>(p, smem, &abort_flag);
     } else if constexpr (C::MT > 1) {
         consumer_mma_mt<C>(p, smem, &abort_flag);
     } else {
@@ -1596,8 +1950,13 @@ template <int D, int BS, bool KQ = false>
 int dispatch_rows(int rows, const CUtensorMap& tk, const CUtensorMap& tv, const Params& prm,
                   int grid, bool pdl, cudaStream_t st)
 {
+    // Tensor-core paths: 128-token stages (8 token warps for one row tile, 4
+    // warps of two 16-token sub-tiles for two or three); more than 24 rows
+    // keep the rows-as-M consumer (its accumulators fit 255 registers).
     if (rows == 1) return launch<Cfg<D, BS, 1, true, KQ>>(tk, tv, prm, grid, pdl, st);
-    if (rows <= 16) return launch<Cfg<D, BS, 1, false, KQ>>(tk, tv, prm, grid, pdl, st);
+    if (rows <= 8) return launch<Cfg<D, BS, 1, false, KQ, 1, 8, 1>>(tk, tv, prm, grid, pdl, st);
+    if (rows <= 16) return launch<Cfg<D, BS, 1, false, KQ, 2, 4, 2>>(tk, tv, prm, grid, pdl, st);
+    if (rows <= 24) return launch<Cfg<D, BS, 1, false, KQ, 3, 4, 2>>(tk, tv, prm, grid, pdl, st);
     return launch<Cfg<D, BS, 2, false, KQ>>(tk, tv, prm, grid, pdl, st);
 }
 
