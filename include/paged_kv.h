@@ -318,8 +318,8 @@ int paged_prefill_attention(const void* q, const void* k_pool, const void* v_poo
  *   use_pdl          1: launch the merge with programmatic dependent launch
  *                    (default), -1: plain launch;
  *   seg_cost_blocks  fixed cost, in blocks, charged to every (sequence,
- *                    kv-head) when work is divided among CTAs (default 8;
- *                    -1 for none);
+ *                    kv-head) when work is divided among CTAs (default: 128
+ *                    tokens' worth, 256 over an int8 K pool; -1 for none);
  *   producer_wait_ns limit, in nanoseconds, of the loading warp's waits for
  *                    a free pipeline stage (default 2 s; below 1000 the
  *                    loader gives up at the first stage that is not already

@@ -51,7 +51,11 @@ namespace pkv {
 constexpr int kMaxMT = 2;                   // m16 tiles of rows per KV head (rows <= 32)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kSmemBudget = 225 * 1024;
-constexpr int kDefaultSegCost = 8;          // virtual blocks per segment (balance)
+// Fixed cost of a (sequence, kv-head) segment when work is divided among CTAs,
+// in tokens of K/V streaming (query load, merge, partial last stage): about
+// one 128-token stage, two for int8 keys (a third less bytes per token)
+constexpr int kSegCostTokens = 128;
+constexpr int kSegCostTokensQ8 = 256;
 constexpr float kNegInf = -__builtin_huge_valf();
 
 enum : int32_t { F_FIRST = 1, F_LAST = 2, F_WHOLE = 4, F_END = 8 };
@@ -1951,10 +1955,15 @@ int dispatch_rows(int rows, const CUtensorMap& tk, const CUtensorMap& tv, const 
                   int grid, bool pdl, cudaStream_t st)
 {
     // Tensor-core paths: 128-token stages (8 token warps for one row tile, 4
-    // warps of two 16-token sub-tiles for two or three); more than 24 rows
-    // keep the rows-as-M consumer (its accumulators fit 255 registers).
+    // warps of two 16-token sub-tiles for two or three; 256 tokens for one
+    // row tile over int8 keys); more than 24 rows keep the rows-as-M consumer
+    // (its accumulators fit 255 registers).
     if (rows == 1) return launch<Cfg<D, BS, 1, true, KQ>>(tk, tv, prm, grid, pdl, st);
-    if (rows <= 8) return launch<Cfg<D, BS, 1, false, KQ, 1, 8, 1>>(tk, tv, prm, grid, pdl, st);
+    if (rows <= 8) {
+        // int8 keys stream 3/4 of the bytes per token: 256-token stages
+        if constexpr (KQ) return launch<Cfg<D, BS, 1, false, KQ, 1, 8, 2>>(tk, tv, prm, grid, pdl, st);
+        else return launch<Cfg<D, BS, 1, false, KQ, 1, 8, 1>>(tk, tv, prm, grid, pdl, st);
+    }
     if (rows <= 16) return launch<Cfg<D, BS, 1, false, KQ, 2, 4, 2>>(tk, tv, prm, grid, pdl, st);
     if (rows <= 24) return launch<Cfg<D, BS, 1, false, KQ, 3, 4, 2>>(tk, tv, prm, grid, pdl, st);
     return launch<Cfg<D, BS, 2, false, KQ>>(tk, tv, prm, grid, pdl, st);
@@ -2029,7 +2038,7 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
     prm.num_blocks = num_blocks;
     prm.min_share = (opts && opts->min_split_blocks > 0) ? opts->min_split_blocks : 16;
     prm.seg_cost = (opts && opts->seg_cost_blocks != 0) ? (opts->seg_cost_blocks > 0 ? opts->seg_cost_blocks : 0)
-                                                        : kDefaultSegCost;
+                                                        : (k_scale ? kSegCostTokensQ8 : kSegCostTokens) / BS;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.slot_wait_ns = (opts && opts->producer_wait_ns > 0) ? (uint64_t)opts->producer_wait_ns
                                                             : kWaitLimitNs;

@@ -200,66 +200,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
         : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// ---- packed arithmetic of the softmax -------------------------------------------
-__device__ __forceinline__ uint64_t f32x2(float lo, float hi)
-{
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ void f32x2_split(uint64_t v, float& lo, float& hi)
-{
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-// two fp32 a*b + c in one instruction
-__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c)
-{
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b)
-{
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-// (lo, hi) rounded to an fp16 pair, lo in the low half
-__device__ __forceinline__ uint32_t cvt_f16x2(float lo, float hi)
-{
-    uint32_t d;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
-    return d;
-}
-// 2^x of both halves of an fp16 pair (one MUFU operation for two weights)
-__device__ __forceinline__ uint32_t ex2_f16x2(uint32_t x)
-{
-    uint32_t d;
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(d) : "r"(x));
-    return d;
-}
-__device__ __forceinline__ uint32_t add_f16x2(uint32_t a, uint32_t b)
-{
-    uint32_t d;
-    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t f16x2_to_f32x2(uint32_t h)
-{
-    float lo, hi;
-    asm("{.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;}"
-        : "=f"(lo), "=f"(hi)
-        : "r"(h));
-    return f32x2(lo, hi);
-}
-// maximum of three (one instruction)
-__device__ __forceinline__ float max3(float a, float b, float c)
-{
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format: version 1).
@@ -577,9 +517,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 float sv[64];
                 load_half(h, vis, full, sv);
 #pragma unroll
-                for (int c = 0; c < 64; c += 8)
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) mx4[k] = max3(mx4[k], sv[c + 2 * k], sv[c + 2 * k + 1]);
+                for (int c = 0; c < 64; c += 4) {
+                    mx4[0] = fmaxf(mx4[0], sv[c]);
+                    mx4[1] = fmaxf(mx4[1], sv[c + 1]);
+                    mx4[2] = fmaxf(mx4[2], sv[c + 2]);
+                    mx4[3] = fmaxf(mx4[3], sv[c + 3]);
+                }
             }
             const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
             // S_t(j) was issued after P V_t(j-1) finished and P V_t(j) waits for
@@ -611,37 +554,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (!ok) break;
             }
             // pass 2: fp16 weights packed in pairs into the first 64 columns of
-            // S_t (half h -> columns 32h ..; those S columns are already read).
-            // Exponents scale*s - mu in fp32 two at a time, rounded to an fp16
-            // pair and raised with one fp16-pair exp2 (half the MUFU work; the
-            // weights are fp16 for the P V product anyway); the denominator sums
-            // those same fp16 weights in fp32.
-            uint64_t ps2[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
-            const uint64_t sl2x2 = f32x2(sl2, sl2), nmu2 = f32x2(-mu, -mu);
+            // S_t (half h -> columns 32h ..; those S columns are already read)
+            float ps4[4] = {0.f, 0.f, 0.f, 0.f};
             for (int h = 0; h < 2; ++h) {
                 float sv[64];
                 load_half(h, vis, full, sv);
-                uint32_t pw[32];
+                float pw[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    float x0, x1;
-                    f32x2_split(fma_f32x2(f32x2(sv[2 * e], sv[2 * e + 1]), sl2x2, nmu2), x0, x1);
-                    pw[e] = ex2_f16x2(cvt_f16x2(x0, x1));
+                    const float a = ex2(fmaf(sv[2 * e], sl2, -mu));
+                    const float bq = ex2(fmaf(sv[2 * e + 1], sl2, -mu));
+                    ps4[e & 3] += a + bq;
+                    pw[e] = __uint_as_float(pack_half2(a, bq));
                 }
-#pragma unroll
-                for (int e = 0; e < 32; e += 2)
-                    ps2[(e >> 1) & 1] = add_f32x2(ps2[(e >> 1) & 1], f16x2_to_f32x2(add_f16x2(pw[e], pw[e + 1])));
-                float pf[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) pf[e] = __uint_as_float(pw[e]);
-                tmem_st32(lane_base + s_col + 32 * h, pf);
+                tmem_st32(lane_base + s_col + 32 * h, pw);
             }
-            {
-                float a0, a1, b0, b1;
-                f32x2_split(ps2[0], a0, a1);
-                f32x2_split(ps2[1], b0, b1);
-                l += (a0 + a1) + (b0 + b1);
-            }
+            l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
             __syncwarp();
             if (lane == 0) mbar_arrive(turn(1 - t));  // the other tile's exp turn
             // V rows past the staged tokens must be finite zeros for the MMA
