@@ -229,7 +229,7 @@ int paged_kv_copy_blocks_q8k(void* kq_pool, void* v_pool, const int32_t* pairs, 
  * K pool: scores use key t = code * k_scales[kvh][:].  The scales are folded
  * into q once per (sequence, kv head) segment (q_d * k_scales[d], rounded to
  * fp16); codes are exact fp16 integers, so the products stay exact in fp32.
- * Requires head_dim 128; k_scales device, 8-byte aligned; workspace as for
+ * Requires head_dim 128; k_scales device, 16-byte aligned; workspace as for
  * paged_attention_workspace_size.  Otherwise as paged_verify_attention. */
 int paged_attention_q8k(const void* q, const void* kq_pool, const float* k_scales,
                         const void* v_pool, const int32_t* block_tables, int32_t max_blocks_per_seq,

@@ -121,12 +121,17 @@ struct Cfg {
     static constexpr int QROW = D * 2 + 16;
     static constexpr int Q_BYTES = (RP * QROW + 1023) / 1024 * 1024;
     static constexpr int Q_OFF = K_BYTES + KV_BYTES;
+    // int8 keys: the segment's channel scales (D fp32) follow the query rows
+    static constexpr int SC_OFF = Q_OFF + RP * QROW;
+    static_assert(!KQ || RP * QROW + D * 4 <= Q_BYTES, "room for the channel scales");
     static constexpr int STAGE_BYTES = Q_OFF + Q_BYTES;
     // floats per obuf row (the transposed consumer's scalar stores of rows
     // 2*tig, 2*tig+1 are conflict-free when 2 * OB_STRIDE = 8 mod 32)
     static constexpr int OB_STRIDE = NR8 ? D + 4 : D + 8;
     static constexpr int OBUF_SLICE = RP * OB_STRIDE;               // floats
-    static constexpr int OBUF_BYTES = 2 * OBUF_SLICE * 4;           // two merge slices
+    // two merge slices (the transposed consumer merges in the stage it just
+    // consumed instead: one slice per token warp, see consumer_tc)
+    static constexpr int OBUF_BYTES = NR8 ? 0 : 2 * OBUF_SLICE * 4;
     static constexpr int ML_BYTES = TW * RP * 2 * 4;
     // CTA copy of the query rows (read again every stage)
     static constexpr bool QPERSIST = NR8 ? NR8 > 2 : MT > 1;
@@ -146,6 +151,7 @@ struct Cfg {
     static constexpr int OBUF_OFF = ML_OFF + ML_BYTES;
     static constexpr int QP_OFF = OBUF_OFF + OBUF_BYTES;
     static constexpr int SMEM_USED = QP_OFF + QP_BYTES;
+    static_assert(!NR8 || TW * OBUF_SLICE * 4 <= STAGE_BYTES, "per-warp merge slices fit a stage");
     static constexpr int SMEM_ALLOC = SMEM_USED + 1024;    // room to align the base
 };
 
@@ -247,28 +253,6 @@ __device__ __forceinline__ void k8_frag(uint32_t st, int t0, int ks, int tig, ui
 {
     i8x4_to_h2x2_biased(lds_u32(st + tile_chunk_k8<C>(t0, ks) + 4 * tig), b0, b1);
     i8x4_to_h2x2_biased(lds_u32(st + tile_chunk_k8<C>(t0 + 8, ks) + 4 * tig), b2, b3);
-}
-
-// q fragments (rows r and r + 8) of an int8-K segment in the permuted dim
-// order of k8_frag, times the channel scales; adds this lane's share of each
-// row's sum of the (rounded) fp16 entries to rsum.
-template <class C>
-__device__ __forceinline__ void q8_frags(const uint8_t* qrow_r, const uint8_t* qrow_r8,
-                                         const float* sc, int tig, uint32_t (&qa)[C::D / 16][4],
-                                         float (&rsum)[2])
-{
-#pragma unroll
-    for (int ks = 0; ks < C::D / 16; ++ks) {
-        const int d = 16 * ks + 4 * tig;
-        const float2 s01 = *reinterpret_cast<const float2*>(sc + d);
-        const float2 s23 = *reinterpret_cast<const float2*>(sc + d + 2);
-        qa[ks][0] = scale_h2(*reinterpret_cast<const uint32_t*>(qrow_r + d * 2), s01);
-        qa[ks][1] = scale_h2(*reinterpret_cast<const uint32_t*>(qrow_r8 + d * 2), s01);
-        qa[ks][2] = scale_h2(*reinterpret_cast<const uint32_t*>(qrow_r + d * 2 + 4), s23);
-        qa[ks][3] = scale_h2(*reinterpret_cast<const uint32_t*>(qrow_r8 + d * 2 + 4), s23);
-        rsum[0] += h2_sum(qa[ks][0]) + h2_sum(qa[ks][2]);
-        rsum[1] += h2_sum(qa[ks][1]) + h2_sum(qa[ks][3]);
-    }
 }
 
 // One TMA copy of the tile whose first row is `y` in the pool's row space.
@@ -407,6 +391,19 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
         prefetch_tmap(tmK);
         prefetch_tmap(tmV);
     }
+    // Each CTA pulls an equal slice of the block tables into L2 while it
+    // scans the lengths, so the table reads that follow the scan (by
+    // whichever CTA) hit L2 instead of waiting on DRAM (and its page walk).
+    {
+        const uint64_t tbytes = (uint64_t)p.B * (uint64_t)p.max_blocks * 4u;
+        uint64_t chunk = (tbytes + gridDim.x - 1) / gridDim.x;
+        chunk = (chunk + 127) / 128 * 128;
+        if (chunk > 65536) chunk = 65536;
+        const uint64_t begin = (uint64_t)blockIdx.x * chunk;
+        const char* tb = reinterpret_cast<const char*>(p.block_tables);
+        for (uint64_t off = begin + (uint64_t)lane * 128; off < begin + chunk && off < tbytes; off += 32 * 128)
+            prefetch_l2(tb + off);
+    }
 
     // Pass 1: total units.  Each lane takes 8 consecutive sequences of a
     // 256-sequence chunk; all loads of a chunk are in flight together.
@@ -535,7 +532,7 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
                 const bool firstst = (d.flags & F_FIRST) != 0;
                 const uint32_t qbytes = (uint32_t)(p.G * C::D * 2);  // query bytes per window row
                 uint32_t bytes = (uint32_t)__popc(lmask) * (uint32_t)(C::K_TILE_BYTES + C::TILE_BYTES);
-                if (firstst) bytes += qbytes * (uint32_t)p.q_len;
+                if (firstst) bytes += qbytes * (uint32_t)p.q_len + (C::KQ ? C::D * 4 : 0);
                 const uint32_t full = full0 + stage * 8;
                 if (lane == 0) {
                     StageMeta& md = smeta[stage];
@@ -565,6 +562,8 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
                         p.q + (((int64_t)d.s * p.q_len + j) * p.Hq + (int64_t)d.kvh * p.G + g) * C::D;
                     bulk_load(st + C::Q_OFF + lane * C::QROW, src, C::D * 2, full);
                 }
+                if (C::KQ && firstst && lane == 31)  // the KV head's channel scales
+                    bulk_load(st + C::SC_OFF, p.k_scale + (int64_t)d.kvh * C::D, C::D * 4, full);
                 ++k_issued;
             }
 #pragma unroll
@@ -671,6 +670,57 @@ __device__ void store_segment(const Params& p, const StageMeta& md, const float*
     }
 }
 
+// Output of a finished segment from TW per-warp slices (each warp's o
+// already scaled by its factor), summed in warp order (bit-reproducible):
+// fp16 output (whole segment) or fp32 partials.
+template <class C>
+__device__ void store_segment_slices(const Params& p, const StageMeta& md, const float* slices,
+                                     const float* mlb, int tid)
+{
+    const int rows = p.rows;
+    const bool whole = (md.flags & F_WHOLE) != 0;
+    const int64_t pbase = ((int64_t)blockIdx.x * 2 + md.slot) * C::RP;
+    for (int idx = tid; idx < rows * (C::D / 8); idx += C::NCW * 32) {
+        const int R = idx / (C::D / 8);
+        const int d0 = (idx % (C::D / 8)) * 8;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+#pragma unroll
+        for (int w = 0; w < C::TW; ++w) {
+            const float4* src = reinterpret_cast<const float4*>(slices + (w * C::RP + R) * C::OB_STRIDE + d0);
+            const float4 x = src[0], y = src[1];
+            a = make_float4(a.x + x.x, a.y + x.y, a.z + x.z, a.w + x.w);
+            b = make_float4(b.x + y.x, b.y + y.y, b.z + y.z, b.w + y.w);
+        }
+        if (whole) {
+            const int j = R / p.G, g = R % p.G;
+            uint4 v;
+            v.x = pack_half2(a.x, a.y);
+            v.y = pack_half2(a.z, a.w);
+            v.z = pack_half2(b.x, b.y);
+            v.w = pack_half2(b.z, b.w);
+            __half* dst = p.out + (((int64_t)md.s * p.q_len + j) * p.Hq + (int64_t)md.kvh * p.G + g) * C::D + d0;
+            *reinterpret_cast<uint4*>(dst) = v;
+        } else {
+            float4* dst = reinterpret_cast<float4*>(p.part_o + (pbase + R) * C::D + d0);
+            dst[0] = a;
+            dst[1] = b;
+        }
+    }
+    if (!whole) {
+        for (int R = tid; R < rows; R += C::NCW * 32) {
+            float M = kNegInf;
+#pragma unroll
+            for (int w = 0; w < C::TW; ++w) M = fmaxf(M, mlb[(w * C::RP + R) * 2]);
+            const float Mu = M == kNegInf ? 0.f : M;
+            float Ls = 0.f;
+#pragma unroll
+            for (int w = 0; w < C::TW; ++w)
+                Ls += mlb[(w * C::RP + R) * 2 + 1] * ex2(mlb[(w * C::RP + R) * 2] - Mu);
+            p.part_lse[pbase + R] = Ls > 0.f ? Mu + lg2(Ls) : kNegInf;
+        }
+    }
+}
+
 // Combine the token-warps' (m, l) for row R; returns this warp's factor
 // 2^(m_w - M) / sum.
 template <class C>
@@ -685,228 +735,6 @@ __device__ __forceinline__ float row_factor(const float* mlb, int R, float m_w)
     for (int w = 0; w < C::TW; ++w)
         Ls += mlb[(w * C::RP + R) * 2 + 1] * ex2(mlb[(w * C::RP + R) * 2] - Mu);
     return Ls > 0.f ? ex2(m_w - Mu) / Ls : 0.f;
-}
-
-// ---------------------------------------------------------------------------
-// Tensor-core consumer: rows = GQA group x window (1 < rows <= 16*MT).
-template <class C>
-__device__ void consumer_mma(const Params& p, uint8_t* smem, volatile int* abort_flag)
-{
-    const int cw = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int mt = cw / C::TW, qw = cw % C::TW;
-    const int gid = lane >> 2, tig = lane & 3;
-    const uint32_t sbase = smem_u32(smem);
-    const StageMeta* smeta = reinterpret_cast<const StageMeta*>(smem + C::META_OFF);
-    const uint32_t full0 = sbase + C::BAR_OFF;
-    const uint32_t empty0 = full0 + C::STAGES * 8;
-    const uint32_t zero_row = sbase + C::ZERO_OFF;
-    float* mlb = reinterpret_cast<float*>(smem + C::ML_OFF);
-    float* obuf = reinterpret_cast<float*>(smem + C::OBUF_OFF);
-    const float sl2 = p.scale_log2;
-
-    // per-lane ldmatrix geometry
-    const int k_tok = qw * 16 + (lane >> 4) * 8 + (lane & 7);   // K: token of this lane's row
-    const int k_sel = (lane >> 3) & 1;                          // K: chunk select
-    const int v_i = ((lane >> 3) & 1) * 8 + (lane & 7);         // V: token within my 16
-    const int v_tok = qw * 16 + v_i;
-    const int v_sel = lane >> 4;
-
-    float O[C::D / 8][4];
-    uint32_t qa[C::D / 16][4];
-    float m[2], l[2];
-    float corr[2] = {0.f, 0.f};  // int8 keys: bias * row sum of q
-    int lim[2];
-
-    int stage = 0;
-    uint32_t phase = 0;
-    for (;;) {
-        if (!mbar_wait_bounded(full0 + stage * 8, phase, kWaitLimitNs)) {
-            *abort_flag = 1;
-            break;
-        }
-        const StageMeta md = smeta[stage];
-        if (md.flags & F_END) break;
-        const uint32_t st = sbase + stage * C::STAGE_BYTES;
-        if (md.flags & F_FIRST) {
-            // A fragments of this warp's 16 query rows: matrices (rows 0-7 | 8-15)
-            // x (columns 16ks.. | 16ks+8..), one padded row address per lane
-            const uint32_t qrow = st + C::Q_OFF +
-                                  (mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * C::QROW;
-            const int r0 = mt * 16 + gid;
-            if constexpr (!C::KQ) {
-#pragma unroll
-                for (int ks = 0; ks < C::D / 16; ++ks)
-                    ldsm_x4(qrow + ((2 * ks + (lane >> 4)) << 4), qa[ks][0], qa[ks][1], qa[ks][2],
-                            qa[ks][3]);
-            } else {
-                // int8 keys: q fragments in the permuted dim order, times the
-                // channel scales; bias correction from the row sums
-                const uint8_t* qr = smem + stage * C::STAGE_BYTES + C::Q_OFF + (mt * 16 + gid) * C::QROW;
-                float rs[2] = {0.f, 0.f};
-                q8_frags<C>(qr, qr + 8 * C::QROW, p.k_scale + (int64_t)md.kvh * C::D, tig, qa, rs);
-#pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    rs[rr] += __shfl_xor_sync(0xffffffffu, rs[rr], 1);
-                    rs[rr] += __shfl_xor_sync(0xffffffffu, rs[rr], 2);
-                    corr[rr] = kCodeBias * rs[rr];
-                }
-            }
-#pragma unroll
-            for (int n = 0; n < C::D / 8; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.f;
-            m[0] = m[1] = kNegInf;
-            l[0] = l[1] = 0.f;
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                const int R = r0 + rr * 8;
-                lim[rr] = R < p.rows ? md.L - p.q_len + R / p.G + 1 : md.L;
-            }
-        }
-        const int nv = md.ntok - qw * 16;
-        if (nv > 0) {
-            // S = q K^T for my 16 tokens (two n8 tiles)
-            // (even and odd k-steps accumulate separately: half the chain length)
-            float S[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            float T[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-            for (int ks = 0; ks < C::D / 16; ++ks) {
-                uint32_t b0, b1, b2, b3;
-                if constexpr (C::KQ)
-                    k8_frag<C>(st, qw * 16 + gid, ks, tig, b0, b1, b2, b3);
-                else
-                    ldsm_x4(st + tile_chunk<C>(k_tok, 2 * ks + k_sel), b0, b1, b2, b3);
-                if (ks & 1) {
-                    mma_16816(T[0], qa[ks], b0, b1);
-                    mma_16816(T[1], qa[ks], b2, b3);
-                } else {
-                    mma_16816(S[0], qa[ks], b0, b1);
-                    mma_16816(S[1], qa[ks], b2, b3);
-                }
-            }
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) S[nt][c] += T[nt][c] - (C::KQ ? corr[c >> 1] : 0.f);
-            // a token counts if its row may see it and this stage loaded it
-            // (with 8-token blocks a warp's second block can lie past the run)
-            const int pos0 = md.t0 + qw * 16 + tig * 2;
-            const int st_end = md.t0 + md.ntok;
-            const int lim0 = min(lim[0], st_end), lim1 = min(lim[1], st_end);
-            float mx[2] = {kNegInf, kNegInf};
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int pos = pos0 + nt * 8 + (c & 1);
-                    const float v = pos < ((c >> 1) ? lim1 : lim0) ? S[nt][c] * sl2 : kNegInf;
-                    S[nt][c] = v;
-                    mx[c >> 1] = fmaxf(mx[c >> 1], v);
-                }
-            float alpha[2], mu[2];
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
-                mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
-                const float mn = fmaxf(m[rr], mx[rr]);
-                mu[rr] = mn == kNegInf ? 0.f : mn;
-                alpha[rr] = ex2(m[rr] - mu[rr]);
-                m[rr] = mn;
-            }
-            float ps[2] = {0.f, 0.f};
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float e = ex2(S[nt][c] - mu[c >> 1]);
-                    S[nt][c] = e;
-                    ps[c >> 1] += e;
-                }
-            l[0] = l[0] * alpha[0] + ps[0];
-            l[1] = l[1] * alpha[1] + ps[1];
-            if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
-#pragma unroll
-                for (int n = 0; n < C::D / 8; ++n) {
-                    O[n][0] *= alpha[0];
-                    O[n][1] *= alpha[0];
-                    O[n][2] *= alpha[1];
-                    O[n][3] *= alpha[1];
-                }
-            }
-            uint32_t pa[4];
-            pa[0] = pack_half2(S[0][0], S[0][1]);
-            pa[1] = pack_half2(S[0][2], S[0][3]);
-            pa[2] = pack_half2(S[1][0], S[1][1]);
-            pa[3] = pack_half2(S[1][2], S[1][3]);
-            // rows of V past the valid tokens read a zero row instead
-            const bool v_ok = v_i < nv;
-#pragma unroll
-            for (int np = 0; np < C::D / 16; ++np) {
-                const uint32_t addr =
-                    v_ok ? st + C::V_OFF + tile_chunk<C>(v_tok, 2 * np + v_sel) : zero_row;
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_trans(addr, b0, b1, b2, b3);
-                mma_16816(O[2 * np], pa, b0, b1);
-                mma_16816(O[2 * np + 1], pa, b2, b3);
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty0 + stage * 8);
-
-        if (md.flags & F_LAST) {
-            // merge the token-warps of each m-tile (fixed order), then store
-            const int tid = threadIdx.x;
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                float lr = l[rr];
-                lr += __shfl_xor_sync(0xffffffffu, lr, 1);
-                lr += __shfl_xor_sync(0xffffffffu, lr, 2);
-                if (tig == 0) {
-                    const int R = mt * 16 + gid + rr * 8;
-                    mlb[(qw * C::RP + R) * 2] = m[rr];
-                    mlb[(qw * C::RP + R) * 2 + 1] = lr;
-                }
-            }
-            named_bar_sync(1, C::NCW * 32);
-            float f[2];
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) f[rr] = row_factor<C>(mlb, mt * 16 + gid + rr * 8, m[rr]);
-            // token-warps 0 and 1 write slices 0 and 1, then each later pair adds to them
-            const bool row0 = mt * 16 + gid < p.rows, row1 = mt * 16 + gid + 8 < p.rows;
-            float* slice = obuf + (qw & 1) * C::OBUF_SLICE;
-            float* r0p = slice + (mt * 16 + gid) * C::OB_STRIDE + tig * 2;
-            float* r1p = r0p + 8 * C::OB_STRIDE;
-            for (int round = 0; round < C::TW / 2; ++round) {
-                if ((qw >> 1) == round) {
-                    // round 1 adds to round 0's values: read them all first so the
-                    // loads pipeline instead of waiting behind each store
-                    float2 x0[C::D / 8], x1[C::D / 8];
-#pragma unroll
-                    for (int n = 0; n < C::D / 8; ++n) {
-                        x0[n] = make_float2(0.f, 0.f);
-                        x1[n] = make_float2(0.f, 0.f);
-                        if (round && row0) x0[n] = *reinterpret_cast<const float2*>(r0p + n * 8);
-                        if (round && row1) x1[n] = *reinterpret_cast<const float2*>(r1p + n * 8);
-                    }
-#pragma unroll
-                    for (int n = 0; n < C::D / 8; ++n) {
-                        if (row0)
-                            *reinterpret_cast<float2*>(r0p + n * 8) =
-                                make_float2(x0[n].x + O[n][0] * f[0], x0[n].y + O[n][1] * f[0]);
-                        if (row1)
-                            *reinterpret_cast<float2*>(r1p + n * 8) =
-                                make_float2(x1[n].x + O[n][2] * f[1], x1[n].y + O[n][3] * f[1]);
-                    }
-                }
-                named_bar_sync(1, C::NCW * 32);
-            }
-            store_segment<C>(p, md, obuf, mlb, tid);
-            named_bar_sync(1, C::NCW * 32);
-        }
-        if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1;
-        }
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -973,7 +801,7 @@ __device__ void consumer_fma(const Params& p, uint8_t* smem, volatile int* abort
                 qh[h][2] = v.z;
                 qh[h][3] = v.w;
                 if constexpr (C::KQ) {  // fold the channel scales of the int8 keys into q
-                    const float* sc = p.k_scale + (int64_t)md.kvh * C::D + d0;
+                    const float* sc = reinterpret_cast<const float*>(st + C::SC_OFF) + d0;
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         qh[h][e] = scale_h2(qh[h][e], *reinterpret_cast<const float2*>(sc + 2 * e));
@@ -1172,7 +1000,7 @@ __device__ void consumer_mma_mt(const Params& p, uint8_t* smem, volatile int* ab
                 // stored in the permuted order of k8_frag (dims 0,1,4,5,8,9,12,13
                 // then 2,3,6,7,10,11,14,15), so ldmatrix yields matching fragments
                 constexpr int CPR = C::QROW / 16;  // 16-byte chunks per row
-                const float* sc = p.k_scale + (int64_t)md.kvh * C::D;
+                const float* sc = reinterpret_cast<const float*>(smem + stage * C::STAGE_BYTES + C::SC_OFF);
                 for (int i = threadIdx.x; i < C::RP * (C::D / 16); i += C::NCW * 32) {
                     const int row = i / (C::D / 16), ks = i % (C::D / 16);
                     const uint4 a = src[row * CPR + 2 * ks], b = src[row * CPR + 2 * ks + 1];
@@ -1395,7 +1223,6 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
     const uint32_t empty0 = full0 + C::STAGES * 8;
     const uint32_t zero_row = sbase + C::ZERO_OFF;
     float* mlb = reinterpret_cast<float*>(smem + C::ML_OFF);
-    float* obuf = reinterpret_cast<float*>(smem + C::OBUF_OFF);
     const float sl2 = p.scale_log2;
 
     // ldmatrix lane geometry.  K as the A operand: matrices (tokens 0-7 |
@@ -1442,7 +1269,7 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
                     // q times the channel scales, each 16-dim chunk stored in the
                     // permuted order of the int8 key fragments (dims 0,1,4,5,8,9,
                     // 12,13 then 2,3,6,7,10,11,14,15)
-                    const float* sc = p.k_scale + (int64_t)md.kvh * C::D;
+                    const float* sc = reinterpret_cast<const float*>(smem + stage * C::STAGE_BYTES + C::SC_OFF);
                     for (int i = threadIdx.x; i < C::RP * KS; i += C::NCW * 32) {
                         const int row = i / KS, ks = i % KS;
                         const uint4 a = src[row * CPR + 2 * ks], b = src[row * CPR + 2 * ks + 1];
@@ -1473,7 +1300,7 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
             } else {
                 // int8 keys: q of row nt*8+gid times the channel scales, in the
                 // permuted dim order (lane tig: dims 4tig, 4tig+1 | 4tig+2, 4tig+3)
-                const float* sc = p.k_scale + (int64_t)md.kvh * C::D;
+                const float* sc = reinterpret_cast<const float*>(smem + stage * C::STAGE_BYTES + C::SC_OFF);
 #pragma unroll
                 for (int nt = 0; nt < NR; ++nt) {
                     const uint8_t* qr = smem + stage * C::STAGE_BYTES + C::Q_OFF + (nt * 8 + gid) * C::QROW;
@@ -1641,10 +1468,13 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
         }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(empty0 + stage * 8);
-
-        if (md.flags & F_LAST) {
-            // merge the token-warps (fixed order), then store
+        if (!(md.flags & F_LAST)) {
+            if (lane == 0) mbar_arrive(empty0 + stage * 8);
+        } else {
+            // Segment end: merge the token-warps.  The stage just consumed is
+            // kept (not yet released) and its shared memory holds one slice per
+            // warp: each warp writes its o scaled by 2^(m_w - M) / L, then one
+            // pass sums the slices in warp order and stores.
             const int tid = threadIdx.x;
 #pragma unroll
             for (int nt = 0; nt < NR; ++nt)
@@ -1660,46 +1490,29 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
                         mlb[(qw * C::RP + R) * 2 + 1] = lr;
                     }
                 }
-            named_bar_sync(1, C::NCW * 32);
-            float f[NR][2];
+            named_bar_sync(1, C::NCW * 32);  // every warp done with the stage's tiles
+            float* slices = reinterpret_cast<float*>(smem + stage * C::STAGE_BYTES);
 #pragma unroll
-            for (int nt = 0; nt < NR; ++nt)
+            for (int nt = 0; nt < NR; ++nt) {
+                const float f0 = row_factor<C>(mlb, nt * 8 + 2 * tig, m[nt][0]);
+                const float f1 = row_factor<C>(mlb, nt * 8 + 2 * tig + 1, m[nt][1]);
+                float* r0 = slices + (qw * C::RP + nt * 8 + 2 * tig) * C::OB_STRIDE + gid;
+                float* r1 = r0 + C::OB_STRIDE;
 #pragma unroll
-                for (int i = 0; i < 2; ++i) f[nt][i] = row_factor<C>(mlb, nt * 8 + 2 * tig + i, m[nt][i]);
-            // token-warps 0 and 1 write slices 0 and 1, then each later pair adds to them
-            float* slice = obuf + (qw & 1) * C::OBUF_SLICE;
-            for (int round = 0; round < C::TW / 2; ++round) {
-                if ((qw >> 1) == round) {
-#pragma unroll
-                    for (int nt = 0; nt < NR; ++nt) {
-                        float* r0 = slice + (nt * 8 + 2 * tig) * C::OB_STRIDE + gid;
-                        float* r1 = r0 + C::OB_STRIDE;
-                        const bool ok0 = nt * 8 + 2 * tig < p.rows, ok1 = nt * 8 + 2 * tig + 1 < p.rows;
-                        float x[KS][4];  // loads first, then stores
-#pragma unroll
-                        for (int np = 0; np < KS; ++np) {
-                            x[np][0] = round && ok0 ? r0[16 * np] : 0.f;
-                            x[np][1] = round && ok1 ? r1[16 * np] : 0.f;
-                            x[np][2] = round && ok0 ? r0[16 * np + 8] : 0.f;
-                            x[np][3] = round && ok1 ? r1[16 * np + 8] : 0.f;
-                        }
-#pragma unroll
-                        for (int np = 0; np < KS; ++np) {
-                            if (ok0) {
-                                r0[16 * np] = x[np][0] + O[np][nt][0] * f[nt][0];
-                                r0[16 * np + 8] = x[np][2] + O[np][nt][2] * f[nt][0];
-                            }
-                            if (ok1) {
-                                r1[16 * np] = x[np][1] + O[np][nt][1] * f[nt][1];
-                                r1[16 * np + 8] = x[np][3] + O[np][nt][3] * f[nt][1];
-                            }
-                        }
-                    }
+                for (int np = 0; np < KS; ++np) {
+                    r0[16 * np] = O[np][nt][0] * f0;
+                    r1[16 * np] = O[np][nt][1] * f1;
+                    r0[16 * np + 8] = O[np][nt][2] * f0;
+                    r1[16 * np + 8] = O[np][nt][3] * f1;
                 }
-                named_bar_sync(1, C::NCW * 32);
             }
-            store_segment<C>(p, md, obuf, mlb, tid);
             named_bar_sync(1, C::NCW * 32);
+            store_segment_slices<C>(p, md, slices, mlb, tid);
+            // the slices and mlb are read: the stage may be refilled (by the
+            // async proxy, after these generic accesses) and mlb rewritten
+            fence_proxy_async();
+            named_bar_sync(1, C::NCW * 32);
+            if (lane == 0) mbar_arrive(empty0 + stage * 8);
         }
         if (++stage == C::STAGES) {
             stage = 0;
@@ -1747,10 +1560,9 @@ __global__ void __maxnreg__(C::MAXREG)
         consumer_fma<C>(p, smem, &abort_flag);
     } else if constexpr (C::NR8 > 0) {
         consumer_tc<C>(p, smem, &abort_flag);
-    } else if constexpr (C::MT > 1) {
-        consumer_mma_mt<C>(p, smem, &abort_flag);
     } else {
-        consumer_mma<C>(p, smem, &abort_flag);
+        static_assert(C::MT > 1, "one row tile of more than one row uses the transposed consumer");
+        consumer_mma_mt<C>(p, smem, &abort_flag);
     }
 }
 
@@ -1984,8 +1796,8 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
     if (D != 64 && D != 128) return kv_fail(KV_ERR_INVALID, "paged attention: head_dim must be 64 or 128");
     if (k_scale && D != 128)
         return kv_fail(KV_ERR_INVALID, "paged attention: int8 K pools need head_dim 128");
-    if (k_scale && (reinterpret_cast<uintptr_t>(k_scale) & 7u))
-        return kv_fail(KV_ERR_INVALID, "paged attention: k_scales must be 8-byte aligned");
+    if (k_scale && (reinterpret_cast<uintptr_t>(k_scale) & 15u))
+        return kv_fail(KV_ERR_INVALID, "paged attention: k_scales must be 16-byte aligned");
     if (BS != 8 && BS != 16) return kv_fail(KV_ERR_INVALID, "paged attention: block_size must be 8 or 16");
     const int G = Hq / Hkv;
     const int rows = G * q_len;

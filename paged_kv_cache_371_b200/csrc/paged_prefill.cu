@@ -23,8 +23,9 @@
 // warp 9 TMEM allocation + MMA issue.  Tensor memory: S_t and O_t for both
 // tiles (512 columns).  S is single-buffered per tile (S_t(j+1) waits for
 // P V_t(j)); the two tiles ping-pong: while one tile is in its softmax the
-// other's MMAs run, and the tiles' exp2 passes take turns so that each has the
-// MUFU pipe to itself.  K and V arrive through separate two-slot rings
+// other's MMAs run.  The softmax does its fp32 arithmetic two values per
+// instruction (packed f32x2 multiply-add and add, three-input maximum).
+// K and V arrive through separate two-slot rings
 // (32 KB slots) shared by the tiles; the producer polls both rings and fills
 // whichever slot frees first.  The MMA warp issues in the one order in which
 // the tiles' work becomes ready (S_0 and S_1 of the first stage, then per
@@ -77,8 +78,8 @@ constexpr int K_OFF = Q_OFF + Q_BYTES;          // K ring
 constexpr int V_OFF = K_OFF + KV_SLOTS * SLOT_BYTES;  // V ring
 constexpr int BAR_OFF = V_OFF + KV_SLOTS * SLOT_BYTES;
 // barriers: q_full, kfull[KS], kempty[KS], vfull[KS], vempty[KS], per tile
-// s_full, s_free, p_full; drain; exp turn per tile
-constexpr int NBARS = 1 + 4 * KV_SLOTS + 3 * NT + 1 + NT;
+// s_full, s_free, p_full; drain
+constexpr int NBARS = 1 + 4 * KV_SLOTS + 3 * NT + 1;
 constexpr int TMEM_SLOT_OFF = BAR_OFF + NBARS * 8;
 constexpr int SMEM_USED = TMEM_SLOT_OFF + 16;
 constexpr int SMEM_ALLOC = SMEM_USED + 1024;
@@ -200,6 +201,37 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
         : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// ---- packed fp32 arithmetic of the softmax (two lanes of work per instruction)
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f32x2_split(uint64_t v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// maximum of three in one instruction
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format: version 1).
@@ -252,11 +284,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     auto s_free = [&](int t) { return bar0 + 8 * (2 + 4 * KV_SLOTS + 3 * t); };
     auto p_full = [&](int t) { return bar0 + 8 * (3 + 4 * KV_SLOTS + 3 * t); };
     const uint32_t drain = bar0 + 8 * (1 + 4 * KV_SLOTS + 3 * NT);
-    // exp turns: the two tiles' exponential passes alternate (tile 0 for
-    // stage j, tile 1 for stage j, tile 0 for stage j+1, ...) so that one tile
-    // has the MUFU pipe while the other's MMAs run.  turn(t) completes a
-    // phase when the other tile's four warps finished an exp pass.
-    auto turn = [&](int t) { return bar0 + 8 * (2 + 4 * KV_SLOTS + 3 * NT + t); };
 
     // work item: NT consecutive tiles of one (sequence, kv head)
     const int pair = blockIdx.x % p.tiles_per_head;
@@ -292,7 +319,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_init(p_full(t), 4);
         }
         mbar_init(drain, 1);
-        for (int t = 0; t < NT; ++t) mbar_init(turn(t), 4);
         fence_barrier_init();
     }
     if (warp == MMA_WARP) {
@@ -438,12 +464,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 umma_commit(s_free(t));
                 if (t == NT - 1) umma_commit(vempty(j % KV_SLOTS));  // V of stage j consumed
             };
-            // The softmax tiles take their exp turns in order, so the work
-            // becomes ready in one fixed order: S_0(0), S_1(0), then per stage
-            // j: P V_0(j), S_0(j+1), P V_1(j), S_1(j+1).  Issuing in that order
-            // with blocking waits wakes on each barrier as it completes; while
-            // one tile is in its softmax, the other's MMAs keep the tensor
-            // pipe busy.
+            // Issue order: S_0(0), S_1(0), then per stage j: P V_0(j),
+            // S_0(j+1), P V_1(j), S_1(j+1) (tile 0's softmax of a stage
+            // usually finishes first: its S was issued first).  Blocking waits
+            // wake on each barrier as it completes; while one tile is in its
+            // softmax, the other's MMAs keep the tensor pipe busy.
             if (ok && nst > 0) ok = mbar_wait_bounded(kfull(0), 0, kWait);
             if (ok && nst > 0) {
                 for (int t = 0; t < NT; ++t) issue_S(t, 0);
@@ -517,12 +542,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 float sv[64];
                 load_half(h, vis, full, sv);
 #pragma unroll
-                for (int c = 0; c < 64; c += 4) {
-                    mx4[0] = fmaxf(mx4[0], sv[c]);
-                    mx4[1] = fmaxf(mx4[1], sv[c + 1]);
-                    mx4[2] = fmaxf(mx4[2], sv[c + 2]);
-                    mx4[3] = fmaxf(mx4[3], sv[c + 3]);
-                }
+                for (int c = 0; c < 64; c += 8)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) mx4[k] = max3(mx4[k], sv[c + 2 * k], sv[c + 2 * k + 1]);
             }
             const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
             // S_t(j) was issued after P V_t(j-1) finished and P V_t(j) waits for
@@ -546,32 +568,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 m = mn;
             }
             const float mu = m == kNegInf ? 0.f : m;
-            // wait for this tile's exp turn: tile 0's pass of stage j follows
-            // tile 1's pass of stage j-1, tile 1's follows tile 0's of stage j.
-            // Neither side can run two phases ahead of the other.
-            if (t == 1 || j >= 1) {
-                ok = mbar_wait_bounded(turn(t), (t == 1 ? j : j - 1) & 1, kWait);
-                if (!ok) break;
-            }
             // pass 2: fp16 weights packed in pairs into the first 64 columns of
-            // S_t (half h -> columns 32h ..; those S columns are already read)
-            float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+            // S_t (half h -> columns 32h ..; those S columns are already read);
+            // the exponents scale*s - mu and the row sum two at a time
+            uint64_t ps2[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
+            const uint64_t sl2x2 = f32x2(sl2, sl2), nmu2 = f32x2(-mu, -mu);
             for (int h = 0; h < 2; ++h) {
                 float sv[64];
                 load_half(h, vis, full, sv);
                 float pw[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const float a = ex2(fmaf(sv[2 * e], sl2, -mu));
-                    const float bq = ex2(fmaf(sv[2 * e + 1], sl2, -mu));
-                    ps4[e & 3] += a + bq;
+                    float x0, x1;
+                    f32x2_split(fma_f32x2(f32x2(sv[2 * e], sv[2 * e + 1]), sl2x2, nmu2), x0, x1);
+                    const float a = ex2(x0), bq = ex2(x1);
+                    ps2[e & 1] = add_f32x2(ps2[e & 1], f32x2(a, bq));
                     pw[e] = __uint_as_float(pack_half2(a, bq));
                 }
                 tmem_st32(lane_base + s_col + 32 * h, pw);
             }
-            l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(turn(1 - t));  // the other tile's exp turn
+            {
+                float a0, a1, b0, b1;
+                f32x2_split(ps2[0], a0, a1);
+                f32x2_split(ps2[1], b0, b1);
+                l += (a0 + b0) + (a1 + b1);
+            }
             // V rows past the staged tokens must be finite zeros for the MMA
             // (tile 0 writes them; tile 1's P V is issued after tile 0's, which
             // waited for these writes).  The copy of this stage's V must have
