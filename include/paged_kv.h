@@ -319,7 +319,8 @@ int paged_prefill_attention(const void* q, const void* k_pool, const void* v_poo
  *                    (default), -1: plain launch;
  *   seg_cost_blocks  fixed cost, in blocks, charged to every (sequence,
  *                    kv-head) when work is divided among CTAs (default: 128
- *                    tokens' worth, 256 over an int8 K pool; -1 for none);
+ *                    tokens' worth, 256 over an int8 K pool with several
+ *                    query rows per KV head; -1 for none);
  *   producer_wait_ns limit, in nanoseconds, of the loading warp's waits for
  *                    a free pipeline stage (default 2 s; below 1000 the
  *                    loader gives up at the first stage that is not already
@@ -348,6 +349,19 @@ int paged_attention_ex(const void* q, const void* k_pool, const void* v_pool,
                        int32_t B, int32_t Hq, int32_t Hkv, int32_t head_dim, int32_t block_size,
                        int32_t num_blocks, void* workspace, size_t workspace_bytes,
                        const paged_attention_opts* opts, void* stream);
+
+/* paged_prefill_attention with launch knobs (opts may be NULL): only
+ * producer_wait_ns is read, as the limit of the loading warp's wait without
+ * progress (a free ring slot); below 1000 it gives up at the first wait.  On
+ * a give-up the kernel stops, sets KV_DEV_TIMEOUT and leaves the output
+ * undefined; the compute warps reach their own 2 s limits first, so the call
+ * returns within a few seconds; later calls are unaffected. */
+int paged_prefill_attention_ex(const void* q, const void* k_pool, const void* v_pool,
+                               const int32_t* block_tables, int32_t max_blocks_per_seq,
+                               const int32_t* context_lens, int32_t q_len, float scale, void* out,
+                               int32_t B, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                               int32_t block_size, int32_t num_blocks,
+                               const paged_attention_opts* opts, void* stream);
 
 /* paged_attention_q8k with the launch knobs of paged_attention_ex (opts may
  * be NULL: defaults). */

@@ -414,9 +414,10 @@ def paged_attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len=
 
 
 def paged_prefill_attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len,
-                            out=None):
+                            out=None, producer_wait_ns=0):
     """Causal chunked prefill over the paged cache (tensor cores): row j of
-    sequence s sees tokens 0 .. context_lens[s] - q_len + j."""
+    sequence s sees tokens 0 .. context_lens[s] - q_len + j.  producer_wait_ns:
+    the loading warp's wait limit, for failure-detection tests."""
     dev = k_pool.device
     for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool")):
         _need(t, n, torch.float16, dev)
@@ -432,11 +433,15 @@ def paged_prefill_attention(q, k_pool, v_pool, block_tables, context_lens, scale
     if out is None:
         out = torch.empty_like(q)
     _need(out, "out", torch.float16, dev)
-    check(_L.paged_prefill_attention(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
-                                     block_tables.data_ptr(), block_tables.shape[1],
-                                     context_lens.data_ptr(), q_len, float(scale), out.data_ptr(),
-                                     B, Hq, Hkv, D, bs, nb, _stream(dev)),
-          "paged_prefill_attention")
+    args = (q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_tables.data_ptr(),
+            block_tables.shape[1], context_lens.data_ptr(), q_len, float(scale), out.data_ptr(),
+            B, Hq, Hkv, D, bs, nb)
+    if producer_wait_ns:
+        o = _abi.PagedAttentionOpts(0, 0, 0, 0, producer_wait_ns)
+        check(_L.paged_prefill_attention_ex(*args, ctypes.byref(o), _stream(dev)),
+              "paged_prefill_attention_ex")
+    else:
+        check(_L.paged_prefill_attention(*args, _stream(dev)), "paged_prefill_attention")
     return out
 
 

@@ -79,6 +79,9 @@ SIGNATURES = {
     "paged_kv_append_q8k": ([_P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
     "paged_attention_q8k": ([_P, _P, _P, _P, _P, _i32, _P, _i32, ctypes.c_float, _P, _i32, _i32, _i32,
                              _i32, _i32, _i32, _P, _sz, _P], ctypes.c_int),
+    "paged_prefill_attention_ex": ([_P, _P, _P, _P, _i32, _P, _i32, ctypes.c_float, _P, _i32, _i32,
+                                    _i32, _i32, _i32, _i32, ctypes.POINTER(PagedAttentionOpts), _P],
+                                   ctypes.c_int),
     "paged_attention_q8k_ex": ([_P, _P, _P, _P, _P, _i32, _P, _i32, ctypes.c_float, _P, _i32, _i32,
                                 _i32, _i32, _i32, _i32, _P, _sz, ctypes.POINTER(PagedAttentionOpts),
                                 _P], ctypes.c_int),

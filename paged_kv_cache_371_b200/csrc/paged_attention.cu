@@ -53,7 +53,8 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kSmemBudget = 225 * 1024;
 // Fixed cost of a (sequence, kv-head) segment when work is divided among CTAs,
 // in tokens of K/V streaming (query load, merge, partial last stage): about
-// one 128-token stage, two for int8 keys (a third less bytes per token)
+// one 128-token stage, two for int8 keys on the tensor-core path (a third
+// less bytes per token, and the scaled query fragments to build)
 constexpr int kSegCostTokens = 128;
 constexpr int kSegCostTokensQ8 = 256;
 constexpr float kNegInf = -__builtin_huge_valf();
@@ -1850,7 +1851,7 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
     prm.num_blocks = num_blocks;
     prm.min_share = (opts && opts->min_split_blocks > 0) ? opts->min_split_blocks : 16;
     prm.seg_cost = (opts && opts->seg_cost_blocks != 0) ? (opts->seg_cost_blocks > 0 ? opts->seg_cost_blocks : 0)
-                                                        : (k_scale ? kSegCostTokensQ8 : kSegCostTokens) / BS;
+                                                        : (k_scale && rows > 1 ? kSegCostTokensQ8 : kSegCostTokens) / BS;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.slot_wait_ns = (opts && opts->producer_wait_ns > 0) ? (uint64_t)opts->producer_wait_ns
                                                             : kWaitLimitNs;

@@ -85,21 +85,23 @@ constexpr int SMEM_USED = TMEM_SLOT_OFF + 16;
 constexpr int SMEM_ALLOC = SMEM_USED + 1024;
 static_assert(SMEM_ALLOC <= 232448, "one CTA per SM must fit");
 
-// Progress watchdog for the producer's polling loop: true once kWait of wall
-// time has passed without progress (the clock is read every 1024 idle polls).
+// Progress watchdog for the producer's polling loop: true once `limit` ns of
+// wall time have passed without progress (the clock is read every 1024 idle
+// polls); a limit below kFineWaitNs expires at the first idle poll.
 struct Idle {
     uint32_t n = 0;
     uint64_t t0 = 0;
     __device__ __forceinline__ void reset() { n = 0; }
-    __device__ __forceinline__ bool expired()
+    __device__ __forceinline__ bool expired(uint64_t limit)
     {
+        if (limit < kFineWaitNs) return true;
         if ((++n & 1023u) != 0) return false;
         const uint64_t now = globaltimer_ns();
         if (n == 1024u) {
             t0 = now;
             return false;
         }
-        return now - t0 > kWait;
+        return now - t0 > limit;
     }
 };
 
@@ -111,6 +113,7 @@ struct Params {
     int* err;
     int32_t max_blocks, B, q_len, Hq, Hkv, G, bs, num_blocks, tiles_per_head;
     float scale_log2;
+    uint64_t idle_ns;  // the loader's limit without progress
 };
 
 // ---- tcgen05 wrappers --------------------------------------------------------
@@ -406,7 +409,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 continue;
             }
             if (__shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&abort_flag), 0) ||
-                __shfl_sync(0xffffffffu, idle.expired() ? 1 : 0, 0)) {
+                __shfl_sync(0xffffffffu, idle.expired(p.idle_ns) ? 1 : 0, 0)) {
                 ok = false;
                 break;
             }
@@ -695,12 +698,40 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 }  // namespace
 
+namespace {
+int prefill_impl(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_tables,
+                 int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t q_len, float scale,
+                 void* out, int32_t B, int32_t Hq, int32_t Hkv, int32_t head_dim, int32_t block_size,
+                 int32_t num_blocks, const paged_attention_opts* opts, void* stream);
+}
+
 extern "C" int paged_prefill_attention(const void* q, const void* k_pool, const void* v_pool,
                                        const int32_t* block_tables, int32_t max_blocks_per_seq,
                                        const int32_t* context_lens, int32_t q_len, float scale,
                                        void* out, int32_t B, int32_t Hq, int32_t Hkv,
                                        int32_t head_dim, int32_t block_size, int32_t num_blocks,
                                        void* stream)
+{
+    return prefill_impl(q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens, q_len, scale,
+                        out, B, Hq, Hkv, head_dim, block_size, num_blocks, nullptr, stream);
+}
+
+extern "C" int paged_prefill_attention_ex(const void* q, const void* k_pool, const void* v_pool,
+                                          const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                          const int32_t* context_lens, int32_t q_len, float scale,
+                                          void* out, int32_t B, int32_t Hq, int32_t Hkv,
+                                          int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                                          const paged_attention_opts* opts, void* stream)
+{
+    return prefill_impl(q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens, q_len, scale,
+                        out, B, Hq, Hkv, head_dim, block_size, num_blocks, opts, stream);
+}
+
+namespace {
+int prefill_impl(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_tables,
+                 int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t q_len, float scale,
+                 void* out, int32_t B, int32_t Hq, int32_t Hkv, int32_t head_dim, int32_t block_size,
+                 int32_t num_blocks, const paged_attention_opts* opts, void* stream)
 {
     if (B < 0 || q_len < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || num_blocks < 1 || max_blocks_per_seq < 1)
         return kv_fail(KV_ERR_INVALID, "paged_prefill_attention: bad sizes");
@@ -760,6 +791,7 @@ extern "C" int paged_prefill_attention(const void* q, const void* k_pool, const 
     prm.num_blocks = num_blocks;
     prm.tiles_per_head = groups;
     prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.idle_ns = (opts && opts->producer_wait_ns > 0) ? (uint64_t)opts->producer_wait_ns : kWait;
     static std::mutex amu;
     static unsigned long long configured = 0;
     int dev = 0;
@@ -778,3 +810,5 @@ extern "C" int paged_prefill_attention(const void* q, const void* k_pool, const 
                                                                                                 prm);
     return kv_cuda_check(cudaGetLastError(), "paged_prefill_attention launch");
 }
+
+}  // namespace

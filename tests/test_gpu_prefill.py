@@ -138,3 +138,27 @@ def test_prefill_chunk_full_size_whole_sequences():
     seqs = sorted({int(np.argmin(wl.lens)), int(np.argmax(wl.lens))})
     ref = oracle_subset(wl, seqs, q_len=q_len)
     assert_close(out[torch.as_tensor(seqs, device="cuda")], ref, "prefill_chunk full size")
+
+
+def test_prefill_loader_wait_limit_times_out_and_recovers():
+    """Failure detection without a fault: a 1 ns limit on the prefill loader's
+    wait for a free K/V slot makes it give up after the first stages; the MMA
+    and softmax warps reach their own bounded waits, tensor memory is
+    released, the call returns with KV_DEV_TIMEOUT in the device error word,
+    and the next ordinary launch is correct."""
+    import time
+    wl = make_workload("llama70b_gqa", "cuda", lens=np.array([1500, 900], np.int32), q_len=64,
+                       Hq=64, Hkv=8, D=128, seed=3)
+    bt, cl = device_inputs(wl)
+    pkv.paged_prefill_attention(wl.q, wl.k_pool, wl.v_pool, bt, cl, wl.scale, 64)  # warm
+    assert pkv.device_error() == 0
+    t0 = time.perf_counter()
+    pkv.paged_prefill_attention(wl.q, wl.k_pool, wl.v_pool, bt, cl, wl.scale, 64, producer_wait_ns=1)
+    err = pkv.device_error()
+    dt = time.perf_counter() - t0
+    assert err & pkv._abi.KV_DEV_TIMEOUT
+    assert dt < 20.0, f"a timed-out launch took {dt:.1f} s"
+    out = pkv.paged_prefill_attention(wl.q, wl.k_pool, wl.v_pool, bt, cl, wl.scale, 64)
+    torch.cuda.synchronize()
+    assert pkv.device_error() == 0
+    assert_close(out, oracle_subset(wl, [0, 1], q_len=64), "prefill after a timeout")
