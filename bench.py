@@ -57,6 +57,9 @@ def parse_args(argv=None):
                     help="skip the 70B GQA decode lines reported beside the default workload")
     ap.add_argument("--batch", type=int, default=0,
                     help="use only the first B sequences of the workload (profiling runs)")
+    ap.add_argument("--consumer", type=int, default=0, choices=[0, 1, 2],
+                    help="compute path for several query rows per KV head: 1 warp-level MMAs, "
+                         "2 tcgen05 with tensor-memory accumulators, 0 the library's default")
     return ap.parse_args(argv)
 
 
@@ -698,7 +701,8 @@ def measure_decode(args, workload, rank, world, local, device, full=True):
                            else "fp16"),
                 "l2": f"flushed before every timed step by reading {flush.bytes >> 20} MiB "
                       "(a sum into one word: no dirty lines left)",
-                "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                "consumer": consumer_path(Hq // Hkv * q_len, D, q8k)},
             "hbm_frac": round(value / peak, 4),
             "hbm_peak_gbs": peak, "hbm_peak_kind": peak_kind,
             "tokens_heads_per_s": round(th_all / (t_all * 1e-3), 1),
@@ -734,6 +738,20 @@ def measure_decode(args, workload, rank, world, local, device, full=True):
     return result
 
 
+CONSUMER = 0  # --consumer (0: the library's default path)
+
+
+def consumer_path(rows, D, q8k):
+    """Which compute path the attention launch takes (mirrors the library's
+    default choice: the warp-level MMAs unless --consumer 2)."""
+    if rows == 1:
+        return "fma (one query row per KV head)"
+    if D != 128:
+        return "mma.sync"
+    c = CONSUMER or 1
+    return "tcgen05 (tensor memory)" if c == 2 else "mma.sync"
+
+
 def decode_step(pkv, wl, q, k_new, v_new, slots, tables, lens, pairs, out, ws, q_len, kq, ksc,
                 ev=None, stream=None):
     """One decode step through the public API: copy-on-write copies, append
@@ -750,7 +768,10 @@ def decode_step(pkv, wl, q, k_new, v_new, slots, tables, lens, pairs, out, ws, q
         ev.record(stream)
     if kq is not None:
         pkv.paged_attention_q8k(q, kq, ksc, wl.v_pool, tables, lens, wl.scale, q_len, out=out,
-                                workspace=ws)
+                                workspace=ws, consumer=CONSUMER)
+    elif CONSUMER:
+        pkv.paged_attention(q, wl.k_pool, wl.v_pool, tables, lens, wl.scale, q_len, out=out,
+                            workspace=ws, consumer=CONSUMER)
     elif q_len == 1:
         pkv.paged_decode_attention(q, wl.k_pool, wl.v_pool, tables, lens, wl.scale, out=out,
                                    workspace=ws)
@@ -1078,7 +1099,9 @@ def run_reference_prefill(args, base, spec, world):
 
 
 def main(argv=None):
+    global CONSUMER
     args = parse_args(argv)
+    CONSUMER = args.consumer
     from workloads.synth import CONFIGS
     if args.impl == "reference":
         res = run_reference(args)

@@ -333,14 +333,21 @@ int paged_prefill_attention(const void* q, const void* k_pool, const void* v_poo
  *                    the call still returns and later calls are unaffected.
  *                    The compute warps' waits keep the default limit (they
  *                    meet at a barrier at the end of every sequence, so they
- *                    must all stop at the same stage). */
+ *                    must all stop at the same stage);
+ *   consumer         the compute path for more than one query row per KV
+ *                    head at head_dim 128: 1 = warp-level tensor-core MMAs
+ *                    (mma.sync, accumulators in registers), 2 = tcgen05 MMAs
+ *                    with accumulators in tensor memory, 0 = default (the
+ *                    warp-level MMAs).  Both compute the same attention;
+ *                    other values are rejected with KV_ERR_INVALID. */
 typedef struct paged_attention_opts {
     int32_t grid_ctas;
     int32_t min_split_blocks;
     int32_t use_pdl;
     int32_t seg_cost_blocks;
     int32_t producer_wait_ns;
-    int32_t reserved[3];
+    int32_t consumer;
+    int32_t reserved[2];
 } paged_attention_opts;
 
 int paged_attention_ex(const void* q, const void* k_pool, const void* v_pool,

@@ -283,7 +283,7 @@ def workspace_size(Hq: int, Hkv: int, q_len: int, head_dim: int, grid_ctas: int 
 
 def _attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len, out, workspace,
                grid_ctas, min_split_blocks, use_pdl, entry, seg_cost_blocks=0, k_scales=None,
-               producer_wait_ns=0):
+               producer_wait_ns=0, consumer=0):
     dev = k_pool.device
     _need(k_pool, "k_pool", torch.int8 if entry == "q8k" else torch.float16, dev)
     for t, n in ((q, "q"), (v_pool, "v_pool")):
@@ -322,15 +322,15 @@ def _attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len, out,
     elif entry == "q8k":
         q8 = (q.data_ptr(), k_pool.data_ptr(), k_scales.data_ptr(), v_pool.data_ptr(),
               block_tables.data_ptr(), mb, context_lens.data_ptr(), q_len)
-        if grid_ctas or min_split_blocks or use_pdl or seg_cost_blocks or producer_wait_ns:
+        if grid_ctas or min_split_blocks or use_pdl or seg_cost_blocks or producer_wait_ns or consumer:
             o = _abi.PagedAttentionOpts(grid_ctas, min_split_blocks, use_pdl, seg_cost_blocks,
-                                        producer_wait_ns)
+                                        producer_wait_ns, consumer)
             rc = _L.paged_attention_q8k_ex(*q8, *tail, ctypes.byref(o), _stream(dev))
         else:
             rc = _L.paged_attention_q8k(*q8, *tail, _stream(dev))
     else:
         o = _abi.PagedAttentionOpts(grid_ctas, min_split_blocks, use_pdl, seg_cost_blocks,
-                                    producer_wait_ns)
+                                    producer_wait_ns, consumer)
         rc = _L.paged_attention_ex(*args, q_len, *tail, ctypes.byref(o), _stream(dev))
     check(rc, f"paged attention ({entry})")
     return out
@@ -380,12 +380,12 @@ def paged_kv_copy_blocks_q8k(kq_pool: torch.Tensor, v_pool: torch.Tensor, pairs:
 
 def paged_attention_q8k(q, kq_pool, k_scales, v_pool, block_tables, context_lens, scale, q_len=1,
                         out=None, workspace=None, grid_ctas=0, min_split_blocks=0, use_pdl=0,
-                        seg_cost_blocks=0, producer_wait_ns=0):
+                        seg_cost_blocks=0, producer_wait_ns=0, consumer=0):
     """Decode (q_len = 1) or causal verify attention over an int8 K pool
     (launch knobs as in paged_attention)."""
     return _attention(q, kq_pool, v_pool, block_tables, context_lens, scale, q_len, out, workspace,
                       grid_ctas, min_split_blocks, use_pdl, "q8k", seg_cost_blocks, k_scales=k_scales,
-                      producer_wait_ns=producer_wait_ns)
+                      producer_wait_ns=producer_wait_ns, consumer=consumer)
 
 
 def paged_decode_attention(q, k_pool, v_pool, block_tables, context_lens, scale, out=None,
@@ -404,13 +404,15 @@ def paged_verify_attention(q, k_pool, v_pool, block_tables, context_lens, scale,
 
 def paged_attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len=1, out=None,
                     workspace=None, grid_ctas=0, min_split_blocks=0, use_pdl=0, seg_cost_blocks=0,
-                    producer_wait_ns=0):
+                    producer_wait_ns=0, consumer=0):
     """Decode / verify with launch knobs (grid size, smallest split, PDL,
     per-segment cost used to balance CTAs, the loading warp's wait limit for
-    failure-detection tests)."""
+    failure-detection tests, the compute path for several query rows per KV
+    head: 1 warp-level MMAs, 2 tcgen05 with tensor-memory accumulators, 0
+    default)."""
     return _attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len, out, workspace,
                       grid_ctas, min_split_blocks, use_pdl, "ex", seg_cost_blocks,
-                      producer_wait_ns=producer_wait_ns)
+                      producer_wait_ns=producer_wait_ns, consumer=consumer)
 
 
 def paged_prefill_attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len,

@@ -27,7 +27,8 @@ class KvPoolConfig(ctypes.Structure):
 class PagedAttentionOpts(ctypes.Structure):
     _fields_ = [("grid_ctas", ctypes.c_int32), ("min_split_blocks", ctypes.c_int32),
                 ("use_pdl", ctypes.c_int32), ("seg_cost_blocks", ctypes.c_int32),
-                ("producer_wait_ns", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+                ("producer_wait_ns", ctypes.c_int32), ("consumer", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 2)]
 
 
 _P = ctypes.c_void_p

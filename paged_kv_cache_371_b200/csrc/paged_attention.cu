@@ -82,7 +82,7 @@ struct Params {
 };
 
 template <int D_, int BS_, int MT_, bool FMA_, bool KQ_ = false, int NR8_ = 0, int TW_ = 0,
-          int SUBS_ = 1>
+          int SUBS_ = 1, int UMR_ = 0>
 struct Cfg {
     static constexpr int D = D_, BS = BS_, MT = MT_;
     static constexpr bool FMA = FMA_;
@@ -90,6 +90,13 @@ struct Cfg {
     // NR8 > 0: tensor-core consumer over S^T = K Q^T (tokens as the MMA's M
     // dimension, query rows as N, in NR8 tiles of 8 rows)
     static constexpr int NR8 = NR8_;
+    // UMR > 0: tcgen05 consumer (accumulators in tensor memory), query rows
+    // padded to UMR; each of the 128 TMEM lanes holds one query row and a
+    // 128/UMR-th of the stage's tokens (see consumer_um)
+    static constexpr int UMR = UMR_;
+    static_assert(!UMR || (D == 128 && MT == 1 && !FMA && NR8 == 0 && SUBS_ == 1 &&
+                           (UMR == 8 || UMR == 16 || UMR == 32)),
+                  "the tcgen05 consumer serves head_dim 128, 8/16/32 padded rows");
     static_assert(!KQ || D == 128, "int8 K pools are served at head_dim 128");
     static constexpr int NH = D / 64;                       // 64-column halves per row
     // consumer warps along the tokens of a stage (16 tokens each) and tokens
@@ -97,7 +104,7 @@ struct Cfg {
     // gain from twice the warps; the tensor-core consumers keep 4 (with 9
     // warps their register cap would drop to 168 and the merge at each
     // segment end would take twice the rounds)
-    static constexpr int TW = TW_ ? TW_ : (FMA ? 8 : 4);
+    static constexpr int TW = UMR ? 8 : (TW_ ? TW_ : (FMA ? 8 : 4));
     // 16-token sub-tiles each consumer warp takes per stage (the transposed
     // tensor-core consumer only): larger stages at the same register count
     static constexpr int SUBS = SUBS_;
@@ -105,9 +112,11 @@ struct Cfg {
     static constexpr int TS = 16 * TW * SUBS;               // tokens per pipeline stage
     static_assert(TS / BS <= 32, "one producer lane per block of a stage");
     static constexpr int NBS = TS / BS;                     // blocks per stage
-    static constexpr int RP = FMA ? 1 : (NR8 ? 8 * NR8 : 16 * MT);  // padded rows
-    static constexpr int NCW = TW;                          // consumer warps
-    static constexpr int THREADS = (NCW + 1) * 32;
+    static constexpr int RP = UMR ? UMR : (FMA ? 1 : (NR8 ? 8 * NR8 : 16 * MT));  // padded rows
+    // consumer warps (the tcgen05 consumer: 4 softmax warps, one per TMEM
+    // lane quarter, plus the MMA-issuing warp after the producer)
+    static constexpr int NCW = UMR ? 4 : TW;
+    static constexpr int THREADS = (NCW + (UMR ? 2 : 1)) * 32;
     // registers per thread for one CTA per SM: warps are spread over the 4
     // SM sub-partitions, each with a 16K-register file
     static constexpr int WARPS_PER_SUBPART = (THREADS / 32 + 3) / 4;
@@ -116,7 +125,12 @@ struct Cfg {
     static constexpr int TILE_BYTES = BS * D * 2;           // one (block, kv-head) fp16 tile
     static constexpr int KV_BYTES = TS * D * 2;             // fp16 K (or V) bytes per stage
     static constexpr int K_TILE_BYTES = KQ ? BS * D : TILE_BYTES;
-    static constexpr int K_BYTES = KQ ? TS * D : KV_BYTES;
+    // the tcgen05 consumer keeps fp16 room for K also over int8 codes: they
+    // land in its upper half and are widened in place
+    static constexpr int K_BYTES = (KQ && !UMR) ? TS * D : KV_BYTES;
+    // one 64-column half of a stage's K or V in the tcgen05 consumer's layout
+    // ([half][token][128 B], the MMA's 128-byte-swizzle K-major / MN-major form)
+    static constexpr int UM_HALF = TS * 128;
     static constexpr int V_OFF = K_BYTES;                   // stage: K, V, query rows
     // query rows of a segment, one per 16-byte-padded row (conflict-free ldmatrix)
     static constexpr int QROW = D * 2 + 16;
@@ -132,15 +146,16 @@ struct Cfg {
     static constexpr int OBUF_SLICE = RP * OB_STRIDE;               // floats
     // two merge slices (the transposed consumer merges in the stage it just
     // consumed instead: one slice per token warp, see consumer_tc)
-    static constexpr int OBUF_BYTES = NR8 ? 0 : 2 * OBUF_SLICE * 4;
-    static constexpr int ML_BYTES = TW * RP * 2 * 4;
+    static constexpr int OBUF_BYTES = (NR8 || UMR) ? 0 : 2 * OBUF_SLICE * 4;
+    static constexpr int ML_BYTES = UMR ? 128 * 2 * 4 : TW * RP * 2 * 4;
     // CTA copy of the query rows (read again every stage)
-    static constexpr bool QPERSIST = NR8 ? NR8 > 2 : MT > 1;
+    static constexpr bool QPERSIST = UMR ? false : (NR8 ? NR8 > 2 : MT > 1);
     // rows of that copy: whole pairs of 8-row tiles (B fragments of two row
     // tiles come from one ldmatrix)
     static constexpr int QP_ROWS = NR8 ? 16 * ((NR8 + 1) / 2) : RP;
     static constexpr int QP_BYTES = QPERSIST ? QP_ROWS * QROW : 0;
-    static constexpr int FIXED = OBUF_BYTES + ML_BYTES + QP_BYTES + 256 + 16 * 64;
+    static constexpr int UM_NBARS = UMR ? 12 : 0;  // the tcgen05 consumer's barriers
+    static constexpr int FIXED = OBUF_BYTES + ML_BYTES + QP_BYTES + 256 + 16 * 64 + UM_NBARS * 8 + 16;
     static constexpr int STAGES_RAW = (kSmemBudget - FIXED) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
     static_assert(STAGES >= 2, "not enough shared memory for two stages");
@@ -151,7 +166,10 @@ struct Cfg {
     static constexpr int ML_OFF = PB_OFF + TW * 32;
     static constexpr int OBUF_OFF = ML_OFF + ML_BYTES;
     static constexpr int QP_OFF = OBUF_OFF + OBUF_BYTES;
-    static constexpr int SMEM_USED = QP_OFF + QP_BYTES;
+    static constexpr int UB_OFF = QP_OFF + QP_BYTES;        // tcgen05 consumer barriers
+    static constexpr int TSLOT_OFF = UB_OFF + UM_NBARS * 8; // its tensor-memory base address
+    static constexpr int SMEM_USED = TSLOT_OFF + (UMR ? 16 : 0);
+    static_assert(!UMR || 128 * D * 4 <= Q_OFF, "the segment-end slices fit a stage's K and V");
     static_assert(!NR8 || TW * OBUF_SLICE * 4 <= STAGE_BYTES, "per-warp merge slices fit a stage");
     static constexpr int SMEM_ALLOC = SMEM_USED + 1024;    // room to align the base
 };
@@ -550,12 +568,26 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
                 const uint32_t st = sbase + stage * C::STAGE_BYTES;
                 if (load) {
                     const int32_t y = (id * p.Hkv + d.kvh) * C::BS;
-                    if constexpr (C::KQ)
-                        tma_load_2d(st + (uint32_t)(lane * C::K_TILE_BYTES), tmK, 0, y, full, pol);
-                    else
-                        tma_load_tile<C::NH>(st + (uint32_t)(lane * C::TILE_BYTES), tmK, y, full, pol);
-                    tma_load_tile<C::NH>(st + C::V_OFF + (uint32_t)(lane * C::TILE_BYTES), tmV, y, full,
-                                         pol);
+                    if constexpr (C::UMR > 0) {
+                        // block `lane` -> rows [lane*BS, lane*BS+BS) of each 64-column
+                        // half; int8 codes (128 per row) into the upper half of K
+                        const uint32_t ko = st + (uint32_t)(lane * C::BS * 128);
+                        if constexpr (C::KQ) {
+                            tma_load_2d(ko + C::UM_HALF, tmK, 0, y, full, pol);
+                        } else {
+                            tma_load_2d(ko, tmK, 0, y, full, pol);
+                            tma_load_2d(ko + C::UM_HALF, tmK, 64, y, full, pol);
+                        }
+                        tma_load_2d(ko + C::V_OFF, tmV, 0, y, full, pol);
+                        tma_load_2d(ko + C::V_OFF + C::UM_HALF, tmV, 64, y, full, pol);
+                    } else {
+                        if constexpr (C::KQ)
+                            tma_load_2d(st + (uint32_t)(lane * C::K_TILE_BYTES), tmK, 0, y, full, pol);
+                        else
+                            tma_load_tile<C::NH>(st + (uint32_t)(lane * C::TILE_BYTES), tmK, y, full, pol);
+                        tma_load_tile<C::NH>(st + C::V_OFF + (uint32_t)(lane * C::TILE_BYTES), tmV, y,
+                                             full, pol);
+                    }
                 }
                 if (firstst && lane < p.rows) {  // row R = j*G + g of the segment's queries
                     const int j = lane / p.G, g = lane % p.G;
@@ -1522,6 +1554,448 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
     }
 }
 
+// ---------------------------------------------------------------------------
+// tcgen05 consumer (query rows > 1, head_dim 128): both products on the
+// 5th-generation tensor cores, accumulators in tensor memory.
+//
+// Each 128-token stage is one MMA pair over all 128 TMEM lanes.  Lane m holds
+// query row r = m mod R (R = UMR, the padded rows) and owns the stage's
+// tokens [g*R, g*R + R), g = m / R: the rows are replicated 128/R times so
+// that every lane, and so every softmax thread, has work.
+//   S = Q K^T   M128 N128 K128, A = the replicated query rows (fp16 pairs in
+//               tensor memory), B = the stage's K (K-major, 128-byte swizzle)
+//   softmax     thread m = lane m: its R scores, its own running maximum and
+//               denominator (online softmax over its tokens only; no
+//               cross-thread reduction per stage)
+//   O += P V    M128 N128 K128, A = P (fp16 pairs in tensor memory, zero
+//               outside the lane's tokens), B = the stage's V (MN-major)
+// At a segment's end the 128/R partial (o, m, l) of each row are combined in
+// a fixed order (bit-reproducible) through the consumed stage's shared
+// memory.  The MMAs do 128/R times the useful flops; at 128 tokens per stage
+// that is ~1000 tensor cycles against ~2700 of HBM time per stage.
+// Int8 keys: the softmax warps widen the stage's codes to fp16 in place (the
+// channel scales are folded into the query rows).
+// Tensor memory: S (128 columns), P (two buffers of 64), O (128), the query
+// rows (two buffers of 64, by segment parity).
+enum : uint32_t { UM_S = 0, UM_P = 128, UM_O = 256, UM_Q = 384, UM_COLS = 512 };
+enum : int { UB_S_FULL = 0, UB_S_FREE = 1, UB_P_FULL = 2, UB_O_DONE = 4, UB_Q_READY = 6, UB_KDQ = 7,
+             UB_EP = 8, UB_DRAIN = 9 };
+constexpr float kRescaleThreshold = 8.f;  // log2 units: weights stay below 2^8
+
+template <class C>
+__device__ void consumer_um(const Params& p, uint8_t* smem, uint32_t tmem, volatile int* abort_flag)
+{
+    constexpr int R = C::UMR;        // padded rows; also tokens per lane (128 tokens / (128 / R) lanes)
+    constexpr int T = R;
+    constexpr int NG = 128 / R;      // lanes per query row
+    constexpr int NSUB = 32 / T;     // token groups in a warp's 32 tokens
+    constexpr int HW = T / 2;        // fp16 pairs of a lane's weights
+    static_assert(C::TS == 128 && C::NCW == 4, "one 128-lane MMA per stage");
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m = threadIdx.x;       // TMEM lane
+    const int r = m % R;
+    const int sub = lane / T;
+    const uint32_t sbase = smem_u32(smem);
+    const StageMeta* smeta = reinterpret_cast<const StageMeta*>(smem + C::META_OFF);
+    const uint32_t full0 = sbase + C::BAR_OFF;
+    const uint32_t empty0 = full0 + C::STAGES * 8;
+    const uint32_t ub = sbase + C::UB_OFF;
+    const uint32_t lb = tmem + ((uint32_t)(32 * w) << 16);  // this warp's lane quarter
+    float* ml = reinterpret_cast<float*>(smem + C::ML_OFF);
+    const float sl2 = p.scale_log2;
+    const bool row_ok = r < p.rows;
+    const int jr = row_ok ? r / p.G : 0;
+
+    {   // both weight buffers start zero; each warp only ever writes its own tokens' columns
+        float z[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) z[i] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 128; c += 32) tmem_st32(lb + UM_P + c, z);
+        tmem_wait_st();
+    }
+
+    bool ok = true;
+    // every lane waits; the warp stops together when any lane gave up.  A
+    // loader that gave up still posts the end marker, so the compute warps
+    // stop there, all at the same stage (they do not read the abort flag:
+    // one warp stopping early would leave the others at the merge barrier)
+    auto wait_all = [&](uint32_t bar, uint32_t par) -> bool {
+        const bool got = mbar_wait_bounded(bar, par, kWaitLimitNs);
+        const bool all = __all_sync(0xffffffffu, got);
+        if (!all) ok = false;
+        return all;
+    };
+    int ep = 0;  // phases of the epilogue barrier used so far
+    auto ep_sync = [&]() -> bool {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ub + 8 * UB_EP);
+        const bool got = wait_all(ub + 8 * UB_EP, (uint32_t)(ep & 1));
+        ++ep;
+        return got;
+    };
+
+    // Everything stage `st` needs before its S can be issued, done by each
+    // warp for its lanes / tokens: the segment's query rows into tensor
+    // memory (first stage of a segment; the buffers alternate by segment),
+    // int8 codes widened to fp16, V rows past the staged tokens zeroed.
+    int qseg = 0;  // segments whose query rows are written
+    auto prep = [&](int st, const StageMeta& mdd) {
+        uint8_t* sg = smem + st * C::STAGE_BYTES;
+        if (mdd.flags & F_FIRST) {
+            // row r in lane m (times the channel scales over int8 keys);
+            // padded rows are zero
+            const uint4* qs = reinterpret_cast<const uint4*>(sg + C::Q_OFF + r * C::QROW);
+            const uint32_t qcol = UM_Q + (uint32_t)((qseg & 1) * 64);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float qv[32];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint4 x = qs[h * 8 + i];
+                    uint32_t wv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        if constexpr (C::KQ) {
+                            const float* sc = reinterpret_cast<const float*>(sg + C::SC_OFF);
+                            const int d = 2 * (h * 32 + i * 4 + e);
+                            wv[e] = scale_h2(wv[e], *reinterpret_cast<const float2*>(sc + d));
+                        }
+                        qv[i * 4 + e] = __uint_as_float(wv[e]);
+                    }
+                }
+                tmem_st32(lb + qcol + 32 * h, qv);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ub + 8 * UB_Q_READY);
+            ++qseg;
+        }
+        if constexpr (C::KQ) {
+            // token m's 128 codes (swizzled 16-byte chunks in the upper half of
+            // K) -> fp16 in both halves; the thread reads its whole row first,
+            // so the in-place widening never races another thread
+            const uint32_t kb = smem_u32(sg);
+            uint4 cw[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                cw[c] = *reinterpret_cast<const uint4*>(sg + C::UM_HALF + m * 128 + ((c ^ (m & 7)) << 4));
+            const uint32_t bias = 0x64806480u;  // fp16 pair (1152, 1152)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint32_t cwords[4] = {cw[c].x, cw[c].y, cw[c].z, cw[c].w};
+                uint32_t hw[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    uint32_t lo, hi;
+                    i8x4_to_h2x2_biased(cwords[e], lo, hi);
+                    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(hw[2 * e]) : "r"(lo), "r"(bias));
+                    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(hw[2 * e + 1]) : "r"(hi), "r"(bias));
+                }
+                // dims 16c .. 16c+7 and 16c+8 .. 16c+15: chunks 2c, 2c+1 of the row
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int dc = 2 * c + q;
+                    const uint32_t addr = kb + (uint32_t)((dc >> 3) * C::UM_HALF + m * 128 +
+                                                          (((dc & 7) ^ (m & 7)) << 4));
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(hw[4 * q]),
+                                 "r"(hw[4 * q + 1]), "r"(hw[4 * q + 2]), "r"(hw[4 * q + 3])
+                                 : "memory");
+                }
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ub + 8 * UB_KDQ);
+        }
+        if (mdd.ntok < C::TS && m >= mdd.ntok) {
+            // V rows past the staged tokens must be finite zeros for the MMA
+            // (ordered before the tensor core's read by the fence ahead of
+            // this stage's weights-written arrive)
+            uint8_t* vr = sg + C::V_OFF + m * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                *reinterpret_cast<uint4*>(vr + (c << 4)) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(vr + C::UM_HALF + (c << 4)) = make_uint4(0, 0, 0, 0);
+            }
+        }
+    };
+
+    float m_run = kNegInf, l_run = 0.f;
+    int stage = 0, j = 0, prepped = -1;
+    uint32_t phase = 0;
+    for (;;) {
+        if (!wait_all(full0 + stage * 8, phase)) break;
+        const StageMeta md = smeta[stage];
+        if (md.flags & F_END) break;
+        uint8_t* stg = smem + stage * C::STAGE_BYTES;
+        if (prepped != j) prep(stage, md);
+        if (md.flags & F_FIRST) {
+            m_run = kNegInf;
+            l_run = 0.f;
+        }
+        // ---- scores of this stage
+        if (!wait_all(ub + 8 * UB_S_FULL, (uint32_t)(j & 1))) break;
+        tc_fence_after();
+        float x[32];
+        tmem_ld32(lb + UM_S + 32 * w, x);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ub + 8 * UB_S_FREE);
+        {   // prepare the next stage now if it has landed (lane 0 decides)
+            const int ns = stage + 1 == C::STAGES ? 0 : stage + 1;
+            const uint32_t np = stage + 1 == C::STAGES ? phase ^ 1u : phase;
+            const bool landed = __shfl_sync(0xffffffffu, mbar_test(full0 + ns * 8, np) ? 1 : 0, 0) != 0;
+            if (landed) {
+                const StageMeta nmd = smeta[ns];
+                if (!(nmd.flags & F_END)) {
+                    prep(ns, nmd);
+                    prepped = j + 1;
+                }
+            }
+        }
+        float v[T];
+#pragma unroll
+        for (int i = 0; i < T; ++i) {
+            v[i] = x[i];
+#pragma unroll
+            for (int s2 = 1; s2 < NSUB; ++s2)
+                if (sub == s2) v[i] = x[s2 * T + i];
+        }
+        // visible: staged (< ntok) and, in a verify window, up to the row's position
+        int lim = md.L - p.q_len + jr + 1 - md.t0;
+        if (lim > md.ntok) lim = md.ntok;
+        if (!row_ok) lim = 0;
+        const int nvis = lim - (32 * w + sub * T);
+        float mx = kNegInf;
+#pragma unroll
+        for (int i = 0; i < T; ++i) {
+            v[i] = i < nvis ? v[i] : kNegInf;
+            mx = fmaxf(mx, v[i]);
+        }
+        mx *= sl2;
+        const bool grow = mx > m_run + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, grow)) {
+            const float mn = grow ? mx : m_run;
+            const float alpha = m_run == kNegInf ? 1.f : ex2(m_run - mn);
+            if (__any_sync(0xffffffffu, grow && m_run != kNegInf)) {
+                // O holds this segment's earlier stages: P V(j-1) (issued right
+                // after S(j)) must have finished before it is rescaled
+                const int jp = j - 1;
+                if (!wait_all(ub + 8 * (UB_O_DONE + (jp & 1)), (uint32_t)((jp >> 1) & 1))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int c0 = 0; c0 < C::D; c0 += 32) {
+                    float o[32];
+                    tmem_ld32(lb + UM_O + c0, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                    tmem_st32(lb + UM_O + c0, o);
+                }
+                tmem_wait_st();
+            }
+            l_run *= alpha;
+            m_run = mn;
+        }
+        const float mu = m_run == kNegInf ? 0.f : m_run;
+        uint32_t pw[HW];
+        float ls = 0.f;
+#pragma unroll
+        for (int e = 0; e < HW; ++e) {
+            const float a = ex2(fmaf(v[2 * e], sl2, -mu));
+            const float b = ex2(fmaf(v[2 * e + 1], sl2, -mu));
+            ls += a + b;
+            pw[e] = pack_half2(a, b);
+        }
+        l_run += ls;
+        // weight buffer j&1 was last read by P V(j-2)
+        if (j >= 2 && !wait_all(ub + 8 * (UB_O_DONE + (j & 1)), (uint32_t)(((j - 2) >> 1) & 1))) break;
+        float pv[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) pv[c] = (c / HW == sub) ? __uint_as_float(pw[c % HW]) : 0.f;
+        tmem_st16(lb + UM_P + (uint32_t)((j & 1) * 64 + 16 * w), pv);
+        tmem_wait_st();
+        fence_proxy_async();  // the V zeros above are read by the tensor core
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ub + 8 * (UB_P_FULL + (j & 1)));
+
+        if (md.flags & F_LAST) {
+            // ---- segment end: combine the NG partials of every row
+            if (!wait_all(ub + 8 * (UB_O_DONE + (j & 1)), (uint32_t)((j >> 1) & 1))) break;
+            tc_fence_after();
+            ml[2 * m] = m_run;
+            ml[2 * m + 1] = l_run;
+            if (!ep_sync()) break;
+            float M = kNegInf;
+#pragma unroll
+            for (int g = 0; g < NG; ++g) M = fmaxf(M, ml[2 * (g * R + r)]);
+            const float Mu = M == kNegInf ? 0.f : M;
+            float Ls = 0.f;
+#pragma unroll
+            for (int g = 0; g < NG; ++g) Ls += ml[2 * (g * R + r) + 1] * ex2(ml[2 * (g * R + r)] - Mu);
+            const float f = Ls > 0.f ? ex2(m_run - Mu) / Ls : 0.f;
+            // lane m's o times its factor -> row m of the consumed stage's K/V
+            // area (512 B per row, 16-byte chunk ch stored at ch ^ (m mod 8))
+#pragma unroll
+            for (int c0 = 0; c0 < C::D; c0 += 32) {
+                float o[32];
+                tmem_ld32(lb + UM_O + c0, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int ch = c0 / 4 + q;
+                    *reinterpret_cast<float4*>(stg + m * 512 + ((ch ^ (m & 7)) << 4)) =
+                        make_float4(o[4 * q] * f, o[4 * q + 1] * f, o[4 * q + 2] * f, o[4 * q + 3] * f);
+                }
+            }
+            if (!ep_sync()) break;
+            const bool whole = (md.flags & F_WHOLE) != 0;
+            const int64_t pbase = ((int64_t)blockIdx.x * 2 + md.slot) * C::RP;
+            for (int idx = m; idx < p.rows * 32; idx += 128) {
+                const int rr = idx >> 5, ch = idx & 31;
+                float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int g = 0; g < NG; ++g) {
+                    const int row = g * R + rr;
+                    const float4 b = *reinterpret_cast<const float4*>(stg + row * 512 + ((ch ^ (row & 7)) << 4));
+                    a = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+                }
+                if (whole) {
+                    const int jj = rr / p.G, gg = rr % p.G;
+                    __half* dst = p.out + (((int64_t)md.s * p.q_len + jj) * p.Hq + (int64_t)md.kvh * p.G + gg) *
+                                              C::D + ch * 4;
+                    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_half2(a.x, a.y), pack_half2(a.z, a.w));
+                } else {
+                    *reinterpret_cast<float4*>(p.part_o + (pbase + rr) * C::D + ch * 4) = a;
+                }
+            }
+            if (!whole && m < p.rows) p.part_lse[pbase + m] = Ls > 0.f ? Mu + lg2(Ls) : kNegInf;
+            fence_proxy_async();  // generic accesses of the stage before its next copy
+            if (!ep_sync()) break;
+            if (m == 0) mbar_arrive(empty0 + stage * 8);
+        }
+        ++j;
+        if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+        }
+    }
+    if (!ok && lane == 0) {
+        atomicOr(p.err, KV_DEV_TIMEOUT);
+        *abort_flag = 1;
+    }
+}
+
+// MMA-issuing warp of the tcgen05 consumer (one thread issues, polling).
+// S(k) needs its stage staged (and widened, for int8 keys), the segment's
+// query rows in tensor memory, and the softmax done reading S(k-1); P V(i)
+// needs the weights of stage i.  Whichever is ready is issued first, P V in
+// stage order, so a P V never waits behind the next stage's copy.  At a
+// segment boundary every earlier P V goes before the new segment's first S
+// (the softmax waits for the last one before it merges the segment).  P V(i)
+// releases its stage, except at a segment end, where the softmax uses the
+// stage for the merge and releases it itself.
+template <class C>
+__device__ void mma_um(const Params& p, uint8_t* smem, uint32_t tmem, volatile int* abort_flag)
+{
+    const int lane = threadIdx.x & 31;
+    if (lane == 0) {
+        const uint32_t sbase = smem_u32(smem);
+        const StageMeta* smeta = reinterpret_cast<const StageMeta*>(smem + C::META_OFF);
+        const uint32_t full0 = sbase + C::BAR_OFF;
+        const uint32_t empty0 = full0 + C::STAGES * 8;
+        const uint32_t ub = sbase + C::UB_OFF;
+        constexpr uint32_t idS = idesc_f16(128, C::TS, false);
+        constexpr uint32_t idO = idesc_f16(128, C::D, true);
+        // stages whose S is issued and P V is not: ring slot and flags
+        constexpr int kPend = 4;
+        int pst[kPend];
+        int32_t pfl[kPend];
+        int k = 0, pv = 0, seg = 0, stage = 0;
+        uint32_t phase = 0;
+        bool have_md = false, end = false, ok = true;
+        int32_t flags = 0;
+        uint32_t idle = 0;
+        uint64_t t_idle = 0;
+        while (ok) {
+            bool prog = false;
+            if (pv < k && mbar_test(ub + 8 * (UB_P_FULL + (pv & 1)), (uint32_t)((pv >> 1) & 1))) {
+                tc_fence_after();
+                const int i = pv % kPend;
+                const uint32_t vb = sbase + pst[i] * C::STAGE_BYTES + C::V_OFF;
+                const uint32_t pa = tmem + UM_P + (uint32_t)((pv & 1) * 64);
+                const bool first = (pfl[i] & F_FIRST) != 0;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_f16_ts(tmem + UM_O, pa + kk * 8, smem_desc(vb + kk * 16 * 128, C::UM_HALF, 1024),
+                                idO, (!first || kk > 0) ? 1u : 0u);
+                umma_commit(ub + 8 * (UB_O_DONE + (pv & 1)));
+                if (!(pfl[i] & F_LAST)) umma_commit(empty0 + pst[i] * 8);
+                ++pv;
+                prog = true;
+            }
+            if (!end) {
+                if (!have_md && mbar_test(full0 + stage * 8, phase)) {
+                    flags = smeta[stage].flags;
+                    have_md = true;
+                    if (flags & F_END) end = true;
+                }
+                if (have_md && !end && k - pv < kPend) {
+                    bool ready = true;
+                    if (flags & F_FIRST)
+                        ready = pv == k && mbar_test(ub + 8 * UB_Q_READY, (uint32_t)(seg & 1));
+                    if constexpr (C::KQ) {
+                        if (ready) ready = mbar_test(ub + 8 * UB_KDQ, (uint32_t)(k & 1));
+                    }
+                    if (ready && k > 0) ready = mbar_test(ub + 8 * UB_S_FREE, (uint32_t)((k - 1) & 1));
+                    if (ready) {
+                        if (flags & F_FIRST) ++seg;
+                        tc_fence_after();
+                        const uint32_t kb = sbase + stage * C::STAGE_BYTES;
+                        const uint32_t qa = tmem + UM_Q + (uint32_t)(((seg - 1) & 1) * 64);
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            umma_f16_ts(tmem + UM_S, qa + kk * 8,
+                                        smem_desc(kb + (kk >> 2) * C::UM_HALF + (kk & 3) * 32, 16, 1024), idS,
+                                        kk > 0 ? 1u : 0u);
+                        umma_commit(ub + 8 * UB_S_FULL);
+                        pst[k % kPend] = stage;
+                        pfl[k % kPend] = flags;
+                        ++k;
+                        have_md = false;
+                        if (++stage == C::STAGES) {
+                            stage = 0;
+                            phase ^= 1;
+                        }
+                        prog = true;
+                    }
+                }
+            } else if (pv == k) {
+                break;
+            }
+            // watchdog: no progress for the wait limit
+            if (prog) {
+                idle = 0;
+            } else if ((++idle & 1023u) == 0) {
+                const uint64_t now = globaltimer_ns();
+                if (idle == 1024u) t_idle = now;
+                else if (now - t_idle > kWaitLimitNs) ok = false;
+            }
+        }
+        if (!ok) {
+            atomicOr(p.err, KV_DEV_TIMEOUT);
+            *abort_flag = 1;
+        }
+        // every MMA issued must have finished before tensor memory is freed
+        umma_commit(ub + 8 * UB_DRAIN);
+        if (!mbar_wait_bounded(ub + 8 * UB_DRAIN, 0, kWaitLimitNs)) atomicOr(p.err, KV_DEV_TIMEOUT);
+    }
+    __syncwarp();
+}
+
 template <class C>
 __global__ void __maxnreg__(C::MAXREG)
     paged_attention_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -1536,7 +2010,14 @@ __global__ void __maxnreg__(C::MAXREG)
         abort_flag = 0;
         for (int i = 0; i < C::STAGES; ++i) {
             mbar_init(sbase + C::BAR_OFF + i * 8, 1);
-            mbar_init(sbase + C::BAR_OFF + (C::STAGES + i) * 8, C::NCW);
+            // the tcgen05 consumer releases a stage with one arrive (an MMA
+            // commit, or the merge at a segment end)
+            mbar_init(sbase + C::BAR_OFF + (C::STAGES + i) * 8, C::UMR ? 1 : C::NCW);
+        }
+        if constexpr (C::UMR > 0) {
+            const uint32_t ub = sbase + C::UB_OFF;
+            const uint32_t counts[10] = {1, 4, 4, 4, 1, 1, 4, 4, 4, 1};  // see the UB_* indices
+            for (int i = 0; i < 10; ++i) mbar_init(ub + 8 * i, counts[i]);
         }
         fence_barrier_init();
     }
@@ -1551,19 +2032,44 @@ __global__ void __maxnreg__(C::MAXREG)
     }
     if (threadIdx.x < 8)
         reinterpret_cast<uint4*>(smem + C::ZERO_OFF)[threadIdx.x] = make_uint4(0, 0, 0, 0);
+    const int warp = threadIdx.x >> 5;
+    if constexpr (C::UMR > 0) {
+        // one CTA per SM: all 512 columns
+        if (warp == C::NCW + 1) {
+            tmem_alloc(sbase + C::TSLOT_OFF, UM_COLS);
+            tmem_relinquish();
+        }
+        tc_fence_before();
+    }
     fence_proxy_async();
     __syncthreads();
     pdl_launch_dependents();
-    const int warp = threadIdx.x >> 5;
-    if (warp == C::NCW) {
-        producer<C>(&tmK, &tmV, p, smem, &abort_flag);
-    } else if constexpr (C::FMA) {
-        consumer_fma<C>(p, smem, &abort_flag);
-    } else if constexpr (C::NR8 > 0) {
-        consumer_tc<C>(p, smem, &abort_flag);
+    if constexpr (C::UMR > 0) {
+        tc_fence_after();
+        const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + C::TSLOT_OFF);
+        if (warp == C::NCW)
+            producer<C>(&tmK, &tmV, p, smem, &abort_flag);
+        else if (warp == C::NCW + 1)
+            mma_um<C>(p, smem, tmem, &abort_flag);
+        else
+            consumer_um<C>(p, smem, tmem, &abort_flag);
+        tc_fence_before();
+        __syncthreads();
+        if (warp == C::NCW + 1) {
+            tc_fence_after();
+            tmem_dealloc(tmem, UM_COLS);
+        }
     } else {
-        static_assert(C::MT > 1, "one row tile of more than one row uses the transposed consumer");
-        consumer_mma_mt<C>(p, smem, &abort_flag);
+        if (warp == C::NCW) {
+            producer<C>(&tmK, &tmV, p, smem, &abort_flag);
+        } else if constexpr (C::FMA) {
+            consumer_fma<C>(p, smem, &abort_flag);
+        } else if constexpr (C::NR8 > 0) {
+            consumer_tc<C>(p, smem, &abort_flag);
+        } else {
+            static_assert(C::MT > 1, "one row tile of more than one row uses the transposed consumer");
+            consumer_mma_mt<C>(p, smem, &abort_flag);
+        }
     }
 }
 
@@ -1571,51 +2077,52 @@ __global__ void __maxnreg__(C::MAXREG)
 // Split-context merge: CTA c merges the (sequence, kv-head) whose last piece
 // it computed, from the partials of CTAs meta.first .. c:
 //   lse* = log2 sum_i 2^(lse_i),  out = sum_i 2^(lse_i - lse*) o_i.
+// One thread per (row, 8 output dims); one pass with a running maximum, two
+// pieces per step with all their loads issued together (the kernel is bound
+// by the latency of those loads, not by their bytes).
 template <int D, int RP>
-__global__ void __launch_bounds__(128) lse_merge_kernel(const Params p)
+__global__ void __launch_bounds__(512) lse_merge_kernel(const Params p)
 {
     pdl_wait();
     const int c = blockIdx.x;
     const int4 md = p.meta[c];
     if (md.x < 0) return;
+    const int idx = threadIdx.x;
+    if (idx >= p.rows * (D / 8)) return;
     const int s = md.x, kvh = md.y, a = md.z, slot_a = md.w;
-    for (int idx = threadIdx.x; idx < p.rows * (D / 8); idx += blockDim.x) {
-        const int R = idx / (D / 8);
-        const int d0 = (idx % (D / 8)) * 8;
-        float M = kNegInf;
-        for (int i = a; i <= c; ++i) {
-            const int slot = i == a ? slot_a : 0;
-            M = fmaxf(M, p.part_lse[((int64_t)i * 2 + slot) * RP + R]);
-        }
-        const float Mu = M == kNegInf ? 0.f : M;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        float W = 0.f;
-        for (int i = a; i <= c; ++i) {
-            const int slot = i == a ? slot_a : 0;
-            const int64_t pr = ((int64_t)i * 2 + slot) * RP + R;
-            const float w = ex2(p.part_lse[pr] - Mu);
-            W += w;
-            const float4* src = reinterpret_cast<const float4*>(p.part_o + pr * D + d0);
-            const float4 x = src[0], y = src[1];
-            acc[0] += w * x.x;
-            acc[1] += w * x.y;
-            acc[2] += w * x.z;
-            acc[3] += w * x.w;
-            acc[4] += w * y.x;
-            acc[5] += w * y.y;
-            acc[6] += w * y.z;
-            acc[7] += w * y.w;
-        }
-        const float inv = W > 0.f ? 1.f / W : 0.f;
-        const int j = R / p.G, g = R % p.G;
-        uint4 v;
-        v.x = pack_half2(acc[0] * inv, acc[1] * inv);
-        v.y = pack_half2(acc[2] * inv, acc[3] * inv);
-        v.z = pack_half2(acc[4] * inv, acc[5] * inv);
-        v.w = pack_half2(acc[6] * inv, acc[7] * inv);
-        __half* dst = p.out + (((int64_t)s * p.q_len + j) * p.Hq + (int64_t)kvh * p.G + g) * D + d0;
-        *reinterpret_cast<uint4*>(dst) = v;
+    const int R = idx / (D / 8);
+    const int d0 = (idx % (D / 8)) * 8;
+    float M = kNegInf, W = 0.f;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int i = a; i <= c; i += 2) {
+        const bool two = i + 1 <= c;
+        const int64_t pr0 = ((int64_t)i * 2 + (i == a ? slot_a : 0)) * RP + R;
+        const int64_t pr1 = two ? ((int64_t)(i + 1) * 2) * RP + R : pr0;
+        const float l0 = p.part_lse[pr0];
+        const float l1 = two ? p.part_lse[pr1] : kNegInf;
+        const float4* o0 = reinterpret_cast<const float4*>(p.part_o + pr0 * D + d0);
+        const float4* o1 = reinterpret_cast<const float4*>(p.part_o + pr1 * D + d0);
+        const float4 x0 = o0[0], y0 = o0[1], x1 = o1[0], y1 = o1[1];
+        const float mn = fmaxf(M, fmaxf(l0, l1));
+        if (mn == kNegInf) continue;  // no visible token so far
+        const float f = ex2(M - mn);  // 0 while M is still -inf
+        const float w0 = ex2(l0 - mn), w1 = two ? ex2(l1 - mn) : 0.f;
+        const float v0[8] = {x0.x, x0.y, x0.z, x0.w, y0.x, y0.y, y0.z, y0.w};
+        const float v1[8] = {x1.x, x1.y, x1.z, x1.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = acc[e] * f + w0 * v0[e] + w1 * v1[e];
+        W = W * f + w0 + w1;
+        M = mn;
     }
+    const float inv = W > 0.f ? 1.f / W : 0.f;
+    const int j = R / p.G, g = R % p.G;
+    uint4 v;
+    v.x = pack_half2(acc[0] * inv, acc[1] * inv);
+    v.y = pack_half2(acc[2] * inv, acc[3] * inv);
+    v.z = pack_half2(acc[4] * inv, acc[5] * inv);
+    v.w = pack_half2(acc[6] * inv, acc[7] * inv);
+    __half* dst = p.out + (((int64_t)s * p.q_len + j) * p.Hq + (int64_t)kvh * p.G + g) * D + d0;
+    *reinterpret_cast<uint4*>(dst) = v;
 }
 
 }  // namespace pkv
@@ -1652,9 +2159,11 @@ int get_encoder()
 }
 
 // Tensor map of a pool viewed as [num_blocks*Hkv*BS rows][D] fp16 whose box
-// is one (block, kv-head) tile, 128-byte swizzle.  Cached by (pointer, shape,
-// device).
-int pool_tmap(const void* pool, uint64_t rows, int D, int BS, CUtensorMap* out, int int8 = 0)
+// is one (block, kv-head) tile, 128-byte swizzle (kind 0); an int8 code pool
+// (kind 1); fp16 with a box of one 64-column half of a tile (kind 2, the
+// tcgen05 consumer's layout).  Cached by (pointer, shape, kind, device).
+enum : int { TMAP_TILE = 0, TMAP_INT8 = 1, TMAP_HALF = 2 };
+int pool_tmap(const void* pool, uint64_t rows, int D, int BS, CUtensorMap* out, int int8 = TMAP_TILE)
 {
     int dev = 0;
     cudaGetDevice(&dev);
@@ -1667,7 +2176,25 @@ int pool_tmap(const void* pool, uint64_t rows, int D, int BS, CUtensorMap* out, 
         }
     int rc = get_encoder();
     if (rc != KV_OK) return rc;
-    if (int8) {
+    if (int8 == TMAP_HALF) {
+        // [rows][D] fp16, box = 64 columns x BS rows (one half of a tile)
+        CUtensorMap m;
+        const cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+        const cuuint64_t gstride[1] = {(cuuint64_t)D * 2};
+        const cuuint32_t box[2] = {64, (cuuint32_t)BS};
+        const cuuint32_t estride[2] = {1, 1};
+        CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(pool), gdim,
+                              gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return kv_fail(KV_ERR_CUDA, "cuTensorMapEncodeTiled failed (half tiles)");
+        TmapEntry& e = g_tmaps[g_tmap_next];
+        g_tmap_next = (g_tmap_next + 1) % kTmapCache;
+        e = {pool, rows, D, BS, dev, int8, m};
+        *out = m;
+        return KV_OK;
+    }
+    if (int8 == TMAP_INT8) {
         // int8 code pool as [rows][128]: a box of BS rows is one (block,
         // kv-head) tile of 128-byte rows, 128-byte swizzle
         CUtensorMap m;
@@ -1751,7 +2278,7 @@ int launch(const CUtensorMap& tk, const CUtensorMap& tv, const Params& prm, int 
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(128);
+    cfg.blockDim = dim3((unsigned)((prm.rows * (C::D / 8) + 31) / 32 * 32));  // <= 512
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -1764,9 +2291,17 @@ int launch(const CUtensorMap& tk, const CUtensorMap& tv, const Params& prm, int 
 }
 
 template <int D, int BS, bool KQ = false>
-int dispatch_rows(int rows, const CUtensorMap& tk, const CUtensorMap& tv, const Params& prm,
+int dispatch_rows(int rows, bool um, const CUtensorMap& tk, const CUtensorMap& tv, const Params& prm,
                   int grid, bool pdl, cudaStream_t st)
 {
+    if constexpr (D == 128) {
+        // tcgen05 consumer, rows padded to 8, 16 or 32
+        if (um) {
+            if (rows <= 8) return launch<Cfg<D, BS, 1, false, KQ, 0, 0, 1, 8>>(tk, tv, prm, grid, pdl, st);
+            if (rows <= 16) return launch<Cfg<D, BS, 1, false, KQ, 0, 0, 1, 16>>(tk, tv, prm, grid, pdl, st);
+            return launch<Cfg<D, BS, 1, false, KQ, 0, 0, 1, 32>>(tk, tv, prm, grid, pdl, st);
+        }
+    }
     // Tensor-core paths: 128-token stages (8 token warps for one row tile, 4
     // warps of two 16-token sub-tiles for two or three; 256 tokens for one
     // row tile over int8 keys); more than 24 rows keep the rows-as-M consumer
@@ -1783,6 +2318,11 @@ int dispatch_rows(int rows, const CUtensorMap& tk, const CUtensorMap& tv, const 
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Default consumer for several query rows per KV head (head_dim 128): the
+// warp-level MMAs, measured faster than the tcgen05 consumer on every
+// benchmark shape (8, 20 and 32 rows; fp16 and int8 keys).
+bool default_tcgen05(int, bool) { return false; }
 
 int attention_impl(const void* q, const void* k_pool, const void* v_pool,
                    const int32_t* block_tables, int32_t max_blocks_per_seq,
@@ -1821,11 +2361,17 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
     int* err = kv_error_word_ptr();
     if (!err) return kv_fail(KV_ERR_CUDA, "paged attention: no device error word");
 
+    // consumer for several query rows per KV head at head_dim 128: tcgen05
+    // (tensor memory) or warp-level MMAs
+    const int consumer = opts ? opts->consumer : 0;
+    if (consumer < 0 || consumer > 2)
+        return kv_fail(KV_ERR_INVALID, "paged attention: opts.consumer must be 0, 1 or 2");
+    const bool um = D == 128 && rows > 1 && (consumer == 2 || (consumer == 0 && default_tcgen05(rows, k_scale != nullptr)));
     CUtensorMap tk, tv;
     const uint64_t prow = (uint64_t)num_blocks * Hkv * BS;
-    int rc = pool_tmap(k_pool, prow, D, BS, &tk, k_scale ? 1 : 0);
+    int rc = pool_tmap(k_pool, prow, D, BS, &tk, k_scale ? TMAP_INT8 : (um ? TMAP_HALF : TMAP_TILE));
     if (rc != KV_OK) return rc;
-    rc = pool_tmap(v_pool, prow, D, BS, &tv);
+    rc = pool_tmap(v_pool, prow, D, BS, &tv, um ? TMAP_HALF : TMAP_TILE);
     if (rc != KV_OK) return rc;
 
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -1858,14 +2404,14 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
     const bool pdl = !(opts && opts->use_pdl < 0);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (k_scale)
-        return BS == 8 ? dispatch_rows<128, 8, true>(rows, tk, tv, prm, grid, pdl, st)
-                       : dispatch_rows<128, 16, true>(rows, tk, tv, prm, grid, pdl, st);
+        return BS == 8 ? dispatch_rows<128, 8, true>(rows, um, tk, tv, prm, grid, pdl, st)
+                       : dispatch_rows<128, 16, true>(rows, um, tk, tv, prm, grid, pdl, st);
     if (D == 64) {
-        return BS == 8 ? dispatch_rows<64, 8>(rows, tk, tv, prm, grid, pdl, st)
-                       : dispatch_rows<64, 16>(rows, tk, tv, prm, grid, pdl, st);
+        return BS == 8 ? dispatch_rows<64, 8>(rows, false, tk, tv, prm, grid, pdl, st)
+                       : dispatch_rows<64, 16>(rows, false, tk, tv, prm, grid, pdl, st);
     }
-    return BS == 8 ? dispatch_rows<128, 8>(rows, tk, tv, prm, grid, pdl, st)
-                   : dispatch_rows<128, 16>(rows, tk, tv, prm, grid, pdl, st);
+    return BS == 8 ? dispatch_rows<128, 8>(rows, um, tk, tv, prm, grid, pdl, st)
+                   : dispatch_rows<128, 16>(rows, um, tk, tv, prm, grid, pdl, st);
 }
 
 }  // namespace
