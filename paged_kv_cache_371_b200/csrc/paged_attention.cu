@@ -31,6 +31,10 @@
 //    (mma.sync m16n8k16, fp16 in, fp32 accumulate), fed by conflict-free
 //    ldmatrix from the swizzled tiles.  With one row (MHA decode) the work is
 //    a matrix-vector product and runs on the FMA pipes with warp shuffles.
+//    An opt-in consumer computes the same on the 5th-generation tensor cores
+//    (tcgen05, accumulators in tensor memory; consumer_um): at 8-24 rows per
+//    KV head the contraction is too thin for it to beat the warp-level MMAs
+//    (each tcgen05.mma holds its issuing thread ~95 cycles whatever its N).
 //  * Every wait is bounded; a timeout or a bad block id sets a bit in the
 //    device error word and the kernel returns without trapping.
 #include <cuda.h>
