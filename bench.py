@@ -636,7 +636,6 @@ def measure_decode(args, workload, rank, world, local, device, full=True):
     assert pkv.device_error() == 0, "device error during warm-up"
 
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     launches = 0
     n_cow = 0
@@ -652,7 +651,7 @@ def measure_decode(args, workload, rank, world, local, device, full=True):
             st = steps[i % n_distinct]
             flush()
             ev_s[k].record(stream)
-            step(i, ev_a[k])
+            step(i)
             ev_e[k].record(stream)
             launches += 3 + (1 if st["pairs"] is not None else 0)
             n_cow += 0 if st["pairs"] is None else int(st["pairs"].shape[0])
@@ -661,10 +660,25 @@ def measure_decode(args, workload, rank, world, local, device, full=True):
             alg_attn.append(allb)
             th_tokens += int(st["lens_host"].sum()) * Hq * q_len
         torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        # the attention launch (+ its split merge) alone, for the roofline:
+        # the same inputs, L2 flushed before each (inside a step it overlaps
+        # its set-up with the append's tail, which an event between the two
+        # would both split and serialise)
+        ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for k in range(args.steps):
+            st = steps[(args.warmup + k) % n_distinct]
+            flush()
+            ev_a[k].record(stream)
+            attention_call(pkv, wl, st["q"], st["tables"], st["lens"], out, ws, q_len, kq, ksc)
+            ev_b[k].record(stream)
+        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     step_ms = [ev_s[k].elapsed_time(ev_e[k]) for k in range(args.steps)]
-    attn_ms = [ev_a[k].elapsed_time(ev_e[k]) for k in range(args.steps)]
+    attn_ms = [ev_a[k].elapsed_time(ev_b[k]) for k in range(args.steps)]
     err = pkv.device_error()
     assert err == 0, f"device error word {err}"
     total_ms = sum(step_ms)
@@ -711,6 +725,8 @@ def measure_decode(args, workload, rank, world, local, device, full=True):
                          "traffic": ncu_traffic(workload),
                          "kernel": "paged_attention_kernel + lse_merge_kernel",
                          "attention_ms": round(attn_avg_ms, 5),
+                         "timing": "the attention launch and its merge alone, a loop of `steps` "
+                                   "launches after the step loop, L2 flushed before each",
                          "peak_kind": peak_kind},
             "gpu_launches": launches,
             "clocks": clk.summary(),
@@ -766,6 +782,11 @@ def decode_step(pkv, wl, q, k_new, v_new, slots, tables, lens, pairs, out, ws, q
         pkv.paged_kv_append_q8k(k_new, v_new, slots, ksc, kq, wl.v_pool)
     if ev is not None:
         ev.record(stream)
+    attention_call(pkv, wl, q, tables, lens, out, ws, q_len, kq, ksc)
+
+
+def attention_call(pkv, wl, q, tables, lens, out, ws, q_len, kq, ksc):
+    """The attention launch of a decode step (+ its split merge)."""
     if kq is not None:
         pkv.paged_attention_q8k(q, kq, ksc, wl.v_pool, tables, lens, wl.scale, q_len, out=out,
                                 workspace=ws, consumer=CONSUMER)

@@ -315,8 +315,16 @@ int paged_prefill_attention(const void* q, const void* k_pool, const void* v_poo
  *   grid_ctas        persistent CTAs (default: SMs x CTAs per SM);
  *   min_split_blocks smallest run of work units one CTA takes (default 16),
  *                    lower values force more context splits (and merges);
- *   use_pdl          1: launch the merge with programmatic dependent launch
- *                    (default), -1: plain launch;
+ *   use_pdl          1 (default): programmatic dependent launch for both
+ *                    launches: the attention kernel may start its set-up
+ *                    (reading context_lens and block_tables) while the
+ *                    preceding kernel in the stream runs, if that kernel
+ *                    allows it (the library's append kernels do), and waits
+ *                    for that kernel before its first read of q or the pools;
+ *                    the split merge overlaps the attention kernel's tail.
+ *                    -1: plain launches (use it when a preceding kernel of
+ *                    your own triggers dependents early and writes
+ *                    context_lens or block_tables after that);
  *   seg_cost_blocks  fixed cost, in blocks, charged to every (sequence,
  *                    kv-head) when work is divided among CTAs (default: 128
  *                    tokens' worth, 256 over an int8 K pool with several

@@ -16,6 +16,7 @@
 
 #include "../../include/paged_kv.h"
 #include "kv_device.h"
+#include "kv_ptx.cuh"
 #include "kv_status.h"
 
 namespace {
@@ -31,6 +32,9 @@ __global__ void append_kernel(const uint4* __restrict__ k_new, const uint4* __re
                               uint4* __restrict__ v_pool, int32_t T, int32_t Hkv,
                               int32_t chunks_per_row, int32_t bs, int64_t num_slots, int* err)
 {
+    // a decode-attention launch that follows may start its set-up (it waits
+    // for this grid before it reads the pools)
+    pkv::pdl_launch_dependents();
     // one thread per 16-byte chunk of one (token, head) row, K and V together
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t per_tok = (int64_t)Hkv * chunks_per_row;
@@ -88,6 +92,7 @@ __global__ void append_q8k_kernel(const uint4* __restrict__ k_new, const uint4* 
                                   uint4* __restrict__ v_pool, int32_t T, int32_t Hkv,
                                   int32_t chunks_per_row, int32_t bs, int64_t num_slots, int* err)
 {
+    pkv::pdl_launch_dependents();  // as in append_kernel
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t per_tok = (int64_t)Hkv * chunks_per_row;
     if (i >= (int64_t)T * per_tok) return;

@@ -174,7 +174,10 @@ struct Cfg {
     static constexpr int TSLOT_OFF = UB_OFF + UM_NBARS * 8; // its tensor-memory base address
     static constexpr int SMEM_USED = TSLOT_OFF + (UMR ? 16 : 0);
     static_assert(!UMR || 128 * D * 4 <= Q_OFF, "the segment-end slices fit a stage's K and V");
-    static_assert(!NR8 || TW * OBUF_SLICE * 4 <= STAGE_BYTES, "per-warp merge slices fit a stage");
+    // merge slices at a segment end: one per token warp, or, when TW of them
+    // do not fit a stage, one per pair of warps (w and w + TW/2, added in place)
+    static constexpr int MSLOTS = (NR8 && TW * OBUF_SLICE * 4 > STAGE_BYTES) ? TW / 2 : TW;
+    static_assert(!NR8 || MSLOTS * OBUF_SLICE * 4 <= STAGE_BYTES, "merge slices fit a stage");
     static constexpr int SMEM_ALLOC = SMEM_USED + 1024;    // room to align the base
 };
 
@@ -535,6 +538,10 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
                 nid[k] = load_id(nxt[k]);
                 ++nnxt;
             }
+        // Everything above reads only the lengths and block tables; the pools
+        // (and q) may still be being written by the grid this launch depends
+        // on (a cache append launched just before): wait for it here.
+        pdl_wait();
         while (ncur > 0 && ok) {
 #pragma unroll
             for (int k = 0; k < kLA; ++k) {
@@ -722,7 +729,7 @@ __device__ void store_segment_slices(const Params& p, const StageMeta& md, const
         const int d0 = (idx % (C::D / 8)) * 8;
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
 #pragma unroll
-        for (int w = 0; w < C::TW; ++w) {
+        for (int w = 0; w < C::MSLOTS; ++w) {
             const float4* src = reinterpret_cast<const float4*>(slices + (w * C::RP + R) * C::OB_STRIDE + d0);
             const float4 x = src[0], y = src[1];
             a = make_float4(a.x + x.x, a.y + x.y, a.z + x.z, a.w + x.w);
@@ -1529,19 +1536,31 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
                 }
             named_bar_sync(1, C::NCW * 32);  // every warp done with the stage's tiles
             float* slices = reinterpret_cast<float*>(smem + stage * C::STAGE_BYTES);
+            // this warp's o times its factor into slot qw mod MSLOTS: written by
+            // the upper warps first, then added to by the lower ones (a fixed
+            // order: bit-reproducible)
+            auto put = [&](bool add) {
 #pragma unroll
-            for (int nt = 0; nt < NR; ++nt) {
-                const float f0 = row_factor<C>(mlb, nt * 8 + 2 * tig, m[nt][0]);
-                const float f1 = row_factor<C>(mlb, nt * 8 + 2 * tig + 1, m[nt][1]);
-                float* r0 = slices + (qw * C::RP + nt * 8 + 2 * tig) * C::OB_STRIDE + gid;
-                float* r1 = r0 + C::OB_STRIDE;
+                for (int nt = 0; nt < NR; ++nt) {
+                    const float f0 = row_factor<C>(mlb, nt * 8 + 2 * tig, m[nt][0]);
+                    const float f1 = row_factor<C>(mlb, nt * 8 + 2 * tig + 1, m[nt][1]);
+                    float* r0 = slices + ((qw % C::MSLOTS) * C::RP + nt * 8 + 2 * tig) * C::OB_STRIDE + gid;
+                    float* r1 = r0 + C::OB_STRIDE;
 #pragma unroll
-                for (int np = 0; np < KS; ++np) {
-                    r0[16 * np] = O[np][nt][0] * f0;
-                    r1[16 * np] = O[np][nt][1] * f1;
-                    r0[16 * np + 8] = O[np][nt][2] * f0;
-                    r1[16 * np + 8] = O[np][nt][3] * f1;
+                    for (int np = 0; np < KS; ++np) {
+                        r0[16 * np] = (add ? r0[16 * np] : 0.f) + O[np][nt][0] * f0;
+                        r1[16 * np] = (add ? r1[16 * np] : 0.f) + O[np][nt][1] * f1;
+                        r0[16 * np + 8] = (add ? r0[16 * np + 8] : 0.f) + O[np][nt][2] * f0;
+                        r1[16 * np + 8] = (add ? r1[16 * np + 8] : 0.f) + O[np][nt][3] * f1;
+                    }
                 }
+            };
+            if constexpr (C::MSLOTS == C::TW) {
+                put(false);
+            } else {
+                if (qw >= C::MSLOTS) put(false);
+                named_bar_sync(1, C::NCW * 32);
+                if (qw < C::MSLOTS) put(true);
             }
             named_bar_sync(1, C::NCW * 32);
             store_segment_slices<C>(p, md, slices, mlb, tid);
@@ -2276,18 +2295,31 @@ int launch(const CUtensorMap& tk, const CUtensorMap& tv, const Params& prm, int 
             configured |= 1ull << dev;
         }
     }
-    paged_attention_kernel<C><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(tk, tv, prm);
-    int rc = kv_cuda_check(cudaGetLastError(), "paged_attention_kernel launch");
-    if (rc != KV_OK) return rc;
+    // With PDL the launch may start while the preceding kernel in the stream
+    // runs, once that kernel allows it (the library's append kernels do at
+    // entry): the set-up (length scan, block-table reads) overlaps its tail,
+    // and the loader waits for it before the first read of the pools.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    {
+        cudaLaunchConfig_t acfg = {};
+        acfg.gridDim = dim3(grid);
+        acfg.blockDim = dim3(C::THREADS);
+        acfg.dynamicSmemBytes = C::SMEM_ALLOC;
+        acfg.stream = stream;
+        acfg.attrs = attr;
+        acfg.numAttrs = pdl ? 1 : 0;
+        int rc = kv_cuda_check(cudaLaunchKernelEx(&acfg, paged_attention_kernel<C>, tk, tv, prm),
+                               "paged_attention_kernel launch");
+        if (rc != KV_OK) return rc;
+    }
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3((unsigned)((prm.rows * (C::D / 8) + 31) / 32 * 32));  // <= 512
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
     return kv_cuda_check(cudaLaunchKernelEx(&cfg, lse_merge_kernel<C::D, C::RP>, prm),
