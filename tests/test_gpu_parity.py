@@ -199,6 +199,55 @@ def test_tiny_config_full_with_append():
     assert_close(out2, ref2, "tiny after append")
 
 
+@pytest.mark.parametrize("name,B", [("llama70b_gqa", 64), ("llama7b_mha", 32)])
+def test_attention_launched_behind_the_append_reads_the_new_token(name, B):
+    """The attention launch may start its set-up while the append just before
+    it in the stream still runs (programmatic dependent launch); its loader
+    must wait for the append before reading the pools.  Each sequence appends
+    a key aligned with its queries, dominating every other score, into a slot
+    that held NaN: a read before the append lands gives NaN or a far-off
+    output, a correct one gives (nearly) the new token's V."""
+    from workloads import CONFIGS
+    rng = np.random.Generator(np.random.PCG64(B))
+    bs = CONFIGS[name].bs
+    lens = rng.integers(100, 900, size=B).astype(np.int32)
+    lens[lens % bs == 0] += 1                      # room left in each last block
+    wl = make_workload(name, "cuda", lens=lens, seed=61 + B)
+    Hkv, D = wl.k_pool.shape[1], wl.k_pool.shape[3]
+    G = wl.q.shape[2] // Hkv
+    # the queries of each (sequence, kv head) share a direction u; the new key is 100 u
+    g = torch.Generator(device="cpu")
+    g.manual_seed(5)
+    u = torch.randn((B, Hkv, D), generator=g, dtype=torch.float64)
+    u /= u.norm(dim=-1, keepdim=True)
+    q = 0.5 * wl.q.double().cpu() + 4.0 * u.repeat_interleave(G, dim=1)[:, None, :, :]
+    wl.q = q.to(torch.float16).cuda()
+    k_new = (100.0 * u).to(torch.float16)
+    v_new = normal_fp16((B, Hkv, D), 62, "cpu")
+    blk = np.array([wl.block_tables[s, lens[s] // bs] for s in range(B)], np.int64)
+    off = (lens % bs).astype(np.int64)
+    slots = blk * bs + off
+    k0, v0 = wl.k_pool.cpu().numpy(), wl.v_pool.cpu().numpy()
+    assert np.isnan(k0[blk, :, off, :]).all() and np.isnan(v0[blk, :, off, :]).all()
+    ref_k, ref_v = oracle.append(k0, v0, k_new.numpy(), v_new.numpy(), slots)
+    new_lens = (lens + 1).astype(np.int32)
+    # every device input in place before the two launches, which run back to back
+    kd, vd, sd = k_new.cuda(), v_new.cuda(), torch.as_tensor(slots, device="cuda")
+    bt = torch.as_tensor(wl.block_tables, device="cuda")
+    cl = torch.as_tensor(new_lens, device="cuda")
+    out = torch.empty_like(wl.q)
+    torch.cuda.synchronize()
+    pkv.paged_kv_append(kd, vd, sd, wl.k_pool, wl.v_pool)
+    pkv.paged_decode_attention(wl.q, wl.k_pool, wl.v_pool, bt, cl, wl.scale, out=out)
+    torch.cuda.synchronize()
+    assert pkv.device_error() == 0
+    ref = oracle.paged_attention(wl.q.cpu().numpy(), ref_k, ref_v, wl.block_tables, new_lens,
+                                 scale=wl.scale)
+    assert_close(out, ref, f"{name} behind the append")
+    want = v_new.repeat_interleave(G, dim=1).double().numpy()
+    assert np.abs(out[:, 0].cpu().double().numpy() - want).max() < 0.02
+
+
 @pytest.mark.parametrize("Hq,Hkv,D,bs,q_len", [
     (4, 4, 64, 16, 1), (8, 8, 128, 8, 1),           # FMA path (one row per KV head)
     (8, 2, 64, 16, 1), (64, 8, 128, 16, 1),          # tensor-core path, one m16 tile
