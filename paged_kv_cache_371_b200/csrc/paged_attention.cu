@@ -62,6 +62,7 @@ constexpr int kSmemBudget = 225 * 1024;
 constexpr int kSegCostTokens = 128;
 constexpr int kSegCostTokensQ8 = 256;
 constexpr float kNegInf = -__builtin_huge_valf();
+constexpr float kRescaleThreshold = 8.f;  // log2 units: weights stay below 2^8
 
 enum : int32_t { F_FIRST = 1, F_LAST = 2, F_WHOLE = 4, F_END = 8 };
 
@@ -1449,11 +1450,17 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
             // mask: a token counts if the row may see it and this stage loaded it
             const int pos0 = md.t0 + tb + gid;
             const int st_end = md.t0 + md.ntok;
+            // Each row keeps a reference maximum m shared by the 8 lanes that
+            // hold its tokens; it is raised (a shuffle reduction, O rescaled)
+            // only when some score of the sub-tile passes it by more than
+            // 2^kRescaleThreshold, so most sub-tiles cost one vote and the
+            // weights stay below 2^kRescaleThreshold (exact after the final
+            // division by l, which uses the same reference)
             bool rescale = false;
-            float alpha[NR][2], mu[NR][2];
+            float alpha[NR][2], mu[NR][2], mx[NR][2];
+            bool over = false;
 #pragma unroll
             for (int nt = 0; nt < NR; ++nt) {
-                float mx[2];
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
                     const int lm = min(lim[nt][i], st_end);
@@ -1461,19 +1468,28 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
                     const float c1 = C::KQ ? S[nt][2 + i] - corr[nt][i] : S[nt][2 + i];
                     S[nt][i] = pos0 < lm ? c0 * sl2 : kNegInf;
                     S[nt][2 + i] = pos0 + 8 < lm ? c1 * sl2 : kNegInf;
-                    mx[i] = fmaxf(S[nt][i], S[nt][2 + i]);
+                    mx[nt][i] = fmaxf(S[nt][i], S[nt][2 + i]);
+                    over |= mx[nt][i] > m[nt][i] + kRescaleThreshold;
+                    alpha[nt][i] = 1.f;
+                    mu[nt][i] = m[nt][i] == kNegInf ? 0.f : m[nt][i];
                 }
+            }
+            if (__any_sync(0xffffffffu, over)) {
 #pragma unroll
-                for (int off = 4; off < 32; off <<= 1)
+                for (int nt = 0; nt < NR; ++nt) {
 #pragma unroll
-                    for (int i = 0; i < 2; ++i) mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], off));
+                    for (int off = 4; off < 32; off <<= 1)
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const float mn = fmaxf(m[nt][i], mx[i]);
-                    mu[nt][i] = mn == kNegInf ? 0.f : mn;
-                    alpha[nt][i] = ex2(m[nt][i] - mu[nt][i]);
-                    m[nt][i] = mn;
-                    rescale |= alpha[nt][i] != 1.f;
+                        for (int i = 0; i < 2; ++i)
+                            mx[nt][i] = fmaxf(mx[nt][i], __shfl_xor_sync(0xffffffffu, mx[nt][i], off));
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const float mn = fmaxf(m[nt][i], mx[nt][i]);
+                        mu[nt][i] = mn == kNegInf ? 0.f : mn;
+                        alpha[nt][i] = ex2(m[nt][i] - mu[nt][i]);
+                        m[nt][i] = mn;
+                        rescale |= alpha[nt][i] != 1.f;
+                    }
                 }
             }
             uint32_t pb[NR][2];
@@ -1603,7 +1619,6 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
 enum : uint32_t { UM_S = 0, UM_P = 128, UM_O = 256, UM_Q = 384, UM_COLS = 512 };
 enum : int { UB_S_FULL = 0, UB_S_FREE = 1, UB_P_FULL = 2, UB_O_DONE = 4, UB_Q_READY = 6, UB_KDQ = 7,
              UB_EP = 8, UB_DRAIN = 9 };
-constexpr float kRescaleThreshold = 8.f;  // log2 units: weights stay below 2^8
 
 template <class C>
 __device__ void consumer_um(const Params& p, uint8_t* smem, uint32_t tmem, volatile int* abort_flag)
