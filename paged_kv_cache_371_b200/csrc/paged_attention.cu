@@ -2354,9 +2354,9 @@ int dispatch_rows(int rows, bool um, const CUtensorMap& tk, const CUtensorMap& t
         }
     }
     // Tensor-core paths: 128-token stages (8 token warps for one row tile, 4
-    // warps of two 16-token sub-tiles for two or three; 256 tokens for one
-    // row tile over int8 keys); more than 24 rows keep the rows-as-M consumer
-    // (its accumulators fit 255 registers).
+    // warps of two 16-token sub-tiles for two or three; 256 tokens over int8
+    // keys for one row tile or three); more than 24 rows keep the rows-as-M
+    // consumer (its accumulators fit 255 registers).
     if (rows == 1) return launch<Cfg<D, BS, 1, true, KQ>>(tk, tv, prm, grid, pdl, st);
     if (rows <= 8) {
         // int8 keys stream 3/4 of the bytes per token: 256-token stages
@@ -2364,7 +2364,11 @@ int dispatch_rows(int rows, bool um, const CUtensorMap& tk, const CUtensorMap& t
         else return launch<Cfg<D, BS, 1, false, KQ, 1, 8, 1>>(tk, tv, prm, grid, pdl, st);
     }
     if (rows <= 16) return launch<Cfg<D, BS, 1, false, KQ, 2, 4, 2>>(tk, tv, prm, grid, pdl, st);
-    if (rows <= 24) return launch<Cfg<D, BS, 1, false, KQ, 3, 4, 2>>(tk, tv, prm, grid, pdl, st);
+    if (rows <= 24) {
+        // int8 keys: 256-token stages (two of them fit the shared memory)
+        if constexpr (KQ) return launch<Cfg<D, BS, 1, false, KQ, 3, 4, 4>>(tk, tv, prm, grid, pdl, st);
+        else return launch<Cfg<D, BS, 1, false, KQ, 3, 4, 2>>(tk, tv, prm, grid, pdl, st);
+    }
     return launch<Cfg<D, BS, 2, false, KQ>>(tk, tv, prm, grid, pdl, st);
 }
 
