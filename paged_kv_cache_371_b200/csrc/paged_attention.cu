@@ -87,7 +87,7 @@ struct Params {
 };
 
 template <int D_, int BS_, int MT_, bool FMA_, bool KQ_ = false, int NR8_ = 0, int TW_ = 0,
-          int SUBS_ = 1, int UMR_ = 0>
+          int SUBS_ = 1, int UMR_ = 0, int HP_ = 1>
 struct Cfg {
     static constexpr int D = D_, BS = BS_, MT = MT_;
     static constexpr bool FMA = FMA_;
@@ -103,6 +103,13 @@ struct Cfg {
                            (UMR == 8 || UMR == 16 || UMR == 32)),
                   "the tcgen05 consumer serves head_dim 128, 8/16/32 padded rows");
     static_assert(!KQ || D == 128, "int8 K pools are served at head_dim 128");
+    // HP = 2: a unit of work is a pair of adjacent KV heads of a block, staged
+    // by one copy of both heads' rows (they are contiguous in the pool): half
+    // the copies per byte, for 8-token blocks.  Row tile h holds the 8 query
+    // rows of head h of the pair (GQA groups of 8, one query per sequence).
+    static constexpr int HP = HP_;
+    static_assert(HP == 1 || (HP == 2 && NR8_ == 2 && !UMR && D == 128),
+                  "head pairs: two row tiles of one head each, head_dim 128");
     static constexpr int NH = D / 64;                       // 64-column halves per row
     // consumer warps along the tokens of a stage (16 tokens each) and tokens
     // per stage: the FMA consumers run latency-bound matrix-vector work and
@@ -127,23 +134,24 @@ struct Cfg {
     static constexpr int WARPS_PER_SUBPART = (THREADS / 32 + 3) / 4;
     static constexpr int MAXREG_RAW = (16384 / (32 * WARPS_PER_SUBPART)) / 8 * 8;
     static constexpr int MAXREG = MAXREG_RAW > 255 ? 255 : MAXREG_RAW;
-    static constexpr int TILE_BYTES = BS * D * 2;           // one (block, kv-head) fp16 tile
-    static constexpr int KV_BYTES = TS * D * 2;             // fp16 K (or V) bytes per stage
-    static constexpr int K_TILE_BYTES = KQ ? BS * D : TILE_BYTES;
+    static constexpr int TROWS = BS * HP;                   // pool rows of one staged tile
+    static constexpr int TILE_BYTES = TROWS * D * 2;        // one (block, kv-head[s]) fp16 tile
+    static constexpr int KV_BYTES = TS * HP * D * 2;        // fp16 K (or V) bytes per stage
+    static constexpr int K_TILE_BYTES = KQ ? TROWS * D : TILE_BYTES;
     // the tcgen05 consumer keeps fp16 room for K also over int8 codes: they
     // land in its upper half and are widened in place
-    static constexpr int K_BYTES = (KQ && !UMR) ? TS * D : KV_BYTES;
+    static constexpr int K_BYTES = (KQ && !UMR) ? TS * HP * D : KV_BYTES;
     // one 64-column half of a stage's K or V in the tcgen05 consumer's layout
     // ([half][token][128 B], the MMA's 128-byte-swizzle K-major / MN-major form)
     static constexpr int UM_HALF = TS * 128;
     static constexpr int V_OFF = K_BYTES;                   // stage: K, V, query rows
     // query rows of a segment, one per 16-byte-padded row (conflict-free ldmatrix)
     static constexpr int QROW = D * 2 + 16;
-    static constexpr int Q_BYTES = (RP * QROW + 1023) / 1024 * 1024;
+    static constexpr int Q_BYTES = (RP * QROW + (KQ ? HP * D * 4 : 0) + 1023) / 1024 * 1024;
     static constexpr int Q_OFF = K_BYTES + KV_BYTES;
-    // int8 keys: the segment's channel scales (D fp32) follow the query rows
+    // int8 keys: the segment's channel scales (D fp32 per head) follow the query rows
     static constexpr int SC_OFF = Q_OFF + RP * QROW;
-    static_assert(!KQ || RP * QROW + D * 4 <= Q_BYTES, "room for the channel scales");
+    static_assert(!KQ || RP * QROW + HP * D * 4 <= Q_BYTES, "room for the channel scales");
     static constexpr int STAGE_BYTES = Q_OFF + Q_BYTES;
     // floats per obuf row (the transposed consumer's scalar stores of rows
     // 2*tig, 2*tig+1 are conflict-free when 2 * OB_STRIDE = 8 mod 32)
@@ -215,21 +223,22 @@ __device__ __forceinline__ int64_t warp_incl_scan64(int64_t v, int lane)
 // Shared-memory layout of a staged tile: one (block, kv-head) tile is its
 // BS rows of D fp16, i.e. BS * NH units of 128 bytes in global order (one TMA
 // copy of the contiguous tile).  The 128-byte swizzle stores 16-byte chunk c
-// of unit u at chunk position c ^ (u mod 8).  Byte offset, inside a stage's K
-// (or V) area, of chunk cg (0 .. D/8-1) of stage token `tok`:
+// of unit u at chunk position c ^ (u mod 8).  A head pair's tile is head 0's
+// BS rows, then head 1's.  Byte offset, inside a stage's K (or V) area, of
+// chunk cg (0 .. D/8-1) of stage token `tok` of head h of the tile:
 template <class C>
-__device__ __forceinline__ uint32_t tile_chunk(int tok, int cg)
+__device__ __forceinline__ uint32_t tile_chunk(int tok, int cg, int h = 0)
 {
-    const int r = tok % C::BS;
+    const int r = h * C::BS + tok % C::BS;  // row of head h of the pair
     const int u = r * C::NH + (cg >> 3);
     return (uint32_t)((tok / C::BS) * C::TILE_BYTES + u * 128 + (((cg & 7) ^ (u & 7)) << 4));
 }
 
 // The same for an int8 K tile: one 128-byte unit (D = 128 codes) per token.
 template <class C>
-__device__ __forceinline__ uint32_t tile_chunk_k8(int tok, int cg)
+__device__ __forceinline__ uint32_t tile_chunk_k8(int tok, int cg, int h = 0)
 {
-    const int r = tok % C::BS;
+    const int r = h * C::BS + tok % C::BS;
     return (uint32_t)((tok / C::BS) * C::K_TILE_BYTES + r * 128 + ((cg ^ (r & 7)) << 4));
 }
 
@@ -563,7 +572,7 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
                 const bool firstst = (d.flags & F_FIRST) != 0;
                 const uint32_t qbytes = (uint32_t)(p.G * C::D * 2);  // query bytes per window row
                 uint32_t bytes = (uint32_t)__popc(lmask) * (uint32_t)(C::K_TILE_BYTES + C::TILE_BYTES);
-                if (firstst) bytes += qbytes * (uint32_t)p.q_len + (C::KQ ? C::D * 4 : 0);
+                if (firstst) bytes += qbytes * (uint32_t)p.q_len + (C::KQ ? C::HP * C::D * 4 : 0);
                 const uint32_t full = full0 + stage * 8;
                 if (lane == 0) {
                     StageMeta& md = smeta[stage];
@@ -579,7 +588,7 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
                 __syncwarp();
                 const uint32_t st = sbase + stage * C::STAGE_BYTES;
                 if (load) {
-                    const int32_t y = (id * p.Hkv + d.kvh) * C::BS;
+                    const int32_t y = (id * p.Hkv + d.kvh) * C::TROWS;
                     if constexpr (C::UMR > 0) {
                         // block `lane` -> rows [lane*BS, lane*BS+BS) of each 64-column
                         // half; int8 codes (128 per row) into the upper half of K
@@ -607,8 +616,9 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
                         p.q + (((int64_t)d.s * p.q_len + j) * p.Hq + (int64_t)d.kvh * p.G + g) * C::D;
                     bulk_load(st + C::Q_OFF + lane * C::QROW, src, C::D * 2, full);
                 }
-                if (C::KQ && firstst && lane == 31)  // the KV head's channel scales
-                    bulk_load(st + C::SC_OFF, p.k_scale + (int64_t)d.kvh * C::D, C::D * 4, full);
+                if (C::KQ && firstst && lane == 31)  // the KV head's (pair's) channel scales
+                    bulk_load(st + C::SC_OFF, p.k_scale + (int64_t)d.kvh * C::HP * C::D, C::HP * C::D * 4,
+                              full);
                 ++k_issued;
             }
 #pragma unroll
@@ -1349,13 +1359,14 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
 #pragma unroll
                 for (int nt = 0; nt < NR; ++nt) {
                     const uint8_t* qr = smem + stage * C::STAGE_BYTES + C::Q_OFF + (nt * 8 + gid) * C::QROW;
+                    const float* sch = sc + (C::HP > 1 ? nt * C::D : 0);  // row tile nt's head
 #pragma unroll
                     for (int ks = 0; ks < KS; ++ks) {
                         const int d = 16 * ks + 4 * tig;
                         qb[ks][nt][0] = scale_h2(*reinterpret_cast<const uint32_t*>(qr + d * 2),
-                                                 *reinterpret_cast<const float2*>(sc + d));
+                                                 *reinterpret_cast<const float2*>(sch + d));
                         qb[ks][nt][1] = scale_h2(*reinterpret_cast<const uint32_t*>(qr + d * 2 + 4),
-                                                 *reinterpret_cast<const float2*>(sc + d + 2));
+                                                 *reinterpret_cast<const float2*>(sch + d + 2));
                     }
                 }
             }
@@ -1413,6 +1424,23 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
                 float (&S)[NR][4] = Sc[ks % NCH];
+                if constexpr (C::HP > 1) {
+                    // row tile nt is head nt of the pair: its own K rows
+#pragma unroll
+                    for (int nt = 0; nt < NR; ++nt) {
+                        uint32_t a[4];
+                        if constexpr (C::KQ) {
+                            i8x4_to_h2x2_biased(lds_u32(st + tile_chunk_k8<C>(tb + gid, ks, nt) + 4 * tig), a[0],
+                                                a[2]);
+                            i8x4_to_h2x2_biased(lds_u32(st + tile_chunk_k8<C>(tb + gid + 8, ks, nt) + 4 * tig),
+                                                a[1], a[3]);
+                        } else {
+                            ldsm_x4(st + tile_chunk<C>(a_tok, 2 * ks + a_sel, nt), a[0], a[1], a[2], a[3]);
+                        }
+                        mma_16816(S[nt], a, qb[ks][nt][0], qb[ks][nt][1]);
+                    }
+                    continue;
+                }
                 uint32_t a[4];
                 if constexpr (C::KQ) {
                     // tokens gid and gid + 8, dims 16ks + 4tig .. +3 (permuted order)
@@ -1519,11 +1547,22 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
             const bool v_ok = v_i < nv;
 #pragma unroll
             for (int np = 0; np < KS; ++np) {
-                const uint32_t addr = v_ok ? st + C::V_OFF + tile_chunk<C>(v_tok, 2 * np + v_sel) : zero_row;
-                uint32_t a[4];
-                ldsm_x4_trans(addr, a[0], a[1], a[2], a[3]);
+                if constexpr (C::HP > 1) {
 #pragma unroll
-                for (int nt = 0; nt < NR; ++nt) mma_16816(O[np][nt], a, pb[nt][0], pb[nt][1]);
+                    for (int nt = 0; nt < NR; ++nt) {  // head nt's V rows
+                        const uint32_t addr =
+                            v_ok ? st + C::V_OFF + tile_chunk<C>(v_tok, 2 * np + v_sel, nt) : zero_row;
+                        uint32_t a[4];
+                        ldsm_x4_trans(addr, a[0], a[1], a[2], a[3]);
+                        mma_16816(O[np][nt], a, pb[nt][0], pb[nt][1]);
+                    }
+                } else {
+                    const uint32_t addr = v_ok ? st + C::V_OFF + tile_chunk<C>(v_tok, 2 * np + v_sel) : zero_row;
+                    uint32_t a[4];
+                    ldsm_x4_trans(addr, a[0], a[1], a[2], a[3]);
+#pragma unroll
+                    for (int nt = 0; nt < NR; ++nt) mma_16816(O[np][nt], a, pb[nt][0], pb[nt][1]);
+                }
             }
         }
         }
@@ -2379,6 +2418,15 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // benchmark shape (8, 20 and 32 rows; fp16 and int8 keys).
 bool default_tcgen05(int, bool) { return false; }
 
+// Head pairs: for 8-token blocks (one block of one head is a 2 KB fp16 copy,
+// 1 KB of int8 codes; the pair's copies are twice that, half the copies per
+// byte), head_dim 128, GQA groups of exactly 8 (one row tile per head),
+// decode (one query), the warp-level consumer.
+bool use_head_pairs(int D, int BS, int G, int q_len, int Hkv, bool, bool um)
+{
+    return D == 128 && BS == 8 && G == 8 && q_len == 1 && Hkv % 2 == 0 && !um;
+}
+
 int attention_impl(const void* q, const void* k_pool, const void* v_pool,
                    const int32_t* block_tables, int32_t max_blocks_per_seq,
                    const int32_t* context_lens, int32_t q_len, float scale, void* out, int32_t B,
@@ -2422,11 +2470,16 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
     if (consumer < 0 || consumer > 2)
         return kv_fail(KV_ERR_INVALID, "paged attention: opts.consumer must be 0, 1 or 2");
     const bool um = D == 128 && rows > 1 && (consumer == 2 || (consumer == 0 && default_tcgen05(rows, k_scale != nullptr)));
+    // head pairs (8-token blocks, GQA groups of 8, one query per sequence):
+    // the kernel sees Hkv / 2 heads of 2 * G query rows, each staged tile
+    // both heads' rows of a block (see Cfg::HP)
+    const bool hp = use_head_pairs(D, BS, G, q_len, Hkv, k_scale != nullptr, um);
     CUtensorMap tk, tv;
     const uint64_t prow = (uint64_t)num_blocks * Hkv * BS;
-    int rc = pool_tmap(k_pool, prow, D, BS, &tk, k_scale ? TMAP_INT8 : (um ? TMAP_HALF : TMAP_TILE));
+    const int trows = hp ? 2 * BS : BS;  // pool rows per staged tile
+    int rc = pool_tmap(k_pool, prow, D, trows, &tk, k_scale ? TMAP_INT8 : (um ? TMAP_HALF : TMAP_TILE));
     if (rc != KV_OK) return rc;
-    rc = pool_tmap(v_pool, prow, D, BS, &tv, um ? TMAP_HALF : TMAP_TILE);
+    rc = pool_tmap(v_pool, prow, D, trows, &tv, um ? TMAP_HALF : TMAP_TILE);
     if (rc != KV_OK) return rc;
 
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -2446,9 +2499,9 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
     prm.B = B;
     prm.q_len = q_len;
     prm.Hq = Hq;
-    prm.Hkv = Hkv;
-    prm.G = G;
-    prm.rows = rows;
+    prm.Hkv = hp ? Hkv / 2 : Hkv;
+    prm.G = hp ? 2 * G : G;
+    prm.rows = hp ? 2 * rows : rows;
     prm.num_blocks = num_blocks;
     prm.min_share = (opts && opts->min_split_blocks > 0) ? opts->min_split_blocks : 16;
     prm.seg_cost = (opts && opts->seg_cost_blocks != 0) ? (opts->seg_cost_blocks > 0 ? opts->seg_cost_blocks : 0)
@@ -2458,6 +2511,9 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
                                                             : kWaitLimitNs;
     const bool pdl = !(opts && opts->use_pdl < 0);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (hp)
+        return k_scale ? launch<Cfg<128, 8, 1, false, true, 2, 4, 2, 0, 2>>(tk, tv, prm, grid, pdl, st)
+                       : launch<Cfg<128, 8, 1, false, false, 2, 4, 1, 0, 2>>(tk, tv, prm, grid, pdl, st);
     if (k_scale)
         return BS == 8 ? dispatch_rows<128, 8, true>(rows, um, tk, tv, prm, grid, pdl, st)
                        : dispatch_rows<128, 16, true>(rows, um, tk, tv, prm, grid, pdl, st);
