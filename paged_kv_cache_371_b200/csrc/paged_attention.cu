@@ -2420,11 +2420,13 @@ bool default_tcgen05(int, bool) { return false; }
 
 // Head pairs: for 8-token blocks (one block of one head is a 2 KB fp16 copy,
 // 1 KB of int8 codes; the pair's copies are twice that, half the copies per
-// byte), head_dim 128, GQA groups of exactly 8 (one row tile per head),
-// decode (one query), the warp-level consumer.
-bool use_head_pairs(int D, int BS, int G, int q_len, int Hkv, bool, bool um)
+// byte) and for int8 keys over 16-token blocks (2 KB of codes), head_dim 128,
+// GQA groups of exactly 8 (one row tile per head), decode (one query), the
+// warp-level consumer.  Measured: fp16 over 16-token blocks (4 KB copies)
+// gains nothing from pairs.
+bool use_head_pairs(int D, int BS, int G, int q_len, int Hkv, bool int8_k, bool um)
 {
-    return D == 128 && BS == 8 && G == 8 && q_len == 1 && Hkv % 2 == 0 && !um;
+    return D == 128 && (BS == 8 || int8_k) && G == 8 && q_len == 1 && Hkv % 2 == 0 && !um;
 }
 
 int attention_impl(const void* q, const void* k_pool, const void* v_pool,
@@ -2511,9 +2513,11 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
                                                             : kWaitLimitNs;
     const bool pdl = !(opts && opts->use_pdl < 0);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (hp)
-        return k_scale ? launch<Cfg<128, 8, 1, false, true, 2, 4, 2, 0, 2>>(tk, tv, prm, grid, pdl, st)
-                       : launch<Cfg<128, 8, 1, false, false, 2, 4, 1, 0, 2>>(tk, tv, prm, grid, pdl, st);
+    if (hp) {
+        if (!k_scale) return launch<Cfg<128, 8, 1, false, false, 2, 4, 1, 0, 2>>(tk, tv, prm, grid, pdl, st);
+        return BS == 8 ? launch<Cfg<128, 8, 1, false, true, 2, 4, 2, 0, 2>>(tk, tv, prm, grid, pdl, st)
+                       : launch<Cfg<128, 16, 1, false, true, 2, 4, 2, 0, 2>>(tk, tv, prm, grid, pdl, st);
+    }
     if (k_scale)
         return BS == 8 ? dispatch_rows<128, 8, true>(rows, um, tk, tv, prm, grid, pdl, st)
                        : dispatch_rows<128, 16, true>(rows, um, tk, tv, prm, grid, pdl, st);
