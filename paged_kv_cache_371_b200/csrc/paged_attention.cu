@@ -1292,7 +1292,7 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
     float O[KS][NR][4];  // O^T tile (dims 16*np.., rows 8*nt..): d = gid(+8), r = 2tig(+1)
     uint32_t qb[C::QPERSIST ? 1 : KS][NR][2];  // B fragments of the query rows
     float m[NR][2], l[NR][2];
-    float corr[NR][2];  // int8 keys: bias * row sum of the scaled q
+    float corr[NR][2];  // int8 keys: bias * row sum of the scaled q, in log2 units (x scale)
     int lim[NR][2];
 
     // B fragments of k-steps ks, ks+1 of row tile nt from padded query rows at `rows`
@@ -1388,8 +1388,8 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
                     }
                     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
                     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                    corr[nt][0] = kCodeBias * __shfl_sync(0xffffffffu, acc, (2 * tig) * 4);
-                    corr[nt][1] = kCodeBias * __shfl_sync(0xffffffffu, acc, (2 * tig + 1) * 4);
+                    corr[nt][0] = kCodeBias * sl2 * __shfl_sync(0xffffffffu, acc, (2 * tig) * 4);
+                    corr[nt][1] = kCodeBias * sl2 * __shfl_sync(0xffffffffu, acc, (2 * tig + 1) * 4);
                 }
             }
 #pragma unroll
@@ -1475,15 +1475,20 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
                     for (int c = 1; c < NCH; ++c) v += Sc[c][nt][e];
                     S[nt][e] = v;
                 }
-            // mask: a token counts if the row may see it and this stage loaded it
+            // mask: a token counts if the row may see it and this stage loaded
+            // it; a sub-tile that every row sees whole (the usual case) skips it
             const int pos0 = md.t0 + tb + gid;
             const int st_end = md.t0 + md.ntok;
+            const bool whole = md.t0 + tb + 16 <= min(md.L - p.q_len + 1, st_end);
             // Each row keeps a reference maximum m shared by the 8 lanes that
             // hold its tokens; it is raised (a shuffle reduction, O rescaled)
             // only when some score of the sub-tile passes it by more than
             // 2^kRescaleThreshold, so most sub-tiles cost one vote and the
             // weights stay below 2^kRescaleThreshold (exact after the final
-            // division by l, which uses the same reference)
+            // division by l, which uses the same reference).  Scores stay raw
+            // dot products (over int8 keys: biased); the score in log2 units,
+            // raw * sl2 - corr (corr: the int8 bias in log2 units), is formed
+            // inside each exponential's argument by one FMA.
             bool rescale = false;
             float alpha[NR][2], mu[NR][2], mx[NR][2];
             bool over = false;
@@ -1491,12 +1496,12 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
             for (int nt = 0; nt < NR; ++nt) {
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
-                    const int lm = min(lim[nt][i], st_end);
-                    const float c0 = C::KQ ? S[nt][i] - corr[nt][i] : S[nt][i];
-                    const float c1 = C::KQ ? S[nt][2 + i] - corr[nt][i] : S[nt][2 + i];
-                    S[nt][i] = pos0 < lm ? c0 * sl2 : kNegInf;
-                    S[nt][2 + i] = pos0 + 8 < lm ? c1 * sl2 : kNegInf;
-                    mx[nt][i] = fmaxf(S[nt][i], S[nt][2 + i]);
+                    if (!whole) {
+                        const int lm = min(lim[nt][i], st_end);
+                        S[nt][i] = pos0 < lm ? S[nt][i] : kNegInf;
+                        S[nt][2 + i] = pos0 + 8 < lm ? S[nt][2 + i] : kNegInf;
+                    }
+                    mx[nt][i] = fmaf(fmaxf(S[nt][i], S[nt][2 + i]), sl2, C::KQ ? -corr[nt][i] : 0.f);
                     over |= mx[nt][i] > m[nt][i] + kRescaleThreshold;
                     alpha[nt][i] = 1.f;
                     mu[nt][i] = m[nt][i] == kNegInf ? 0.f : m[nt][i];
@@ -1523,8 +1528,10 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
             uint32_t pb[NR][2];
 #pragma unroll
             for (int nt = 0; nt < NR; ++nt) {
-                const float e0 = ex2(S[nt][0] - mu[nt][0]), e1 = ex2(S[nt][1] - mu[nt][1]);
-                const float e2 = ex2(S[nt][2] - mu[nt][0]), e3 = ex2(S[nt][3] - mu[nt][1]);
+                const float b0 = C::KQ ? mu[nt][0] + corr[nt][0] : mu[nt][0];
+                const float b1 = C::KQ ? mu[nt][1] + corr[nt][1] : mu[nt][1];
+                const float e0 = ex2(fmaf(S[nt][0], sl2, -b0)), e1 = ex2(fmaf(S[nt][1], sl2, -b1));
+                const float e2 = ex2(fmaf(S[nt][2], sl2, -b0)), e3 = ex2(fmaf(S[nt][3], sl2, -b1));
                 l[nt][0] = l[nt][0] * alpha[nt][0] + (e0 + e2);
                 l[nt][1] = l[nt][1] * alpha[nt][1] + (e1 + e3);
                 // P^T (tokens x rows) -> P (rows x tokens) fragments: b0 = P[gid][2tig..],
