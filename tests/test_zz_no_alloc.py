@@ -51,6 +51,8 @@ def _split_ctas(pkv, wl, bt, cl):
 @pytest.mark.parametrize("name,kw,warm_kw", [
     ("llama70b_gqa", {"B": 24, "max_len": 3000}, {"name": "llama7b_mha", "B": 5, "max_len": 900}),
     ("llama7b_mha", {"B": 8, "max_len": 2000}, {"name": "llama70b_gqa", "B": 40, "max_len": 700}),
+    # 8-token blocks: the head-pair form (two KV heads per staged tile, 16 rows)
+    ("llama70b_gqa_bs8", {"B": 24, "max_len": 3000}, {"name": "llama7b_mha", "B": 5, "max_len": 900}),
     # MQA at head_dim 128: 32 query rows per KV head, the largest shape the
     # fixed scratch admits; long enough that every CTA splits a context
     ("llama70b_gqa", {"lens": np.full(6, 9000, np.int32), "Hq": 32, "Hkv": 1, "seed": 41},
