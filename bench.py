@@ -823,19 +823,39 @@ def run_e2e(pkv, wl, steps, n_distinct, args, ws, stream, device, Hq, Hkv, D, bs
     parents = beam_parents(wl.B, BEAMS, n_total, seed) if beams else None
     n = steps[0]["q"].shape[0]
     cap = tables.shape[1]
-    # per-step q / K / V in pinned host memory (the model's outputs of the step)
-    host_qkv = [{k: st[k].cpu().pin_memory() for k in ("q", "k_new", "v_new")} for st in steps]
-    names = ("slots", "pairs", "tables", "lens")
-    stage = [{"slots": torch.empty(n, dtype=torch.int64).pin_memory(),
-              "pairs": torch.empty((n, 2), dtype=torch.int32).pin_memory(),
-              "tables": torch.empty((n, cap), dtype=torch.int32).pin_memory(),
-              "lens": torch.empty(n, dtype=torch.int32).pin_memory()} for _ in range(2)]
-    dbuf = []
-    for _ in range(2):
-        d = {k: torch.empty_like(steps[0][k]) for k in ("q", "k_new", "v_new")}
-        d.update({k: torch.empty(v.shape, dtype=v.dtype, device=device)
-                  for k, v in stage[0].items()})
-        dbuf.append(d)
+    # Each step's inputs travel in two copies: q / K / V (the model's outputs
+    # of the step, in one pinned block per distinct step) and the bookkeeping
+    # (slots, tables, lengths, then the copy-on-write pairs) in one pinned
+    # staging block per buffer; each tensor is a 256-byte-aligned view.
+    def layout(specs):
+        offs, o = {}, 0
+        for name, shape, dt in specs:
+            nbytes = int(np.prod(shape)) * torch.empty((), dtype=dt).element_size()
+            offs[name] = (o, shape, dt, nbytes)
+            o += (nbytes + 255) // 256 * 256
+        return offs, o
+
+    def views(buf, offs):
+        return {k: buf[o:o + nb].view(dt).view(shape) for k, (o, shape, dt, nb) in offs.items()}
+
+    qkv_offs, qkv_bytes = layout([(k, tuple(steps[0][k].shape), steps[0][k].dtype)
+                                  for k in ("q", "k_new", "v_new")])
+    meta_offs, meta_bytes = layout([("slots", (n,), torch.int64), ("tables", (n, cap), torch.int32),
+                                    ("lens", (n,), torch.int32), ("pairs", (n, 2), torch.int32)])
+    pairs_off = meta_offs["pairs"][0]
+    host_qkv = []
+    for st in steps:
+        hb = torch.empty(qkv_bytes, dtype=torch.uint8).pin_memory()
+        for k, v in views(hb, qkv_offs).items():
+            v.copy_(st[k].cpu())
+        host_qkv.append(hb)
+    stage_buf = [torch.empty(meta_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
+    stage = [views(b, meta_offs) for b in stage_buf]
+    dqkv = [torch.empty(qkv_bytes, dtype=torch.uint8, device=device) for _ in range(2)]
+    dmeta = [torch.empty(meta_bytes, dtype=torch.uint8, device=device) for _ in range(2)]
+    dbuf = [dict(views(dqkv[b], qkv_offs), **views(dmeta[b], meta_offs)) for b in range(2)]
+    data_bytes = sum(nb for (_, _, _, nb) in qkv_offs.values()) + sum(
+        meta_offs[k][3] for k in ("slots", "tables", "lens"))
     out0 = torch.empty((n, q_len, Hq, D), dtype=torch.float16, device=device)
     outs = [out0, torch.empty_like(out0)]
     houts = [torch.empty(out0.shape, dtype=out0.dtype).pin_memory() for _ in range(2)]
@@ -876,21 +896,15 @@ def run_e2e(pkv, wl, steps, n_distinct, args, ws, stream, device, Hq, Hkv, D, bs
         for k in range(k0, k0 + cnt):
             b = k % 2
             npairs = host_step(k, b)
-            h, sg, d = host_qkv[k % n_distinct], stage[b], dbuf[b]
+            d = dbuf[b]
             if k - k0 >= 2:
                 s_in.wait_event(ev_done[b])      # step k-2 finished reading buffer b
             with torch.cuda.stream(s_in):
-                nbytes = 0
-                for name, src in (("q", h["q"]), ("k_new", h["k_new"]), ("v_new", h["v_new"]),
-                                  ("slots", sg["slots"]), ("tables", sg["tables"]),
-                                  ("lens", sg["lens"])):
-                    d[name].copy_(src, non_blocking=True)
-                    nbytes += src.numel() * src.element_size()
-                pairs = None
-                if npairs:
-                    pairs = d["pairs"][:npairs]
-                    pairs.copy_(sg["pairs"][:npairs], non_blocking=True)
-                    nbytes += npairs * 8
+                dqkv[b].copy_(host_qkv[k % n_distinct], non_blocking=True)
+                mlen = pairs_off + npairs * 8 if npairs else pairs_off
+                dmeta[b][:mlen].copy_(stage_buf[b][:mlen], non_blocking=True)
+                nbytes = data_bytes + npairs * 8
+                pairs = d["pairs"][:npairs] if npairs else None
                 ev_in[b].record(s_in)
             stream.wait_event(ev_in[b])
             if k - k0 >= 2:
