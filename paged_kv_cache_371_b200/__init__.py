@@ -306,9 +306,9 @@ def _attention(q, k_pool, v_pool, block_tables, context_lens, scale, q_len, out,
     _need(out, "out", torch.float16, dev)
     if out.shape != q.shape:
         raise ValueError("out must have q's shape")
-    need = workspace_size(Hq, Hkv, q_len, D, grid_ctas)
-    if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace is None:  # (a caller's workspace is size-checked by the library)
+        workspace = torch.empty(workspace_size(Hq, Hkv, q_len, D, grid_ctas), dtype=torch.uint8,
+                                device=dev)
     _need(workspace, "workspace", torch.uint8, dev)
     mb = block_tables.shape[1]
     args = (q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_tables.data_ptr(), mb,
