@@ -211,7 +211,7 @@ def test_head_pairs(Hkv, grid, min_split, bs, int8_k):
     row tile's keys, values, scales or queries from the other head of the
     pair moves the outputs far from the oracle's."""
     from planted import plant
-    lens = np.array([1, 7, 8, 9, 64, 65, 333, 1500], np.int32)
+    lens = np.array([0, 1, 7, 8, 9, 64, 65, 333, 1500], np.int32)
     wl = make_workload("llama70b_gqa", "cuda", lens=lens, bs=bs, q_len=1, Hq=8 * Hkv, Hkv=Hkv, D=128,
                        seed=90 + Hkv + bs)
     plan = {s: [(int(L) // 3, 60.0), (int(L) - 1, 120.0)] for s, L in enumerate(lens) if L > 3}
@@ -231,6 +231,7 @@ def test_head_pairs(Hkv, grid, min_split, bs, int8_k):
         torch.cuda.synchronize()
         ref = oracle_subset(wl, list(range(wl.B)))
     assert_close(out, ref, f"head pairs bs{bs} Hkv{Hkv} grid{grid} int8 {int8_k}")
+    assert not out[0].any()  # an empty context gives zeros
 
 
 @pytest.mark.parametrize("name,B", [("llama70b_gqa", 64), ("llama7b_mha", 32)])
