@@ -82,9 +82,29 @@ struct Params {
     const float* k_scale;  // [Hkv][D] channel scales of an int8 K pool (else null)
     int32_t max_blocks, B, q_len, Hq, Hkv, G, rows, num_blocks, min_share;
     int32_t seg_cost;  // virtual blocks charged per (sequence, kv-head) segment
+    // head pairs (Hkv above counts pairs): query rows per head; padded rows
+    // 8h .. 8h + pr - 1 belong to head h of the pair.  0: one head per unit.
+    int32_t pr;
     float scale_log2;
     uint64_t slot_wait_ns;  // limit of the producer's waits for a free ring slot
 };
+
+// Query head and window position j of padded row R of KV head (or head pair)
+// kvh; -1 for a padding row.  Row r of a head is window position r / G,
+// query head g = r % G of the head's group.
+__device__ __forceinline__ int row_head(const Params& p, int kvh, int R, int& j)
+{
+    int r = R, h0 = kvh;
+    if (p.pr) {
+        r = R & 7;
+        h0 = 2 * kvh + (R >> 3);
+        if (r >= p.pr) return -1;
+    } else if (R >= p.rows) {
+        return -1;
+    }
+    j = r / p.G;
+    return h0 * p.G + r % p.G;
+}
 
 template <int D_, int BS_, int MT_, bool FMA_, bool KQ_ = false, int NR8_ = 0, int TW_ = 0,
           int SUBS_ = 1, int UMR_ = 0, int HP_ = 1>
@@ -570,7 +590,7 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
                 const unsigned lmask = __ballot_sync(0xffffffffu, load);
                 if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, KV_DEV_BAD_BLOCK);
                 const bool firstst = (d.flags & F_FIRST) != 0;
-                const uint32_t qbytes = (uint32_t)(p.G * C::D * 2);  // query bytes per window row
+                const uint32_t qbytes = (uint32_t)(p.G * C::D * 2) * (p.pr ? 2u : 1u);  // per window row
                 uint32_t bytes = (uint32_t)__popc(lmask) * (uint32_t)(C::K_TILE_BYTES + C::TILE_BYTES);
                 if (firstst) bytes += qbytes * (uint32_t)p.q_len + (C::KQ ? C::HP * C::D * 4 : 0);
                 const uint32_t full = full0 + stage * 8;
@@ -610,10 +630,10 @@ __device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const P
                                              full, pol);
                     }
                 }
-                if (firstst && lane < p.rows) {  // row R = j*G + g of the segment's queries
-                    const int j = lane / p.G, g = lane % p.G;
-                    const __half* src =
-                        p.q + (((int64_t)d.s * p.q_len + j) * p.Hq + (int64_t)d.kvh * p.G + g) * C::D;
+                int qj = 0;
+                const int qh = (firstst && lane < p.rows) ? row_head(p, d.kvh, lane, qj) : -1;
+                if (qh >= 0) {  // padded row `lane` of the segment's queries
+                    const __half* src = p.q + (((int64_t)d.s * p.q_len + qj) * p.Hq + qh) * C::D;
                     bulk_load(st + C::Q_OFF + lane * C::QROW, src, C::D * 2, full);
                 }
                 if (C::KQ && firstst && lane == 31)  // the KV head's (pair's) channel scales
@@ -747,13 +767,15 @@ __device__ void store_segment_slices(const Params& p, const StageMeta& md, const
             b = make_float4(b.x + y.x, b.y + y.y, b.z + y.z, b.w + y.w);
         }
         if (whole) {
-            const int j = R / p.G, g = R % p.G;
+            int j = 0;
+            const int qh = row_head(p, md.kvh, R, j);
+            if (qh < 0) continue;
             uint4 v;
             v.x = pack_half2(a.x, a.y);
             v.y = pack_half2(a.z, a.w);
             v.z = pack_half2(b.x, b.y);
             v.w = pack_half2(b.z, b.w);
-            __half* dst = p.out + (((int64_t)md.s * p.q_len + j) * p.Hq + (int64_t)md.kvh * p.G + g) * C::D + d0;
+            __half* dst = p.out + (((int64_t)md.s * p.q_len + j) * p.Hq + qh) * C::D + d0;
             *reinterpret_cast<uint4*>(dst) = v;
         } else {
             float4* dst = reinterpret_cast<float4*>(p.part_o + (pbase + R) * C::D + d0);
@@ -1403,7 +1425,8 @@ __device__ void consumer_tc(const Params& p, uint8_t* smem, volatile int* abort_
                     const int R = nt * 8 + 2 * tig + i;
                     m[nt][i] = kNegInf;
                     l[nt][i] = 0.f;
-                    lim[nt][i] = R < p.rows ? md.L - p.q_len + R / p.G + 1 : md.L;
+                    int j = 0;
+                    lim[nt][i] = row_head(p, md.kvh, R, j) >= 0 ? md.L - p.q_len + j + 1 : md.L;
                 }
         }
 #pragma unroll 1
@@ -2107,7 +2130,7 @@ __global__ void __maxnreg__(C::MAXREG)
     }
     // zero the padded query rows of every stage and the zero row
     if constexpr (!C::FMA) {
-        const int used = p.rows * C::QROW;
+        const int used = p.pr ? 0 : p.rows * C::QROW;  // head pairs: padding rows inside
         for (int st = 0; st < C::STAGES; ++st) {
             uint8_t* qa = smem + st * C::STAGE_BYTES + C::Q_OFF;
             for (int i = used + threadIdx.x * 16; i < C::RP * C::QROW; i += C::THREADS * 16)
@@ -2176,6 +2199,9 @@ __global__ void __launch_bounds__(512) lse_merge_kernel(const Params p)
     const int s = md.x, kvh = md.y, a = md.z, slot_a = md.w;
     const int R = idx / (D / 8);
     const int d0 = (idx % (D / 8)) * 8;
+    int j = 0;
+    const int qh = row_head(p, kvh, R, j);
+    if (qh < 0) return;  // a padding row
     float M = kNegInf, W = 0.f;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int i = a; i <= c; i += 2) {
@@ -2199,13 +2225,12 @@ __global__ void __launch_bounds__(512) lse_merge_kernel(const Params p)
         M = mn;
     }
     const float inv = W > 0.f ? 1.f / W : 0.f;
-    const int j = R / p.G, g = R % p.G;
     uint4 v;
     v.x = pack_half2(acc[0] * inv, acc[1] * inv);
     v.y = pack_half2(acc[2] * inv, acc[3] * inv);
     v.z = pack_half2(acc[4] * inv, acc[5] * inv);
     v.w = pack_half2(acc[6] * inv, acc[7] * inv);
-    __half* dst = p.out + (((int64_t)s * p.q_len + j) * p.Hq + (int64_t)kvh * p.G + g) * D + d0;
+    __half* dst = p.out + (((int64_t)s * p.q_len + j) * p.Hq + qh) * D + d0;
     *reinterpret_cast<uint4*>(dst) = v;
 }
 
@@ -2428,12 +2453,27 @@ bool default_tcgen05(int, bool) { return false; }
 // Head pairs: for 8-token blocks (one block of one head is a 2 KB fp16 copy,
 // 1 KB of int8 codes; the pair's copies are twice that, half the copies per
 // byte) and for int8 keys over 16-token blocks (2 KB of codes), head_dim 128,
-// GQA groups of exactly 8 (one row tile per head), decode (one query), the
-// warp-level consumer.  Measured: fp16 over 16-token blocks (4 KB copies)
+// decode (one query), the warp-level consumer; GQA groups of 8 (a row tile
+// per head), and over int8 keys also groups of 1, 2 or 4 (a row tile per
+// head, partly padding).  Measured: fp16 over 16-token blocks (4 KB copies)
 // gains nothing from pairs.
+bool pairs_possible(int D, int G, int q_len, int Hkv)
+{
+    return D == 128 && q_len == 1 && Hkv % 2 == 0 && (G == 1 || G == 2 || G == 4 || G == 8);
+}
+
 bool use_head_pairs(int D, int BS, int G, int q_len, int Hkv, bool int8_k, bool um)
 {
-    return D == 128 && (BS == 8 || int8_k) && G == 8 && q_len == 1 && Hkv % 2 == 0 && !um;
+    if (um || !pairs_possible(D, G, q_len, Hkv)) return false;
+    return int8_k || (G == 8 && BS == 8);
+}
+
+// Padded query rows of the split partials a launch of this shape may use
+// (head pairs take two 8-row tiles whatever the group size).
+int rows_padded_for(int G, int q_len, int Hkv, int D)
+{
+    const int rp = rows_padded(G * q_len);
+    return pairs_possible(D, G, q_len, Hkv) && rp < 16 ? 16 : rp;
 }
 
 int attention_impl(const void* q, const void* k_pool, const void* v_pool,
@@ -2467,22 +2507,20 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
     const int sms = device_sms();
     int grid = sms;
     if (opts && opts->grid_ctas > 0) grid = opts->grid_ctas;
-    const int rp = rows_padded(rows);
-    if (ws_bytes < workspace_bytes_for(grid, rp, D))
-        return kv_fail(KV_ERR_INVALID, "paged attention: workspace too small");
-    int* err = kv_error_word_ptr();
-    if (!err) return kv_fail(KV_ERR_CUDA, "paged attention: no device error word");
-
     // consumer for several query rows per KV head at head_dim 128: tcgen05
     // (tensor memory) or warp-level MMAs
     const int consumer = opts ? opts->consumer : 0;
     if (consumer < 0 || consumer > 2)
         return kv_fail(KV_ERR_INVALID, "paged attention: opts.consumer must be 0, 1 or 2");
     const bool um = D == 128 && rows > 1 && (consumer == 2 || (consumer == 0 && default_tcgen05(rows, k_scale != nullptr)));
-    // head pairs (8-token blocks, GQA groups of 8, one query per sequence):
-    // the kernel sees Hkv / 2 heads of 2 * G query rows, each staged tile
-    // both heads' rows of a block (see Cfg::HP)
+    // head pairs: the kernel sees Hkv / 2 units of two heads, rows 8h.. of
+    // head h, each staged tile both heads' rows of a block (see Cfg::HP)
     const bool hp = use_head_pairs(D, BS, G, q_len, Hkv, k_scale != nullptr, um);
+    const int rp = hp ? 16 : rows_padded(rows);
+    if (ws_bytes < workspace_bytes_for(grid, rp, D))
+        return kv_fail(KV_ERR_INVALID, "paged attention: workspace too small");
+    int* err = kv_error_word_ptr();
+    if (!err) return kv_fail(KV_ERR_CUDA, "paged attention: no device error word");
     CUtensorMap tk, tv;
     const uint64_t prow = (uint64_t)num_blocks * Hkv * BS;
     const int trows = hp ? 2 * BS : BS;  // pool rows per staged tile
@@ -2509,8 +2547,9 @@ int attention_impl(const void* q, const void* k_pool, const void* v_pool,
     prm.q_len = q_len;
     prm.Hq = Hq;
     prm.Hkv = hp ? Hkv / 2 : Hkv;
-    prm.G = hp ? 2 * G : G;
-    prm.rows = hp ? 2 * rows : rows;
+    prm.G = G;
+    prm.rows = hp ? 16 : rows;
+    prm.pr = hp ? rows : 0;
     prm.num_blocks = num_blocks;
     prm.min_share = (opts && opts->min_split_blocks > 0) ? opts->min_split_blocks : 16;
     prm.seg_cost = (opts && opts->seg_cost_blocks != 0) ? (opts->seg_cost_blocks > 0 ? opts->seg_cost_blocks : 0)
@@ -2550,7 +2589,7 @@ int paged_attention_workspace_size(int32_t Hq, int32_t Hkv, int32_t q_len, int32
     if (rows > 16 * kMaxMT)
         return kv_fail(KV_ERR_INVALID, "paged_attention_workspace_size: rows must be <= 32");
     const int grid = grid_ctas > 0 ? grid_ctas : device_sms();
-    *bytes_out = workspace_bytes_for(grid, rows_padded(rows), head_dim);
+    *bytes_out = workspace_bytes_for(grid, rows_padded_for(Hq / Hkv, q_len, Hkv, head_dim), head_dim);
     return KV_OK;
 }
 
@@ -2675,7 +2714,7 @@ extern "C" int paged_decode_attention_static_ws(const void* q, const void* k_poo
     const int rows = Hq / Hkv;
     if (rows > 16 * kMaxMT)
         return kv_fail(KV_ERR_INVALID, "paged_decode_attention_static_ws: Hq/Hkv must be <= 32");
-    const size_t need = workspace_bytes_for(device_sms(), rows_padded(rows), head_dim);
+    const size_t need = workspace_bytes_for(device_sms(), rows_padded_for(rows, 1, Hkv, head_dim), head_dim);
     if (need > kStaticScratchBytes)
         return kv_fail(KV_ERR_INVALID,
                        "paged_decode_attention_static_ws: this shape needs more scratch than the "

@@ -199,21 +199,22 @@ def test_tiny_config_full_with_append():
     assert_close(out2, ref2, "tiny after append")
 
 
-@pytest.mark.parametrize("bs,int8_k", [(8, False), (8, True), (16, True)])
+@pytest.mark.parametrize("bs,int8_k,G", [(8, False, 8), (8, True, 8), (16, True, 8), (16, True, 1),
+                                          (8, True, 1), (16, True, 4)])
 @pytest.mark.parametrize("Hkv", [2, 8])
 @pytest.mark.parametrize("grid,min_split", [(0, 0), (300, 1), (7, 1)])
-def test_head_pairs(Hkv, grid, min_split, bs, int8_k):
-    """8-token blocks, or int8 keys over 16-token blocks, GQA groups of 8,
-    one query per sequence: each staged tile holds two adjacent KV heads of a
-    block (one copy), and row tile h reads head h's rows (and, over int8
-    keys, head h's channel scales).  Each
+def test_head_pairs(Hkv, grid, min_split, bs, int8_k, G):
+    """8-token blocks with GQA groups of 8, or int8 keys with groups of 8, 4
+    or 1 (MHA), one query per sequence: each staged tile holds two adjacent
+    KV heads of a block (one copy), and row tile h (padded rows 8h ..)
+    reads head h's rows (and, over int8 keys, head h's channel scales).  Each
     head's queries and planted keys follow their own direction, so taking a
     row tile's keys, values, scales or queries from the other head of the
     pair moves the outputs far from the oracle's."""
     from planted import plant
     lens = np.array([0, 1, 7, 8, 9, 64, 65, 333, 1500], np.int32)
-    wl = make_workload("llama70b_gqa", "cuda", lens=lens, bs=bs, q_len=1, Hq=8 * Hkv, Hkv=Hkv, D=128,
-                       seed=90 + Hkv + bs)
+    wl = make_workload("llama70b_gqa", "cuda", lens=lens, bs=bs, q_len=1, Hq=G * Hkv, Hkv=Hkv, D=128,
+                       seed=90 + Hkv + bs + G)
     plan = {s: [(int(L) // 3, 60.0), (int(L) - 1, 120.0)] for s, L in enumerate(lens) if L > 3}
     plant(wl, plan, seed=13 + Hkv)
     if int8_k:
@@ -230,7 +231,7 @@ def test_head_pairs(Hkv, grid, min_split, bs, int8_k):
         out = _run(wl, 1, grid_ctas=grid, min_split_blocks=min_split)
         torch.cuda.synchronize()
         ref = oracle_subset(wl, list(range(wl.B)))
-    assert_close(out, ref, f"head pairs bs{bs} Hkv{Hkv} grid{grid} int8 {int8_k}")
+    assert_close(out, ref, f"head pairs bs{bs} G{G} Hkv{Hkv} grid{grid} int8 {int8_k}")
     assert not out[0].any()  # an empty context gives zeros
 
 
