@@ -262,10 +262,12 @@ int paged_kv_swap_in(void* k_pool, void* v_pool, const int32_t* block_ids, int32
                      int32_t num_blocks, void* stream);
 
 /* Bytes of device workspace paged_decode_attention / paged_verify_attention
- * need for these head counts on the current device (partial results of
- * context splits).  grid_ctas: 0 for the default launch, else the value given
- * in paged_attention_opts.grid_ctas.  The workspace holds no state between
- * calls and needs no initialisation. */
+ * (and the int8-K entries) need for these head counts on the current device
+ * (partial results of context splits; a shape the kernel may serve as pairs
+ * of KV heads, two 8-row tiles, is sized for that form whatever the block
+ * size or pool type).  grid_ctas: 0 for the default launch, else the value
+ * given in paged_attention_opts.grid_ctas.  The workspace holds no state
+ * between calls and needs no initialisation. */
 int paged_attention_workspace_size(int32_t Hq, int32_t Hkv, int32_t q_len, int32_t head_dim,
                                    int32_t grid_ctas, size_t* bytes_out);
 

@@ -125,8 +125,8 @@ struct Cfg {
     static_assert(!KQ || D == 128, "int8 K pools are served at head_dim 128");
     // HP = 2: a unit of work is a pair of adjacent KV heads of a block, staged
     // by one copy of both heads' rows (they are contiguous in the pool): half
-    // the copies per byte, for 8-token blocks.  Row tile h holds the 8 query
-    // rows of head h of the pair (GQA groups of 8, one query per sequence).
+    // the copies per byte.  Row tile h holds the query rows of head h of the
+    // pair (padded rows 8h .., at most 8 per head; see row_head).
     static constexpr int HP = HP_;
     static_assert(HP == 1 || (HP == 2 && NR8_ == 2 && !UMR && D == 128),
                   "head pairs: two row tiles of one head each, head_dim 128");
