@@ -138,3 +138,29 @@ def test_batch_reserve_matches_sequential_spec():
         for s in range(B):
             assert tables[s, :nblk[s]].tolist() == spec_tables[s]
         lens = lens + 1
+
+
+def test_workspace_size_covers_the_head_pair_form():
+    """The split partials are [grid][2][rows][head_dim] fp32 plus one log-sum
+    per row and 16 bytes of metadata per CTA.  A shape the kernel may serve as
+    pairs of KV heads (head_dim 128, one query, an even number of KV heads,
+    groups of 1, 2, 4 or 8) is sized for two 8-row tiles, 16 rows, whatever
+    its group size; others for their rows padded to 16 (1 for one row)."""
+    grid = 148
+
+    def expect(rp, D):
+        lse = (grid * 2 * rp * 4 + 15) // 16 * 16
+        return grid * 16 + lse + grid * 2 * rp * D * 4
+
+    cases = [  # (Hq, Hkv, q_len, D, padded rows)
+        (32, 32, 1, 128, 16),   # MHA, head_dim 128: pairs possible
+        (32, 32, 1, 64, 1),     # MHA, head_dim 64: one row
+        (31, 31, 1, 128, 1),    # odd KV heads: no pairs
+        (32, 8, 1, 128, 16),    # GQA 4
+        (64, 8, 1, 128, 16),    # GQA 8
+        (32, 8, 5, 128, 32),    # 5-token verify window, 20 rows
+        (32, 1, 1, 128, 32),    # MQA, 32 rows
+        (16, 16, 3, 128, 16),   # MHA verify window of 3 rows
+    ]
+    for Hq, Hkv, q_len, D, rp in cases:
+        assert pkv.workspace_size(Hq, Hkv, q_len, D, grid) == expect(rp, D), (Hq, Hkv, q_len, D)
